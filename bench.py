@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark: dual-stream Gated DeltaNet forward on B200, tokens/s (clean + noisy tokens).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Each rank runs its own replica of the workload
+(documents are independent units, so ranks share nothing on the data path: weak scaling).
+Rank 0 prints ONE JSON line.  A step is one gdn_dual_forward call (both streams, all
+documents and heads) on inputs already resident in HBM; `e2e` repeats the measurement
+through the public Python API with pinned-host inputs copied in and outputs copied back
+inside the timed region.  `--impl reference` times the fp64 CPU oracle on the host cores
+(a bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_dual_b200 import binding as gb  # noqa: E402
+from gated_deltanet_dual_b200 import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "train_8x4096_h16_d128"
+METRIC = "dual-stream GDN fwd tokens/s on 1 B200 and % of roofline (HBM/tensor)"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = {
+    gb.ALGO_SEQUENTIAL: ["gated_deltanet_dual_b200/csrc/gdn_sequential.cu"],
+    gb.ALGO_CHUNKED: ["gated_deltanet_dual_b200/csrc/gdn_chunked.cu"],
+}
+KERNEL_NAMES = {gb.ALGO_SEQUENTIAL: "gdn_sequential_kernel", gb.ALGO_CHUNKED: "gdn_chunked_kernel"}
+
+
+# ----------------------------------------------------------------------------- work model
+def algorithmic_work(prob) -> dict:
+    """Algorithmic bytes and FLOPs of one forward (what must move / be computed at minimum):
+    per (stream-token, head) read q, k, v and g, beta, write o; plus the fp32 final state per
+    (doc, head) and the conv weights.  FLOPs: k^T S, the rank-1 update and S^T q = 6 d_k d_v
+    per (stream-token, head), plus 2 W FLOPs per conv'd channel."""
+    s = prob.q.element_size()
+    H, dk, dv = prob.num_heads, prob.d_k, prob.d_v
+    toks = prob.tokens()
+    per_tok_head = (2 * dk + dv) * s + 8 + dv * s
+    nbytes = toks * H * per_tok_head + prob.num_docs * H * dk * dv * 4
+    flops = toks * H * 6 * dk * dv
+    if prob.conv_width:
+        nbytes += 3 * H * dk * prob.conv_width * 4
+        flops += toks * H * (2 * dk + dv) * 2 * prob.conv_width
+    return {"bytes": int(nbytes), "flops": int(flops), "bytes_per_token_head": per_tok_head}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_hash(algo) -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES.get(algo, []) + ["gated_deltanet_dual_b200/csrc/gdn_internal.cuh"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(algo, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel source (same hash) for this workload; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        rec = json.load(open(path)).get(f"{KERNEL_NAMES[algo]}:{workload}")
+    except Exception:
+        return None
+    if not rec or rec.get("kernel_hash") != kernel_hash(algo):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.gpu)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def oracle_sample_problem(wl, max_units: int, seed: int = 0):
+    """A bounded sample of the workload for the CPU oracle: its first documents (all heads),
+    generated on the host with the same distributions."""
+    offs, prompts = synth.doc_layout(wl, seed)
+    H = wl.num_heads
+    ndocs = max(1, min(len(prompts), max_units // H))
+    sub_offs = offs[:ndocs + 1] - offs[0]
+    prob = synth.make_problem_from_layout(sub_offs, prompts[:ndocs], num_heads=H, d_k=wl.d, d_v=wl.d,
+                                          block_size=wl.block_size, num_views=wl.num_views, dtype=wl.dtype,
+                                          g_lo=wl.g_lo, beta_std=wl.beta_std, conv_width=wl.conv_width,
+                                          conv_std=wl.conv_std, seed=seed, device="cpu")
+    return prob, ndocs
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def time_oracle(wl, steps: int, warmup: int, max_units: int):
+    import oracle  # test infrastructure: the CPU baseline / reference arm only
+    prob, ndocs = oracle_sample_problem(wl, max_units)
+    threads = min(host_cores(), prob.num_docs * prob.num_heads)
+    for _ in range(warmup):
+        oracle.forward_problem(prob, num_threads=threads)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.forward_problem(prob, num_threads=threads)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    return {"value": prob.tokens() * steps / tot, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{ndocs} of the workload's documents x all {wl.num_heads} heads "
+                      f"({prob.tokens()} clean+noisy tokens), fp64, host-generated with the same distributions",
+            "seconds_per_step": tot / steps}
+
+
+def units_for_seconds(wl, target_s: float) -> int:
+    """Units (doc, head) the oracle finishes in about target_s on this host (one probe unit)."""
+    import oracle
+    probe = synth.make_problem_from_layout([0, 512], [128], num_heads=1, d_k=wl.d, d_v=wl.d,
+                                           block_size=wl.block_size, num_views=wl.num_views, dtype=wl.dtype,
+                                           conv_width=wl.conv_width, device="cpu")
+    t0 = time.perf_counter()
+    oracle.forward_problem(probe, num_threads=1)
+    per_token = (time.perf_counter() - t0) / probe.tokens()
+    offs, prompts = synth.doc_layout(wl, 0)
+    lens = np.diff(offs)
+    unit_tokens = float(np.mean(lens + wl.num_views * (lens - prompts)))
+    per_unit = per_token * unit_tokens
+    return max(wl.num_heads, int(target_s * host_cores() / max(per_unit, 1e-9)))
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    max_units = units_for_seconds(wl, target_s=min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    cb = time_oracle(wl, args.steps, args.warmup, max_units)
+    line = {"metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["seconds_per_step"] * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "parallelism": "replicas", "l2": "not applicable (host)"},
+            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--algo", default="auto", choices=["auto", "sequential", "chunked"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    wl = synth.get_workload(args.workload)
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+
+    import torch.distributed as dist
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    algo = {"auto": gb.ALGO_AUTO, "sequential": gb.ALGO_SEQUENTIAL, "chunked": gb.ALGO_CHUNKED}[args.algo]
+
+    prob = synth.make_problem(wl, seed=rank, device=dev)
+    T, TR, V, H, d = prob.T, prob.T_R, prob.num_views, prob.num_heads, prob.d_k
+    desc = gb.make_desc(prob.num_docs, H, d, d, V, prob.block_size, gb._dtype_code(prob.q), prob.conv_width, algo)
+    used_algo = gb.select_algo(desc)
+    ws = gb.Workspace(gb.workspace_size(desc, prob.doc_offsets), device=dev)
+    out = torch.empty(T, H, d, dtype=prob.q.dtype, device=dev)
+    out_n = torch.empty(V, TR, H, d, dtype=prob.q.dtype, device=dev)
+    fs = torch.empty(prob.num_docs, H, d, d, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gb.forward_problem(prob, algo=algo, out=out, out_noisy=out_n, final_state=fs, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dstatus = gb.read_device_status(ws)
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop))
+    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    kernel_ms = max_over_ranks(sum(launch_ms) / len(launch_ms))
+
+    work = algorithmic_work(prob)
+    toks_all = prob.tokens() * world
+    value = toks_all * args.steps / (elapsed_ms / 1e3)
+    peaks = measured_peaks()
+    achieved_gbs = work["bytes"] / (kernel_ms / 1e3) / 1e9
+    traffic = profiled_traffic(used_algo, wl.name)
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": peaks["source"], "kernel": KERNEL_NAMES.get(used_algo),
+                "algorithmic_bytes_per_launch": work["bytes"], "algorithmic_flops_per_launch": work["flops"],
+                "tensor_frac_at_algorithmic_flops": work["flops"] / (kernel_ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
+
+    # ---- end to end through the public API: pinned host inputs in, outputs back ----
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k", "v", "g", "beta", "qn", "kn", "vn", "gn", "betan"] + (["conv_w"] if prob.conv_w is not None else [])
+        host = {n: getattr(prob, n).cpu().pin_memory() for n in names}
+        dbuf = {n: torch.empty_like(getattr(prob, n)) for n in names}
+        h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h_outn = torch.empty(out_n.shape, dtype=out_n.dtype, pin_memory=True)
+        h_fs = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in (h_out, h_outn, h_fs))
+
+        def e2e_step():
+            for n in names:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            gb.forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["qn"], dbuf["kn"], dbuf["vn"],
+                       dbuf["gn"], dbuf["betan"], prob.doc_offsets, prob.prompt_len, prob.block_size,
+                       conv_w=dbuf.get("conv_w"), algo=algo, out=out, out_noisy=out_n, final_state=fs, workspace=ws)
+            h_out.copy_(out, non_blocking=True)
+            h_outn.copy_(out_n, non_blocking=True)
+            h_fs.copy_(fs, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 10))
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        z.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(z)) / e2e_steps
+        e2e = {"value": toks_all / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms, "steps": e2e_steps}
+        del host, dbuf
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        max_units = units_for_seconds(wl, target_s=10.0)
+        cb = time_oracle(wl, steps=1, warmup=0, max_units=max_units)
+        cpu_baseline = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if prob.q.dtype == torch.bfloat16 else "fp32",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "docs": prob.num_docs, "tokens_clean": T, "tokens_noisy": V * TR,
+                       "heads": H, "d": d, "block_size": prob.block_size, "views": V, "conv_width": prob.conv_width,
+                       "algo": {1: "sequential", 2: "chunked"}.get(used_algo, str(used_algo)),
+                       "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush)"},
+            "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clocks.summary(),
+            "device_status": gb.status_string(dstatus), "kernel_ms_mean": kernel_ms}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

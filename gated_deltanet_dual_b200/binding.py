@@ -1,0 +1,202 @@
+"""Thin ctypes binding of libgdn_dual.so (the C ABI in include/gdn_dual.h).
+
+Argument marshalling only: every step of the forward runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream.  There is no fallback: if the
+library is missing or cannot load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdn_dual.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_ALIGNMENT, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
+GDN_BF16, GDN_FP32 = 0, 1
+ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED = 0, 1, 2
+EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device_status",
+            "gdn_status_string", "gdn_dual_version", "gdn_dual_select_algo")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("num_docs", "num_heads", "d_k", "d_v", "num_views",
+                                               "block_size", "dtype", "conv_width", "algo", "reserved")]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the CUDA library (raises OSError if it is missing; nothing falls back)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise OSError(f"{path} not found: build it with `python -m gated_deltanet_dual_b200.build`")
+            lib = ctypes.CDLL(path)
+            vp, fp, ip = ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32)
+            lib.gdn_dual_forward.restype = ctypes.c_int
+            lib.gdn_dual_forward.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                             ip, ip, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+            lib.gdn_dual_workspace_size.restype = ctypes.c_size_t
+            lib.gdn_dual_workspace_size.argtypes = [ctypes.POINTER(Desc), ip]
+            lib.gdn_dual_read_device_status.restype = ctypes.c_int
+            lib.gdn_dual_read_device_status.argtypes = [vp, vp]
+            lib.gdn_status_string.restype = ctypes.c_char_p
+            lib.gdn_status_string.argtypes = [ctypes.c_int]
+            lib.gdn_dual_version.restype = ctypes.c_int32
+            lib.gdn_dual_select_algo.restype = ctypes.c_int32
+            lib.gdn_dual_select_algo.argtypes = [ctypes.POINTER(Desc)]
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load_library().gdn_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_FP32
+    raise TypeError(f"unsupported I/O dtype {t.dtype}")
+
+
+def make_desc(num_docs, num_heads, d_k, d_v, num_views, block_size, dtype_code, conv_width=0, algo=ALGO_AUTO):
+    return Desc(num_docs, num_heads, d_k, d_v, num_views, block_size, dtype_code, conv_width, algo, 0)
+
+
+def _host_i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def workspace_size(desc: Desc, doc_offsets) -> int:
+    offs = _host_i32(doc_offsets)
+    return int(load_library().gdn_dual_workspace_size(ctypes.byref(desc),
+                                                      offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))))
+
+
+def select_algo(desc: Desc) -> int:
+    return int(load_library().gdn_dual_select_algo(ctypes.byref(desc)))
+
+
+def forward_raw(desc: Desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, conv_w,
+                out, out_noisy, final_state, workspace, stream=None) -> int:
+    """Direct C-ABI call with tensors (or None) for every pointer; returns the status code."""
+    lib = load_library()
+    offs = _host_i32(doc_offsets)
+    pl = _host_i32(prompt_len)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else 0
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return int(lib.gdn_dual_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                    _ptr(qn), _ptr(kn), _ptr(vn), _ptr(gn), _ptr(betan),
+                                    offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(conv_w),
+                                    _ptr(out), _ptr(out_noisy), _ptr(final_state),
+                                    _ptr(workspace), ctypes.c_size_t(ws_bytes), ctypes.c_void_p(stream)))
+
+
+class Workspace:
+    """Caller-owned device scratch for gdn_dual_forward (allocated by torch, reused)."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        self.tensor = torch.zeros(max(256, (nbytes + 255) // 256 * 256), dtype=torch.uint8, device=device)
+
+
+def _check(t: Optional[torch.Tensor], name: str, shape, dtype, device):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype} != {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def forward(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, block_size,
+            conv_w=None, *, algo: int = ALGO_AUTO, out=None, out_noisy=None, final_state=None,
+            workspace: Optional[Workspace] = None, stream=None):
+    """Dual-stream Gated DeltaNet forward on the GPU.
+
+    Shapes: q, k [T,H,d]; v [T,H,d]; g, beta [T,H] fp32; qn, kn, vn [V,T_R,H,d]; gn, betan
+    [V,T_R,H] fp32; conv_w [3,H*d,4] fp32 or None; doc_offsets [N+1], prompt_len [N] host ints.
+    Returns (out [T,H,d], out_noisy [V,T_R,H,d], final_state [N,H,d,d] fp32)."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    V, TR = qn.shape[0], qn.shape[1]
+    offs = _host_i32(doc_offsets)
+    pl = _host_i32(prompt_len)
+    N = offs.shape[0] - 1
+    io = q.dtype
+    f32 = torch.float32
+    if offs.ndim != 1 or pl.shape != (N,):
+        raise ValueError("doc_offsets must be [N+1] and prompt_len [N]")
+    if N >= 1 and int(offs[-1]) != T:
+        raise ValueError(f"doc_offsets[-1] = {int(offs[-1])} but q has {T} tokens")
+    if N >= 1 and int((np.diff(offs.astype(np.int64)) - pl).sum()) != TR:
+        raise ValueError(f"noisy tensors have {TR} rows but the documents have "
+                         f"{int((np.diff(offs.astype(np.int64)) - pl).sum())} response tokens")
+    for t, name, shape, dt in ((q, "q", (T, H, dk), io), (k, "k", (T, H, dk), io), (v, "v", (T, H, dv), io),
+                               (g, "g", (T, H), f32), (beta, "beta", (T, H), f32),
+                               (qn, "qn", (V, TR, H, dk), io), (kn, "kn", (V, TR, H, dk), io),
+                               (vn, "vn", (V, TR, H, dv), io), (gn, "gn", (V, TR, H), f32),
+                               (betan, "betan", (V, TR, H), f32)):
+        _check(t, name, shape, dt, dev)
+    conv_width = 0
+    if conv_w is not None:
+        conv_width = int(conv_w.shape[-1])
+        _check(conv_w, "conv_w", (3, H * dk, conv_width), f32, dev)
+    if out is None:
+        out = torch.empty(T, H, dv, dtype=io, device=dev)
+    if out_noisy is None:
+        out_noisy = torch.empty(V, TR, H, dv, dtype=io, device=dev)
+    if final_state is None:
+        final_state = torch.empty(N, H, dk, dv, dtype=f32, device=dev)
+    _check(out, "out", (T, H, dv), io, dev)
+    _check(out_noisy, "out_noisy", (V, TR, H, dv), io, dev)
+    _check(final_state, "final_state", (N, H, dk, dv), f32, dev)
+    desc = make_desc(N, H, dk, dv, V, int(block_size), _dtype_code(q), conv_width, algo)
+    if workspace is None:
+        workspace = Workspace(workspace_size(desc, offs), device=dev)
+    st = forward_raw(desc, q, k, v, g, beta, qn, kn, vn, gn, betan, offs, pl, conv_w,
+                     out, out_noisy, final_state, workspace.tensor, stream=stream)
+    if st != GDN_OK:
+        raise GdnError(st, f"gdn_dual_forward failed: {status_string(st)}")
+    return out, out_noisy, final_state
+
+
+def read_device_status(workspace: Workspace, stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return int(load_library().gdn_dual_read_device_status(_ptr(workspace.tensor), ctypes.c_void_p(stream)))
+
+
+def forward_problem(prob, **kw):
+    """Run the forward on a synthetic problem whose tensors live on the GPU."""
+    return forward(prob.q, prob.k, prob.v, prob.g, prob.beta, prob.qn, prob.kn, prob.vn, prob.gn,
+                   prob.betan, prob.doc_offsets, prob.prompt_len, prob.block_size, conv_w=prob.conv_w, **kw)

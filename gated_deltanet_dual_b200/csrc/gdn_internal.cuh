@@ -1,0 +1,57 @@
+// gdn_internal.cuh -- parameters shared by the host entry points and the kernels of the
+// dual-stream Gated DeltaNet forward (sm_100a).  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/gdn_dual.h"
+
+namespace gdn {
+
+// Documents are passed to the kernels by value (kernel parameter space), so a launch needs no
+// host-to-device copy and no allocation.  1024 documents keep the parameter block ~16 KB.
+constexpr int kMaxDocs = 1024;
+
+// Device-side status words at the start of the workspace.
+struct WorkspaceHeader {
+    int32_t status;         // GDN_OK or GDN_ERR_TIMEOUT, written by kernels
+    int32_t next_unit;      // dynamic work counter of the persistent kernel
+    int32_t timeout_where;  // diagnostic: which wait gave up
+    int32_t pad[61];        // header is 256 bytes
+};
+static_assert(sizeof(WorkspaceHeader) == 256, "workspace header is 256 bytes");
+
+struct Params {
+    const void *q, *k, *v;
+    const float *g, *beta;
+    const void *qn, *kn, *vn;
+    const float *gn, *betan;
+    const float *conv_w;
+    void *out, *out_noisy;
+    float *final_state;
+    WorkspaceHeader *ws;
+    int64_t T, TR;
+    int32_t N, H, dk, dv, V, B, conv_width, num_units;
+    float scale;                      // 1 / sqrt(d_k)
+    int32_t doc_start[kMaxDocs + 1];  // token offset of each document (doc_offsets)
+    int32_t doc_prompt[kMaxDocs];     // prompt length of each document
+    int32_t resp_off[kMaxDocs + 1];   // first packed noisy row of each document
+    int32_t unit_doc[kMaxDocs];       // documents in scheduling order (longest first)
+};
+
+// Launchers (one per kernel family).  Return a CUDA error code; the caller maps it.
+cudaError_t launch_sequential(const Params &p, int dtype, cudaStream_t stream);
+cudaError_t launch_chunked(const Params &p, cudaStream_t stream);
+bool chunked_supported(int dtype, int d, int B, int conv_width);
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+}  // namespace gdn

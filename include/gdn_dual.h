@@ -1,0 +1,142 @@
+/*
+ * gdn_dual.h -- C ABI of the B200 (sm_100a) dual-stream Gated DeltaNet forward.
+ *
+ * The operation is the forward pass of the two streams described in
+ * "FLARE: Diffusion for Hybrid Language Model" (papernotes.org notes):
+ *
+ *   Method > Key design 2 -- clean causal stream, the gated delta rule
+ *       S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,  alpha_t = exp(g_t),
+ *       o_t = S_t^T q_t / sqrt(d_k)                  (S is d_k x d_v, read after the update);
+ *     and the block-bidirectional noisy stream: for every response block b of B tokens and
+ *     every noisy view, S~ starts from the clean state S_{e(b-1)} just before the block, runs
+ *     the same rule over the block's noisy tokens, and every position of the block reads the
+ *     block-end state: o~_l = S~_{e(b)}^T q~_l / sqrt(d_k).  No per-block state is ever
+ *     written to memory by this library.
+ *   Method > Key design 3 -- optional width-4 depthwise causal ShortConv on q, k, v whose
+ *     noisy taps that reach before the block start read the clean raw input; state reset and
+ *     no tap across packed-document boundaries; document boundaries aligned to B.
+ *   Method > Overall framework -- prompt tokens are causal context only; the response of
+ *     each document is cut into blocks of B tokens; each block has complementary noisy views.
+ *
+ * Tensor layouts (row-major, contiguous, device memory owned by the caller):
+ *   q, k         [T, H, d_k]        dtype = desc->dtype (bf16 or fp32)
+ *   v            [T, H, d_v]
+ *   g, beta      [T, H]             fp32 (g = log alpha, any real; beta any real)
+ *   qn, kn       [V, T_R, H, d_k]   noisy twins, packed over RESPONSE tokens only,
+ *   vn           [V, T_R, H, d_v]   documents in order (row r of doc n = its response token r)
+ *   gn, betan    [V, T_R, H]        fp32
+ *   conv_w       [3, H*d_k, 4]      fp32 weights for q, k, v channels; tap 3 is the current
+ *                                   token: x'_p = sum_j w[c][3-j] x_{p-j}; NULL when conv is off
+ *   out          [T, H, d_v]        dtype = desc->dtype
+ *   out_noisy    [V, T_R, H, d_v]   dtype = desc->dtype
+ *   final_state  [N, H, d_k, d_v]   fp32, the state after each document's last token
+ * where T = doc_offsets[N] and T_R = sum_n (len_n - prompt_len[n]).
+ *
+ * Threading / ownership: the library allocates nothing and keeps no state between calls.
+ * gdn_dual_forward only validates on the host, then enqueues work on `stream` and returns;
+ * results are ready when the stream is.  Calls on different streams that share a workspace
+ * race.  All functions are thread-safe.
+ *
+ * Errors: every entry point returns a gdn_status.  Bad arguments are rejected on the host
+ * before anything is enqueued (no partial writes).  CUDA launch failures return
+ * GDN_ERR_CUDA.  Device code never traps or asserts; bounded waits inside kernels record
+ * GDN_ERR_TIMEOUT in the workspace (see gdn_dual_read_device_status).
+ */
+#ifndef GDN_DUAL_H
+#define GDN_DUAL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* inconsistent sizes, offsets, block alignment, NULL pointer */
+    GDN_ERR_ALIGNMENT = 2,     /* a tensor pointer is not 16-byte aligned */
+    GDN_ERR_UNSUPPORTED = 3,   /* valid but not implemented here (d, dtype, conv width, algo) */
+    GDN_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    GDN_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (reported by the device) */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
+
+typedef enum {
+    GDN_ALGO_AUTO = 0,        /* chunked tensor-core kernel when supported, else sequential */
+    GDN_ALGO_SEQUENTIAL = 1,  /* token-sequential CUDA-core kernel, fp32 state (any dtype) */
+    GDN_ALGO_CHUNKED = 2      /* chunked WY/UT tcgen05 kernel (bf16, d_k = d_v = 128) */
+} gdn_algo;
+
+/* Problem descriptor.  num_docs N >= 1; num_heads H >= 1; d_k == d_v in {32, 64, 128};
+ * num_views V in [0, 8]; block_size B >= 1 (the chunked kernel needs B | 64); dtype a
+ * gdn_dtype; conv_width 0 (off) or 4; algo a gdn_algo; reserved must be 0. */
+typedef struct {
+    int32_t num_docs;
+    int32_t num_heads;
+    int32_t d_k;
+    int32_t d_v;
+    int32_t num_views;
+    int32_t block_size;
+    int32_t dtype;
+    int32_t conv_width;
+    int32_t algo;
+    int32_t reserved;
+} gdn_dual_desc;
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *gdn_stream_t;
+
+/* Bytes of device workspace gdn_dual_forward needs for this problem (>= 256, a multiple of
+ * 256).  doc_offsets_host: HOST array [N+1].  Returns 0 if the descriptor or offsets are
+ * invalid. */
+size_t gdn_dual_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host);
+
+/*
+ * Dual-stream GDN forward (Key design 2 and 3 of the FLARE notes; see the file comment).
+ *   desc                 problem descriptor (host).
+ *   q k v g beta         clean-stream inputs (device), layouts above.
+ *   qn kn vn gn betan    noisy-stream inputs (device); may be NULL when V == 0 or T_R == 0.
+ *   doc_offsets          HOST int32 [N+1]: doc_offsets[0] == 0, non-decreasing.  Document n
+ *                        covers tokens [doc_offsets[n], doc_offsets[n+1]).
+ *   prompt_len           HOST int32 [N]: 0 <= prompt_len[n] <= len_n and
+ *                        (len_n - prompt_len[n]) % B == 0 (response aligned to B).
+ *   conv_w               device fp32 [3, H*d_k, 4], or NULL when desc->conv_width == 0.
+ *   out out_noisy final_state   outputs (device), fully overwritten.
+ *   workspace            device scratch of at least gdn_dual_workspace_size() bytes,
+ *                        16-byte aligned; contents on entry are ignored.
+ *   stream               CUDA stream to enqueue on.
+ * Every device pointer must be 16-byte aligned.
+ */
+gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
+                            const void *q, const void *k, const void *v,
+                            const float *g, const float *beta,
+                            const void *qn, const void *kn, const void *vn,
+                            const float *gn, const float *betan,
+                            const int32_t *doc_offsets, const int32_t *prompt_len,
+                            const float *conv_w,
+                            void *out, void *out_noisy, float *final_state,
+                            void *workspace, size_t workspace_bytes,
+                            gdn_stream_t stream);
+
+/* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
+ * last gdn_dual_forward on it (GDN_OK or GDN_ERR_TIMEOUT), or GDN_ERR_CUDA if the sync fails.
+ * For debugging and tests; the forward path itself never synchronises. */
+gdn_status gdn_dual_read_device_status(const void *workspace, gdn_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *gdn_status_string(gdn_status status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int32_t gdn_dual_version(void);
+
+/* Which algorithm GDN_ALGO_AUTO selects for this descriptor (a gdn_algo value), or -1 if the
+ * descriptor is invalid.  Host only. */
+int32_t gdn_dual_select_algo(const gdn_dual_desc *desc);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_DUAL_H */

@@ -1,0 +1,170 @@
+"""C-ABI library: loads, exports every declared symbol, validates on the host (CPU only).
+
+The error-path cases here pass placeholder addresses that the host validation must reject
+before anything is enqueued; they never run where a GPU is visible."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from gated_deltanet_dual_b200 import binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn_dual.h")
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers: host-only check")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(gdn_[a-z_]+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    assert "gdn_dual_forward" in names and "gdn_dual_workspace_size" in names
+    assert set(b.EXPORTED) <= set(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = b.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/gdn_dual.h but not exported"
+
+
+def test_version_and_status_strings():
+    lib = b.load_library()
+    assert lib.gdn_dual_version() >= 100
+    for code, name in enumerate(["GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_ALIGNMENT", "GDN_ERR_UNSUPPORTED",
+                                 "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT"]):
+        assert b.status_string(code) == name
+    assert b.status_string(99) == "GDN_ERR_UNKNOWN"
+
+
+def test_workspace_size_and_algo_selection():
+    d = b.make_desc(2, 4, 128, 128, 2, 4, b.GDN_BF16)
+    assert b.workspace_size(d, [0, 64, 128]) >= 256
+    assert b.workspace_size(d, [0, 64, 32]) == 0          # non-monotone
+    assert b.workspace_size(d, [1, 64, 128]) == 0         # must start at 0
+    assert b.select_algo(b.make_desc(1, 2, 32, 32, 2, 4, b.GDN_FP32)) == b.ALGO_SEQUENTIAL
+    assert b.select_algo(b.make_desc(1, 2, 32, 32, 2, 4, b.GDN_FP32, algo=7)) == -1
+
+
+class _Fake:
+    """Stands in for a tensor: a placeholder device address (never dereferenced)."""
+    def __init__(self, addr):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+
+def _call(desc, offs, pl, **over):
+    base = 0x7f0000000000
+    names = ["q", "k", "v", "g", "beta", "qn", "kn", "vn", "gn", "betan", "conv_w",
+             "out", "out_noisy", "final_state", "workspace"]
+    ptr = {n: _Fake(base + 0x10000000 * i) for i, n in enumerate(names)}
+    ptr["conv_w"] = None
+    ptr.update(over)
+    lib = b.load_library()
+    ip = ctypes.POINTER(ctypes.c_int32)
+    offs = np.ascontiguousarray(offs, dtype=np.int32)
+    pl = np.ascontiguousarray(pl, dtype=np.int32)
+    p = lambda n: None if ptr[n] is None else ctypes.c_void_p(ptr[n].data_ptr())
+    ws_bytes = over.get("_ws_bytes", 256)
+    return lib.gdn_dual_forward(ctypes.byref(desc), p("q"), p("k"), p("v"), p("g"), p("beta"),
+                                p("qn"), p("kn"), p("vn"), p("gn"), p("betan"),
+                                offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), p("conv_w"),
+                                p("out"), p("out_noisy"), p("final_state"), p("workspace"),
+                                ctypes.c_size_t(ws_bytes), None)
+
+
+@no_gpu
+@pytest.mark.parametrize("case,expect", [
+    ("offsets_not_from_zero", b.GDN_ERR_INVALID_ARG),
+    ("offsets_decreasing", b.GDN_ERR_INVALID_ARG),
+    ("prompt_longer_than_doc", b.GDN_ERR_INVALID_ARG),
+    ("negative_prompt", b.GDN_ERR_INVALID_ARG),
+    ("response_not_multiple_of_B", b.GDN_ERR_INVALID_ARG),
+    ("null_q", b.GDN_ERR_INVALID_ARG),
+    ("null_noisy", b.GDN_ERR_INVALID_ARG),
+    ("null_final_state", b.GDN_ERR_INVALID_ARG),
+    ("conv_without_weights", b.GDN_ERR_INVALID_ARG),
+    ("workspace_too_small", b.GDN_ERR_INVALID_ARG),
+    ("null_workspace", b.GDN_ERR_INVALID_ARG),
+    ("misaligned_k", b.GDN_ERR_ALIGNMENT),
+    ("misaligned_out", b.GDN_ERR_ALIGNMENT),
+    ("unsupported_d", b.GDN_ERR_UNSUPPORTED),
+    ("unequal_dk_dv", b.GDN_ERR_UNSUPPORTED),
+    ("unsupported_conv_width", b.GDN_ERR_UNSUPPORTED),
+    ("bad_dtype", b.GDN_ERR_INVALID_ARG),
+    ("zero_docs", b.GDN_ERR_INVALID_ARG),
+    ("zero_block", b.GDN_ERR_INVALID_ARG),
+    ("reserved_nonzero", b.GDN_ERR_INVALID_ARG),
+    ("too_many_docs", b.GDN_ERR_UNSUPPORTED),
+])
+def test_host_validation_rejects(case, expect):
+    d = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32)
+    offs, pl = [0, 16, 40], [8, 4]
+    kw = {}
+    if case == "offsets_not_from_zero":
+        offs = [4, 16, 40]
+    elif case == "offsets_decreasing":
+        offs = [0, 16, 12]
+    elif case == "prompt_longer_than_doc":
+        pl = [20, 4]
+    elif case == "negative_prompt":
+        pl = [-4, 4]
+    elif case == "response_not_multiple_of_B":
+        pl = [7, 4]
+    elif case == "null_q":
+        kw["q"] = None
+    elif case == "null_noisy":
+        kw["vn"] = None
+    elif case == "null_final_state":
+        kw["final_state"] = None
+    elif case == "conv_without_weights":
+        d = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32, conv_width=4)
+    elif case == "workspace_too_small":
+        kw["_ws_bytes"] = 64
+    elif case == "null_workspace":
+        kw["workspace"] = None
+    elif case == "misaligned_k":
+        kw["k"] = _Fake(0x7f0000000008)
+    elif case == "misaligned_out":
+        kw["out"] = _Fake(0x7f0000000004)
+    elif case == "unsupported_d":
+        d = b.make_desc(2, 2, 48, 48, 2, 4, b.GDN_FP32)
+    elif case == "unequal_dk_dv":
+        d = b.make_desc(2, 2, 64, 32, 2, 4, b.GDN_FP32)
+    elif case == "unsupported_conv_width":
+        d = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32, conv_width=3)
+        kw["conv_w"] = _Fake(0x7f0000000000)
+    elif case == "bad_dtype":
+        d = b.make_desc(2, 2, 32, 32, 2, 4, 5)
+    elif case == "zero_docs":
+        d = b.make_desc(0, 2, 32, 32, 2, 4, b.GDN_FP32)
+        offs, pl = [0], []
+    elif case == "zero_block":
+        d = b.make_desc(2, 2, 32, 32, 2, 0, b.GDN_FP32)
+    elif case == "reserved_nonzero":
+        d = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32)
+        d.reserved = 1
+    elif case == "too_many_docs":
+        n = 1025
+        d = b.make_desc(n, 1, 32, 32, 0, 4, b.GDN_FP32)
+        offs, pl = list(range(0, 4 * (n + 1), 4)), [0] * n
+    assert _call(d, offs, pl, **kw) == expect
+
+
+@no_gpu
+def test_valid_arguments_without_device_report_cuda_error():
+    """All arguments valid, no GPU visible: the first CUDA call fails and maps to GDN_ERR_CUDA
+    (no crash, no abort)."""
+    d = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32)
+    assert _call(d, [0, 16, 40], [8, 4]) == b.GDN_ERR_CUDA
