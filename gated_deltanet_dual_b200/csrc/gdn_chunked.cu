@@ -1,16 +1,821 @@
-// gdn_chunked.cu -- chunked WY/UT dual-stream forward on tcgen05 tensor cores (sm_100a).
+// gdn_chunked.cu -- dual-stream Gated DeltaNet forward, chunked WY/UT form on tcgen05 tensor
+// cores (sm_100a).  bf16 I/O, fp32 state and accumulation, d_k = d_v = 128, chunk C = 64.
+//
+// Method ("FLARE: Diffusion for Hybrid Language Model", papernotes.org notes, Method > Key
+// design 2 and 3): clean causal gated delta rule
+//     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,  o_t = S_t^T q_t / sqrt(d),
+// and a block-bidirectional noisy stream: block b of every view restarts from S_{e(b-1)}, runs
+// its B noisy tokens and every position reads the block-end state.  No per-block state is ever
+// formed: each noisy row is carried as one extra row against the chunk's start state.
+//
+// Chunked form (derived from the rule; gamma = inclusive cumsum of g inside the chunk):
+//   A_ti = beta_t e^{gamma_t-gamma_i} k_t.k_i (i<t),  T = (I + A)^{-1},
+//   P_ti = e^{gamma_t-gamma_i} q_t.k_i (i<=t),       R = beta V - beta Gamma K S0,
+//   [P U ; U] = [P T ; T] R,  O = Gamma Q S0 + P U,  S_C = Gamma_C S0 + Khat^T U,
+//   Khat_t = e^{gamma_C-gamma_t} k_t.
+// Noisy row j of a block starting at chunk row bs (boundary e = bs-1): with y = Ptil_j Ttil
+// (Ttil the block's own WY inverse, Ptil_jl = e^{gammatil_B-gammatil_l} q~_j.k~_l),
+//   Z_j  = Gammatil_B q~_j - sum_l y_l beta~_l Gammatil_l k~_l,   WV_j = sum_l y_l beta~_l v~_l,
+//   o~_j = Gamma_e Z_j S0 + (Z_j K^T o M_j) U + WV_j,   M_ji = e^{gamma_e-gamma_i} [i <= e].
+//
+// One CTA per (document, head) unit (static schedule over the longest-first unit order), one
+// CTA per SM: 8 math warps + 1 control warp (TMA producer and single-thread MMA issuer).  Each
+// chunk runs five tensor-core phases, each followed by a math phase:
+//   PK1  [Q;K]K^T, [q~0;q~1][k~0;k~1]^T, [k~0;k~1][k~0;k~1]^T     (S-independent)
+//   PK2  [P;T] T -> P T,  [Z0;Z1] K^T                              (S-independent)
+//   S1   [Q;K] S0,  [Gamma_e Z] S0 (+= WV)                         (needs S0)
+//   S2   [P T; T] R                                                (needs R)
+//   S3   Khat^T U,  M'_Z U (+=)                                    (needs U)
+// Inputs of the next chunk are prefetched by TMA while the current chunk's S-dependent phases
+// run.  All waits are bounded; on timeout the kernel records GDN_ERR_TIMEOUT and exits.
+#include <cudaTypedefs.h>
+#include <mutex>
+
 #include "gdn_internal.cuh"
+#include "sm100.cuh"
 
 namespace gdn {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;                 // d_k = d_v
+constexpr int CH = 64;                 // chunk length
+constexpr int kMathWarps = 8;
+constexpr int kMathThreads = kMathWarps * 32;
+constexpr int kThreads = kMathThreads;   // thread 0 also issues TMA and MMA
+constexpr uint32_t kWaitIters = 1u << 22;
+
+// Dynamic shared memory layout (offsets from a 1024-byte aligned base).
+constexpr int OFF_S0 = 0;          // 32 KB  S0 bf16, MN-major B: 2 v-halves x [128 k-rows x 128 B]
+constexpr int OFF_QK = 32768;      // 32 KB  [Q;K] K-major: 2 d-halves x [Q 64 rows | K 64 rows]
+constexpr int OFF_V = 65536;       // 16 KB  V -> R -> U, MN-major: 2 v-halves x [64 rows x 128 B]
+constexpr int OFF_KH = 81920;      // 16 KB  Khat, MN-major A: 2 k-halves x [64 rows x 128 B]
+constexpr int OFF_Y = 98304;       // 16 KB  fp32 solve scratch, then [P;T] -> [P T;T] K-major
+constexpr int OFF_NQ = 114688;     // 32 KB  [q~0;q~1] -> Z -> Gamma_e Z, K-major
+constexpr int OFF_NK = 147456;     // 32 KB  [k~0;k~1] K-major; d-half 0 later holds M'_Z
+constexpr int OFF_NV = 180224;     // 32 KB  [v~0;v~1] per v-half (row-major, swizzled)
+constexpr int OFF_W = 212992;      //  3 KB  solve staging (three 16x16 fp32 blocks)
+constexpr int SMEM_USED = 216064;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;   // alignment slack
+
+// TMEM columns (512 allocated)
+constexpr uint32_t TM_R0 = 0;      // q~k~^T | [Q;K]S0 | dS
+constexpr uint32_t TM_R1 = 128;    // k~k~^T | [P U; U]
+constexpr uint32_t TM_N = 256;     // noisy accumulator (WV + Gamma_e Z S0 + M'_Z U)
+constexpr uint32_t TM_TK = 384;    // [Q;K]K^T | P T
+constexpr uint32_t TM_ZK = 448;    // Z K^T
+
+struct Maps {
+    CUtensorMap q, k, v, qn, kn, vn;
+};
+
+__device__ __forceinline__ void bar_all() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
+__device__ __forceinline__ void bar_math() { bar_all(); }
+
+__device__ __forceinline__ uint4 pack8(const float *f) {
+    uint4 r;
+    __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(f[2], f[3]);
+    __nv_bfloat162 c = __floats2bfloat162_rn(f[4], f[5]);
+    __nv_bfloat162 d = __floats2bfloat162_rn(f[6], f[7]);
+    r.x = *reinterpret_cast<uint32_t *>(&a);
+    r.y = *reinterpret_cast<uint32_t *>(&b);
+    r.z = *reinterpret_cast<uint32_t *>(&c);
+    r.w = *reinterpret_cast<uint32_t *>(&d);
+    return r;
+}
+
+__device__ __forceinline__ void unpack8(uint4 u, float *f) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
+        float2 p = __bfloat1622float2(h);
+        f[2 * i] = p.x;
+        f[2 * i + 1] = p.y;
+    }
+}
+
+// fp32 64x64 solve scratch, element (r, c) at r*64 + (c ^ (r & 31)) (conflict-free columns).
+__device__ __forceinline__ int sidx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+
+struct Unit {
+    int n, h;
+    int s, len, prompt, R, roff;
+    int nchunks, m_first;
+};
+
+__device__ __forceinline__ Unit make_unit(const Params &P, int u) {
+    Unit U;
+    U.n = P.unit_doc[u / P.H];
+    U.h = u % P.H;
+    U.s = P.doc_start[U.n];
+    U.len = P.doc_start[U.n + 1] - U.s;
+    U.prompt = P.doc_prompt[U.n];
+    U.R = U.len - U.prompt;
+    U.roff = P.resp_off[U.n];
+    const int npre = (U.prompt + CH - 1) / CH;
+    const int nres = (U.R + CH - 1) / CH;
+    U.m_first = -npre;
+    U.nchunks = npre + nres;
+    return U;
+}
+
+// Block coefficients of one noisy row: y = Ptil_j Ttil (back substitution against the block's
+// own I + Atil), then ycoef = y beta~ Gammatil (for Z) and wcoef = y beta~ (for WV).
+template <int B>
+__device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float (&wk)[32], int lane, int j,
+                                             const float *ngam, const float *nbeta,
+                                             float (&ycoef)[B], float (&wcoef)[B], float &gend) {
+    const int bs = (j / B) * B;
+    const int jl = j - bs;
+    const int wofs = bs & 31;
+    float aq[B], ak[B], gl[B], bl[B];
+#pragma unroll
+    for (int l = 0; l < B; ++l) {
+        aq[l] = 0.f;
+        ak[l] = 0.f;
+        gl[l] = ngam[bs + l];
+        bl[l] = nbeta[bs + l];
+    }
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        if ((c / B) * B == wofs) {
+            aq[c % B] = wq[c];
+            ak[c % B] = wk[c];
+        }
+    }
+    const float gj = ngam[j], bj = nbeta[j];
+    gend = gl[B - 1];
+    float arow[B], pt[B], y[B];
+#pragma unroll
+    for (int l = 0; l < B; ++l) {
+        arow[l] = (l < jl) ? bj * expf(fminf(gj - gl[l], 0.f)) * ak[l] : 0.f;
+        pt[l] = aq[l] * expf(gend - gl[l]);
+    }
+    const int base = lane - jl;
+#pragma unroll
+    for (int l = B - 1; l >= 0; --l) {
+        float acc = pt[l];
+#pragma unroll
+        for (int mm = l + 1; mm < B; ++mm) acc -= y[mm] * __shfl_sync(0xffffffffu, arow[l], base + mm);
+        y[l] = acc;
+    }
+#pragma unroll
+    for (int l = 0; l < B; ++l) {
+        wcoef[l] = y[l] * bl[l];
+        ycoef[l] = wcoef[l] * expf(gl[l]);
+    }
+}
+
+// Z row (in place of q~ row) and the W~V~ term into TMEM, for one 64-column half.
+template <int B>
+__device__ __forceinline__ void noisy_row_build(uint8_t *sm, uint32_t tb, int q, int ch, int rho, int j, int v,
+                                                const float (&ycoef)[B], const float (&wcoef)[B], float gend) {
+    const int bs = (j / B) * B;
+    const float Gend = expf(gend);
+    uint8_t *nq = sm + OFF_NQ + ch * 16384;
+    const uint8_t *nk = sm + OFF_NK + ch * 16384;
+    const uint8_t *nv = sm + OFF_NV + ch * 16384;
+#pragma unroll 1
+    for (int c8 = 0; c8 < 8; ++c8) {
+        float z[8], kv[8];
+        unpack8(*reinterpret_cast<const uint4 *>(nq + sw128_off(rho, c8)), z);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] *= Gend;
+#pragma unroll
+        for (int l = 0; l < B; ++l) {
+            unpack8(*reinterpret_cast<const uint4 *>(nk + sw128_off(64 * v + bs + l, c8)), kv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) z[e] = fmaf(-ycoef[l], kv[e], z[e]);
+        }
+        *reinterpret_cast<uint4 *>(nq + sw128_off(rho, c8)) = pack8(z);
+    }
+#pragma unroll 1
+    for (int hf = 0; hf < 2; ++hf) {
+        float acc[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int l = 0; l < B; ++l) {
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float vv[8];
+                unpack8(*reinterpret_cast<const uint4 *>(nv + sw128_off(64 * v + bs + l, hf * 4 + c4)), vv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[c4 * 8 + e] = fmaf(wcoef[l], vv[e], acc[c4 * 8 + e]);
+            }
+        }
+        tmem_st32(tmem_addr(tb, q * 32, TM_N + 64 * ch + 32 * hf), acc);
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void noisy_phase1(uint8_t *sm, uint32_t tb, int q, int ch, int lane, int rho,
+                                             const float *s_ngam, const float *s_nbeta) {
+    float wq[32], wk[32];
+    tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 32 * q), wq);
+    tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 32 * q), wk);
+    tmem_wait_ld();
+    const int v = rho >> 6, j = rho & 63;
+    float ycoef[B], wcoef[B], gend;
+    noisy_coeffs<B>(wq, wk, lane, j, s_ngam + 64 * v, s_nbeta + 64 * v, ycoef, wcoef, gend);
+    noisy_row_build<B>(sm, tb, q, ch, rho, j, v, ycoef, wcoef, gend);
+}
+
+// T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch (in place), blocked in
+// 16x16 tiles: diagonal tiles by forward substitution, then block rows 1..3.
+__device__ void solve_T(float *sa, float *sw, int mw, int lane) {
+    // diagonal blocks: warp I (0..3), lane c < 16 owns column c of D_I = (I + A_II)^{-1}
+    if (mw < 4 && lane < 16) {
+        const int I = mw, c = lane;
+        float x[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+            float acc = (jj == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int l = 0; l < jj; ++l) acc = fmaf(-sa[sidx(16 * I + jj, 16 * I + l)], x[l], acc);
+            x[jj] = acc;
+        }
+        __syncwarp(0x0000ffffu);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) sa[sidx(16 * I + jj, 16 * I + c)] = x[jj];
+    }
+    bar_math();
+    // block rows: T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ  (T_JJ = D_J), J < I
+    for (int I = 1; I < 4; ++I) {
+        float t8[8];
+        const int J = mw;
+        const int r = lane >> 1, c0 = (lane & 1) * 8;
+        if (J < I) {
+            float w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w8[e] = 0.f;
+            for (int K = J; K < I; ++K) {
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const float a = sa[sidx(16 * I + r, 16 * K + kk)];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) w8[e] = fmaf(a, sa[sidx(16 * K + kk, 16 * J + c0 + e)], w8[e]);
+                }
+            }
+            float *wst = sw + J * 256;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) wst[r * 16 + c0 + e] = w8[e];
+            __syncwarp();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t8[e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+                const float dik = sa[sidx(16 * I + r, 16 * I + kk)];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t8[e] = fmaf(-dik, wst[kk * 16 + c0 + e], t8[e]);
+            }
+        }
+        bar_math();
+        if (J < I) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sa[sidx(16 * I + r, 16 * J + c0 + e)] = t8[e];
+        }
+        bar_math();
+    }
+}
+
+template <int B>
+__global__ void __launch_bounds__(kThreads, 1)
+gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps M) {
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar_a, bar_b, bar_mma;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ float s_g[CH], s_gam[CH], s_beta[CH];
+    __shared__ float s_ng[2 * CH], s_ngam[2 * CH], s_nbeta[2 * CH];
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, ch = (warp >> 2) & 1, rho = q * 32 + lane;   // TMEM row (lane) and column half
+    const int H = P.H, V = P.V;
+    const int64_t TR = P.TR;
+    const float scale = P.scale;
+
+    if (tid == 0) {
+        mbar_init(&bar_a, 1);
+        mbar_init(&bar_b, 1);
+        mbar_init(&bar_mma, 1);
+        fence_mbar_init();
+        s_abort = 0;
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tmem_alloc(&s_tmem, 512);
+        tmem_relinquish();
+        if (lane == 0) {
+            prefetch_tmap(&M.q); prefetch_tmap(&M.k); prefetch_tmap(&M.v);
+            prefetch_tmap(&M.qn); prefetch_tmap(&M.kn); prefetch_tmap(&M.vn);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = s_tmem;
+    uint32_t ph_a = 0, ph_b = 0, ph_mma = 0;
+
+    auto fail = [&](int where) {
+        if (atomicExch(&s_abort, 1) == 0) {
+            atomicExch(&P.ws->status, (int)GDN_ERR_TIMEOUT);
+            atomicExch(&P.ws->timeout_where, where);
+        }
+    };
+    auto wait_mma = [&](int where) {
+        if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(where);
+        ++ph_mma;
+        __syncwarp();            // reconverge before warp-collective tcgen05.ld/st
+        tc_fence_after();
+    };
+
+    // Issue the TMA loads of chunk m of unit U (control lane 0).  group A: [Q;K] and, for a
+    // response chunk, [q~;.] and v~;  group B: V and, for a response chunk, [k~;.].
+    auto issue_a = [&](const Unit &U, int m) {
+        const bool nz = (m >= 0) && V > 0;
+        const int cstart = U.s + U.prompt + CH * m;
+        mbar_arrive_expect_tx(&bar_a, 32768u + (nz ? 65536u : 0u));
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_3d(sm + OFF_QK + hf * 16384, &M.q, &bar_a, hf * 64, U.h, cstart);
+            tma_load_3d(sm + OFF_QK + hf * 16384 + 8192, &M.k, &bar_a, hf * 64, U.h, cstart);
+        }
+        if (nz) {
+            for (int vw = 0; vw < 2; ++vw) {
+                const int row = vw * (int)TR + U.roff + CH * m;
+                for (int hf = 0; hf < 2; ++hf) {
+                    tma_load_3d(sm + OFF_NQ + hf * 16384 + vw * 8192, &M.qn, &bar_a, hf * 64, U.h, row);
+                    tma_load_3d(sm + OFF_NV + hf * 16384 + vw * 8192, &M.vn, &bar_a, hf * 64, U.h, row);
+                }
+            }
+        }
+    };
+    auto issue_b = [&](const Unit &U, int m) {
+        const bool nz = (m >= 0) && V > 0;
+        const int cstart = U.s + U.prompt + CH * m;
+        mbar_arrive_expect_tx(&bar_b, 16384u + (nz ? 32768u : 0u));
+        for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_V + hf * 8192, &M.v, &bar_b, hf * 64, U.h, cstart);
+        if (nz) {
+            for (int vw = 0; vw < 2; ++vw) {
+                const int row = vw * (int)TR + U.roff + CH * m;
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_3d(sm + OFF_NK + hf * 16384 + vw * 8192, &M.kn, &bar_b, hf * 64, U.h, row);
+            }
+        }
+    };
+
+    const uint32_t a_s0 = smem_u32(sm + OFF_S0), a_qk = smem_u32(sm + OFF_QK), a_v = smem_u32(sm + OFF_V);
+    const uint32_t a_kh = smem_u32(sm + OFF_KH), a_y = smem_u32(sm + OFF_Y), a_nq = smem_u32(sm + OFF_NQ);
+    const uint32_t a_nk = smem_u32(sm + OFF_NK);
+    float *scratch = reinterpret_cast<float *>(sm + OFF_Y);
+    float *wstage = reinterpret_cast<float *>(sm + OFF_W);
+
+    for (int u = blockIdx.x; u < P.num_units; u += gridDim.x) {
+        const Unit U = make_unit(P, u);
+        float S[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) S[c] = 0.f;
+        {
+            // zero S0 (bf16): thread (rho, ch) owns row rho of v-half ch
+            uint8_t *s0 = sm + OFF_S0 + ch * 16384;
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) *reinterpret_cast<uint4 *>(s0 + sw128_off(rho, c8)) = z;
+            fence_async_smem();
+            if (U.nchunks == 0) {
+                float *fs = P.final_state + ((int64_t)U.n * H + U.h) * D * D + (int64_t)rho * D + 64 * ch;
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4 *>(fs + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        if (tid == 0 && U.nchunks > 0) {
+            issue_a(U, U.m_first);
+            issue_b(U, U.m_first);
+        }
+        for (int ci = 0; ci < U.nchunks; ++ci) {
+            const int m = U.m_first + ci;
+            const bool noisy = (m >= 0) && V > 0;
+            const bool last = ci == U.nchunks - 1;
+            const int cstart = U.s + U.prompt + CH * m;   // global token of chunk row 0
+            // ---- per-chunk scalars: gates, betas, cumulative log-decays ----
+            {
+                if (tid < CH) {
+                    const int tok = cstart + tid;
+                    const bool ok = tok >= U.s && tok < U.s + U.len;
+                    s_g[tid] = ok ? P.g[(int64_t)tok * H + U.h] : 0.f;
+                    s_beta[tid] = ok ? P.beta[(int64_t)tok * H + U.h] : 0.f;
+                } else if (noisy && tid < 3 * CH) {
+                    const int idx = tid - CH, vw = idx >> 6, jj = idx & 63;
+                    const int rr = CH * m + jj;
+                    const bool ok = vw < V && rr < U.R;
+                    const int64_t row = (int64_t)vw * TR + U.roff + rr;
+                    s_ng[idx] = ok ? P.gn[row * H + U.h] : 0.f;
+                    s_nbeta[idx] = ok ? P.betan[row * H + U.h] : 0.f;
+                }
+                bar_math();
+                if (tid < CH) {
+                    float acc = 0.f;
+                    for (int i = 0; i <= tid; ++i) acc += s_g[i];
+                    s_gam[tid] = acc;
+                } else if (noisy && tid < 3 * CH) {
+                    const int idx = tid - CH, jj = idx & 63, base = idx - jj;
+                    const int bs = (jj / B) * B;
+                    float acc = 0.f;
+                    for (int i = bs; i <= jj; ++i) acc += s_ng[base + i];
+                    s_ngam[idx] = acc;
+                }
+            }
+            // ---- wait for this chunk's tiles ----
+            if (!mbar_wait(&bar_a, ph_a & 1, kWaitIters)) fail(1);
+            ++ph_a;
+            if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
+            ++ph_b;
+            __syncwarp();
+            bar_all();
+            if (s_abort) break;
+
+            // ================= PK1 =================
+            if (tid == 0) {
+                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_bf16(tb + TM_TK, make_sdesc(a_qk + off, 16, 1024), make_sdesc(a_qk + 8192 + off, 16, 1024),
+                             make_idesc_bf16(128, 64, 0, 0), kk > 0);
+                }
+                if (noisy) {
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_bf16(tb + TM_R0, make_sdesc(a_nq + off, 16, 1024), make_sdesc(a_nk + off, 16, 1024),
+                                 make_idesc_bf16(128, 128, 0, 0), kk > 0);
+                        mma_bf16(tb + TM_R1, make_sdesc(a_nk + off, 16, 1024), make_sdesc(a_nk + off, 16, 1024),
+                                 make_idesc_bf16(128, 128, 0, 0), kk > 0);
+                    }
+                }
+                mma_commit(&bar_mma);
+            }
+            wait_mma(10);
+            // clean: P rows (lanes 0-63) into registers, A rows (lanes 64-127) into scratch
+            if (rho >= 64) {
+                float tk[32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), tk);
+                tmem_wait_ld();
+                const int t = rho - 64;
+                const float gt = s_gam[t], bt = s_beta[t];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int i = 32 * ch + c;
+                    scratch[sidx(t, i)] = (i < t) ? bt * expf(fminf(gt - s_gam[i], 0.f)) * tk[c] : 0.f;
+                }
+            }
+            // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout)
+            const float gC = s_gam[CH - 1];
+            for (int it = tid; it < 64 * 16; it += kMathThreads) {
+                const int t = it >> 4, c16 = it & 15, hf = c16 >> 3, c8 = c16 & 7;
+                float f[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QK + hf * 16384 + sw128_off(64 + t, c8)), f);
+                const float sc = expf(fminf(gC - s_gam[t], 0.f));
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] *= sc;
+                *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
+            }
+            // noisy: block coefficients, Z rows (in place of q~) and W~V~ into TMEM
+            if (noisy) noisy_phase1<B>(sm, tb, q, ch, lane, rho, s_ngam, s_nbeta);
+            bar_math();
+            solve_T(scratch, wstage, warp, lane);
+            // [P ; T] as bf16 K-major A (128 rows x 64): this thread writes row rho, cols [32ch, 32ch+32)
+            float tv[32];
+            if (rho >= 64) {
+                const int t = rho - 64;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) tv[c] = scratch[sidx(t, 32 * ch + c)];
+            }
+            bar_math();
+            if (rho < 64) {
+                // P_ti = e^{gamma_t - gamma_i} q_t.k_i (i <= t), from [Q;K]K^T still in TMEM
+                float pv[32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), pv);
+                tmem_wait_ld();
+                const int t = rho;
+                const float gt = s_gam[t];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int i = 32 * ch + c;
+                    pv[c] = (i <= t) ? pv[c] * expf(fminf(gt - s_gam[i], 0.f)) : 0.f;
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(pv + 8 * c4);
+            } else {
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(tv + 8 * c4);
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            bar_all();
+            if (s_abort) break;
+
+            // ================= PK2 =================
+            if (tid == 0) {
+                tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tb + TM_TK, make_sdesc(a_y + kk * 32, 16, 1024),
+                             make_sdesc(a_y + 8192 + kk * 2048, 8192, 1024), make_idesc_bf16(128, 64, 0, 1), kk > 0);
+                if (noisy) {
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_bf16(tb + TM_ZK, make_sdesc(a_nq + off, 16, 1024), make_sdesc(a_qk + 8192 + off, 16, 1024),
+                                 make_idesc_bf16(128, 64, 0, 0), kk > 0);
+                    }
+                }
+                mma_commit(&bar_mma);
+            }
+            wait_mma(20);
+            if (rho < 64) {
+                float pt[32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), pt);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(pt + 8 * c4);
+            }
+            if (noisy) {
+                float zk[32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_ZK + 32 * ch), zk);
+                tmem_wait_ld();
+                const int jj = rho & 63;
+                const int e = (jj / B) * B - 1;          // chunk-local boundary row (-1: S0)
+                const float ge = e >= 0 ? s_gam[e] : 0.f;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int i = 32 * ch + c;
+                    zk[c] = (i <= e) ? zk[c] * expf(fminf(ge - s_gam[i], 0.f)) : 0.f;
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
+                    *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
+                const float Ge = expf(ge);        // Gamma_e (1 for e = -1)
+                uint8_t *zrow = sm + OFF_NQ + ch * 16384;
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    float f[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(zrow + sw128_off(rho, c8)), f);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) f[x] *= Ge;
+                    *reinterpret_cast<uint4 *>(zrow + sw128_off(rho, c8)) = pack8(f);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            bar_all();
+            if (s_abort) break;
+
+            // ================= S1 =================
+            if (tid == 0) {
+                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_bf16(tb + TM_R0, make_sdesc(a_qk + off, 16, 1024), make_sdesc(a_s0 + kk * 2048, 16384, 1024),
+                             make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                }
+                if (noisy) {
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_bf16(tb + TM_N, make_sdesc(a_nq + off, 16, 1024), make_sdesc(a_s0 + kk * 2048, 16384, 1024),
+                                 make_idesc_bf16(128, 128, 0, 1), 1u);
+                    }
+                }
+                mma_commit(&bar_mma);
+                // prefetch group A of the next chunk once S1 has consumed [Q;K] and Z
+                if (!last) {
+                    if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(30);
+                    else issue_a(U, m + 1);
+                }
+            }
+            wait_mma(30);
+            if (rho >= 64) {
+                const int t = rho - 64;
+                const float bt = s_beta[t], bg = bt * expf(s_gam[t]);
+                uint8_t *vrow = sm + OFF_V + ch * 8192;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float ks[32];
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32 * hf), ks);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        float f[8];
+                        const uint32_t o = sw128_off(t, 4 * hf + c4);
+                        unpack8(*reinterpret_cast<const uint4 *>(vrow + o), f);
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) f[x] = bt * f[x] - bg * ks[8 * c4 + x];
+                        *reinterpret_cast<uint4 *>(vrow + o) = pack8(f);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            bar_all();
+            if (s_abort) break;
+
+            // ================= S2 =================
+            if (tid == 0) {
+                tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tb + TM_R1, make_sdesc(a_y + kk * 32, 16, 1024), make_sdesc(a_v + kk * 2048, 8192, 1024),
+                             make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                mma_commit(&bar_mma);
+            }
+            wait_mma(40);
+            if (rho < 64) {
+                const int t = rho;
+                const int tok = cstart + t;
+                const bool ok = tok >= U.s && tok < U.s + U.len;
+                const float Gt = expf(s_gam[t]);
+                __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(P.out) + ((int64_t)tok * H + U.h) * D + 64 * ch;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float qs[32], pu[32];
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32 * hf), qs);
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32 * hf), pu);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) qs[x] = (Gt * qs[x] + pu[x]) * scale;
+                    if (ok) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(qs + 8 * c4);
+                    }
+                }
+            } else {
+                const int t = rho - 64;
+                uint8_t *vrow = sm + OFF_V + ch * 8192;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float uu[32];
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32 * hf), uu);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4)
+                        *reinterpret_cast<uint4 *>(vrow + sw128_off(t, 4 * hf + c4)) = pack8(uu + 8 * c4);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            bar_all();
+            if (s_abort) break;
+
+            // ================= S3 =================
+            if (tid == 0) {
+                tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tb + TM_R0, make_sdesc(a_kh + kk * 2048, 8192, 1024), make_sdesc(a_v + kk * 2048, 8192, 1024),
+                             make_idesc_bf16(128, 128, 1, 1), kk > 0);
+                if (noisy) {
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tb + TM_N, make_sdesc(a_nk + kk * 32, 16, 1024), make_sdesc(a_v + kk * 2048, 8192, 1024),
+                                 make_idesc_bf16(128, 128, 0, 1), 1u);
+                }
+                mma_commit(&bar_mma);
+                if (!last) {
+                    if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(50);
+                    else issue_b(U, m + 1);
+                }
+            }
+            wait_mma(50);
+            const float GC = expf(s_gam[CH - 1]);
+            uint8_t *srow = sm + OFF_S0 + ch * 16384;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float ds[32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32 * hf), ds);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) S[32 * hf + x] = fmaf(GC, S[32 * hf + x], ds[x]);
+            }
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8)
+                *reinterpret_cast<uint4 *>(srow + sw128_off(rho, c8)) = pack8(S + 8 * c8);
+            if (last) {
+                float *fs = P.final_state + ((int64_t)U.n * H + U.h) * D * D + (int64_t)rho * D + 64 * ch;
+#pragma unroll
+                for (int c = 0; c < 64; c += 4)
+                    *reinterpret_cast<float4 *>(fs + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+            }
+            if (noisy) {
+                const int vw = rho >> 6, jj = rho & 63;
+                const int rr = CH * m + jj;
+                const bool ok = vw < V && rr < U.R;
+                __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(P.out_noisy) +
+                                      (((int64_t)vw * TR + U.roff + rr) * H + U.h) * D + 64 * ch;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float on[32];
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_N + 64 * ch + 32 * hf), on);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) on[x] *= scale;
+                    if (ok) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(on + 8 * c4);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            bar_all();
+            if (s_abort) break;
+        }
+        if (s_abort) break;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tb, 512);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a [rows, H, 128] bf16 tensor; box = 64 rows x 1 head x 64 columns, 128B swizzle.
+bool encode_map(CUtensorMap *m, const void *ptr, int H, int64_t rows) {
+    auto enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 bool chunked_supported(int dtype, int d, int B, int conv_width) {
-    (void)dtype; (void)d; (void)B; (void)conv_width;
-    return false;
+    return dtype == GDN_BF16 && d == D && conv_width == 0 && B >= 1 && B <= 32 && (32 % B) == 0;
 }
 
 cudaError_t launch_chunked(const Params &p, cudaStream_t stream) {
-    (void)p; (void)stream;
-    return cudaErrorNotSupported;
+    if (p.num_units == 0) return cudaSuccess;
+    if (p.V > 2 || p.T == 0) return cudaErrorNotSupported;
+    Maps maps;
+    const bool noisy = p.V > 0 && p.TR > 0;
+    if (!encode_map(&maps.q, p.q, p.H, p.T) || !encode_map(&maps.k, p.k, p.H, p.T) ||
+        !encode_map(&maps.v, p.v, p.H, p.T))
+        return cudaErrorInvalidValue;
+    if (noisy) {
+        if (!encode_map(&maps.qn, p.qn, p.H, (int64_t)p.V * p.TR) || !encode_map(&maps.kn, p.kn, p.H, (int64_t)p.V * p.TR) ||
+            !encode_map(&maps.vn, p.vn, p.H, (int64_t)p.V * p.TR))
+            return cudaErrorInvalidValue;
+    } else {
+        maps.qn = maps.q;
+        maps.kn = maps.k;
+        maps.vn = maps.v;
+    }
+    static int num_sms = 0;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaError_t e = cudaSuccess;
+        for (auto fn : {gdn_chunked_kernel<1>, gdn_chunked_kernel<2>, gdn_chunked_kernel<4>,
+                        gdn_chunked_kernel<8>, gdn_chunked_kernel<16>, gdn_chunked_kernel<32>}) {
+            cudaError_t r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+            if (r != cudaSuccess) e = r;
+        }
+        attr_err = e;
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    const int grid = std::min(p.num_units, num_sms > 0 ? num_sms : 148);
+    switch (p.B) {
+        case 1: gdn_chunked_kernel<1><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
+        case 2: gdn_chunked_kernel<2><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
+        case 4: gdn_chunked_kernel<4><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
+        case 8: gdn_chunked_kernel<8><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
+        case 16: gdn_chunked_kernel<16><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
+        case 32: gdn_chunked_kernel<32><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace gdn

@@ -33,3 +33,18 @@ def test_chunk_bounds_anchor_at_response_start():
     starts = [x for x, _ in b]
     assert 150 in starts and all((s - 150) % 64 == 0 for s in starts[1:])
     assert b[-1][1] == 300 and all(y == x2 for (_, y), (x2, _) in zip(b, b[1:]))
+
+
+@pytest.mark.parametrize("B", [1, 2, 4, 8])
+@pytest.mark.parametrize("conv", [0, 4])
+def test_folded_noisy_rows_equal_sequential(B, conv):
+    """The folded per-row form of the noisy stream (Z rows, W~V~ term, masked Z K^T) used by
+    the tensor-core kernel equals the sequential oracle."""
+    rng = np.random.default_rng(200 + B + conv)
+    lens, prompts = [13 + 6 * B, 5 * B, 29 + 3 * B], [13, 0, 29]
+    P = brute.rand_problem(rng, lens, prompts, H=2, dk=6, dv=6, V=2, B=B, conv=conv, g_lo=-0.6)
+    ref = pins._run(oracle.forward, P)
+    got = chunk_reference.forward_chunked_folded(P, C=max(8, 2 * B))
+    for key in ("out", "out_noisy", "final_state"):
+        err = np.max(np.abs(got[key] - ref[key]))
+        assert err < 1e-10 * max(1.0, np.max(np.abs(ref[key]))), (key, err)

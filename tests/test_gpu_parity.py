@@ -58,15 +58,22 @@ def test_head_dims_and_dtypes(d, dtype):
     check(prob, dtype, b.ALGO_SEQUENTIAL)
 
 
+def algos_for(conv):
+    """Algorithms that implement a bf16 d=128 problem with this conv setting."""
+    return [b.ALGO_SEQUENTIAL] + ([b.ALGO_CHUNKED] if conv == 0 else [])
+
+
 @pytest.mark.parametrize("B", [1, 2, 4, 8, 16, 32])
 @pytest.mark.parametrize("conv", [0, 4])
 def test_block_sizes_and_conv(B, conv):
-    """Ragged prompts (not multiples of 64 or B), several tiles, a response-only document."""
+    """Ragged prompts (not multiples of 64 or B), several chunks, a partial last chunk, a
+    response-only document."""
     lens = [37 + 3 * 64, 2 * 64, 96]
     prompts = [37, 0, 32]
     lens = [p + ((l - p) // B) * B for l, p in zip(lens, prompts)]
     prob = small(lens, prompts, H=3, d=128, B=B, dtype="bf16", conv=conv, seed=B + conv)
-    check(prob, "bf16", b.ALGO_AUTO)
+    for algo in algos_for(conv):
+        check(prob, "bf16", algo)
 
 
 @pytest.mark.parametrize("V", [0, 1, 3])
@@ -75,19 +82,38 @@ def test_view_counts(V):
     check(prob, "fp32", b.ALGO_AUTO)
 
 
-def test_packed_documents_with_degenerate_lengths():
+@pytest.mark.parametrize("V", [0, 1, 2])
+def test_view_counts_chunked(V):
+    prob = small([200, 136], [72, 8], H=2, d=128, V=V, dtype="bf16", seed=20 + V)
+    check(prob, "bf16", b.ALGO_CHUNKED)
+
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_packed_documents_with_degenerate_lengths(conv):
     """Packed row with an empty document, a prompt-only document, a response-only document and
     one-block documents."""
     lens = [0, 24, 4, 100, 8, 0, 52]
     prompts = [0, 24, 0, 20, 4, 0, 0]
-    prob = small(lens, prompts, H=2, d=128, B=4, dtype="bf16", conv=4, seed=7)
-    check(prob, "bf16")
+    prob = small(lens, prompts, H=2, d=128, B=4, dtype="bf16", conv=conv, seed=7)
+    for algo in algos_for(conv):
+        check(prob, "bf16", algo)
 
 
 def test_strong_gates_and_large_beta():
     """g ~ U(-0.5, 0), beta = sigmoid(N(0, 2)) as in the large workload, over long chunks."""
     prob = small([512 + 256, 640], [256, 128], H=2, d=128, B=4, dtype="bf16", seed=11, g_lo=-0.5, beta_std=2.0)
-    check(prob, "bf16")
+    for algo in algos_for(0):
+        check(prob, "bf16", algo)
+
+
+def test_chunked_matches_sequential_kernel():
+    """The two CUDA kernels agree with each other on a multi-unit problem (both fp32 state)."""
+    prob = small([1000, 1536, 520], [232, 512, 8], H=4, d=128, B=4, dtype="bf16", seed=31)
+    a = [t.float().clone() for t in b.forward_problem(prob, algo=b.ALGO_SEQUENTIAL)]
+    c = [t.float().clone() for t in b.forward_problem(prob, algo=b.ALGO_CHUNKED)]
+    torch.cuda.synchronize()
+    for x, y in zip(a, c):
+        assert float((x - y).abs().max()) <= 2e-2 * float(x.abs().max())
 
 
 def test_doc_reset_equivalence_on_gpu():
