@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from gated_deltanet_dual_b200 import binding as gb  # noqa: E402
+from gated_deltanet_dual_b200 import replicas  # noqa: E402
 from gated_deltanet_dual_b200 import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "train_8x4096_h16_d128"
@@ -237,24 +238,19 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
-    rank = int(os.environ.get("RANK", 0))
-    world = int(os.environ.get("WORLD_SIZE", 1))
-    local = int(os.environ.get("LOCAL_RANK", 0))
+    rank, world, local = replicas.env_rank()
     wl = synth.get_workload(args.workload)
 
     if args.impl == "reference":
         run_reference(args, wl, rank)
         return
 
-    import torch.distributed as dist
-    from datetime import timedelta
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    replicas.init(world, backend="nccl", device=dev)
     algo = {"auto": gb.ALGO_AUTO, "sequential": gb.ALGO_SEQUENTIAL, "chunked": gb.ALGO_CHUNKED}[args.algo]
 
-    prob = synth.make_problem(wl, seed=rank, device=dev)
+    prob = synth.make_problem(wl, seed=replicas.replica_seed(0, rank), device=dev)
     T, TR, V, H, d = prob.T, prob.T_R, prob.num_views, prob.num_heads, prob.d_k
     desc = gb.make_desc(prob.num_docs, H, d, d, V, prob.block_size, gb._dtype_code(prob.q), prob.conv_width, algo)
     used_algo = gb.select_algo(desc)
@@ -268,15 +264,10 @@ def main():
         gb.forward_problem(prob, algo=algo, out=out, out_noisy=out_n, final_state=fs, workspace=ws)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(world)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, world, device=dev)
 
     for _ in range(args.warmup):
         step()
@@ -302,7 +293,7 @@ def main():
 
     work = algorithmic_work(prob)
     toks_all = prob.tokens() * world
-    value = toks_all * args.steps / (elapsed_ms / 1e3)
+    value = replicas.throughput(prob.tokens(), world, args.steps, elapsed_ms)
     peaks = measured_peaks()
     achieved_gbs = work["bytes"] / (kernel_ms / 1e3) / 1e9
     traffic = profiled_traffic(used_algo, wl.name)
@@ -357,9 +348,7 @@ def main():
         cb = time_oracle(wl, steps=1, warmup=0, max_units=max_units)
         cpu_baseline = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.shutdown(world)
     if rank != 0:
         return
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
