@@ -200,3 +200,21 @@ def forward_problem(prob, **kw):
     """Run the forward on a synthetic problem whose tensors live on the GPU."""
     return forward(prob.q, prob.k, prob.v, prob.g, prob.beta, prob.qn, prob.kn, prob.vn, prob.gn,
                    prob.betan, prob.doc_offsets, prob.prompt_len, prob.block_size, conv_w=prob.conv_w, **kw)
+
+
+def forward_noalloc_raw(desc: Desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, conv_w,
+                        out, out_noisy, final_state, stream=None) -> int:
+    """C-ABI call of gdn_dual_forward_noalloc (no workspace: the library's fixed device scratch
+    is used, for callers that cannot allocate).  Returns the status code."""
+    lib = load_library()
+    fn = lib.gdn_dual_forward_noalloc
+    vp, ip = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(Desc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ip, ip, vp, vp, vp, vp, vp]
+    offs = _host_i32(doc_offsets)
+    pl = _host_i32(prompt_len)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return int(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(qn), _ptr(kn), _ptr(vn),
+                  _ptr(gn), _ptr(betan), offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(conv_w),
+                  _ptr(out), _ptr(out_noisy), _ptr(final_state), ctypes.c_void_p(stream)))

@@ -120,6 +120,34 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
                             void *workspace, size_t workspace_bytes,
                             gdn_stream_t stream);
 
+/*
+ * gdn_dual_forward without a workspace argument, for callers that cannot allocate device
+ * memory: e.g. an engine that reserved all device memory for its own pool up front, or a
+ * plugin/FFI host with no device allocator reachable through the C ABI.  (The FLARE notes have
+ * no counterpart; this is an interface convenience.)  Same inputs, outputs, layouts, stream
+ * semantics and host validation as gdn_dual_forward.
+ *   Scratch: a fixed 4096-byte array in the library's own device memory (a file-scope
+ *     __device__ array; every GPU that loads the library holds it until the process exits).
+ *     A problem whose gdn_dual_workspace_size() exceeds 4096 bytes returns
+ *     GDN_ERR_UNSUPPORTED (the current kernels need 256 bytes).
+ *   Allocation: none, on any call (no cudaMalloc or cudaFree).
+ *   Set-up: the first call on a device, with that device current, looks up the array's device
+ *     address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Sharing: all calls on a device share the array, which keeps the last call's contents; the
+ *     status words are cleared on `stream` at the start of every call.  Calls whose work
+ *     overlaps on the GPU (e.g. on two streams at once) race on the array: serialise them.
+ *   Errors: as gdn_dual_forward, plus GDN_ERR_CUDA if the set-up lookup fails.
+ */
+gdn_status gdn_dual_forward_noalloc(const gdn_dual_desc *desc,
+                                    const void *q, const void *k, const void *v,
+                                    const float *g, const float *beta,
+                                    const void *qn, const void *kn, const void *vn,
+                                    const float *gn, const float *betan,
+                                    const int32_t *doc_offsets, const int32_t *prompt_len,
+                                    const float *conv_w,
+                                    void *out, void *out_noisy, float *final_state,
+                                    gdn_stream_t stream);
+
 /* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
  * last gdn_dual_forward on it (GDN_OK or GDN_ERR_TIMEOUT), or GDN_ERR_CUDA if the sync fails.
  * For debugging and tests; the forward path itself never synchronises. */
