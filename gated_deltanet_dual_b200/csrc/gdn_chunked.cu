@@ -30,6 +30,7 @@
 // run.  All waits are bounded; on timeout the kernel records GDN_ERR_TIMEOUT and exits.
 #include <cudaTypedefs.h>
 #include <mutex>
+#include <type_traits>
 
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
@@ -55,8 +56,8 @@ constexpr int OFF_Y = 98304;       // 16 KB  fp32 solve scratch, then [P;T] -> [
 constexpr int OFF_NQ = 114688;     // 32 KB  [q~0;q~1] -> Z -> Gamma_e Z, K-major
 constexpr int OFF_NK = 147456;     // 32 KB  [k~0;k~1] K-major; d-half 0 later holds M'_Z
 constexpr int OFF_NV = 180224;     // 32 KB  [v~0;v~1] per v-half (row-major, swizzled)
-constexpr int OFF_W = 212992;      //  3 KB  solve staging (three 16x16 fp32 blocks)
-constexpr int SMEM_USED = 216064;
+constexpr int OFF_W = 212992;      //  4 KB  triangular-solve staging (one 32x32 fp32 block)
+constexpr int SMEM_USED = 217088;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;   // alignment slack
 
 // TMEM columns (512 allocated)
@@ -97,8 +98,12 @@ __device__ __forceinline__ void unpack8(uint4 u, float *f) {
     }
 }
 
-// fp32 64x64 solve scratch, element (r, c) at r*64 + (c ^ (r & 31)) (conflict-free columns).
-__device__ __forceinline__ int sidx(int r, int c) { return r * 64 + (c ^ (r & 31)); }
+// fp32 64x64 solve scratch: 16-byte chunk c>>2 of row r sits at chunk (c>>2) ^ (r & 7), so both
+// row-segment accesses by one thread (float4) and column accesses across a warp avoid conflicts.
+__device__ __forceinline__ int sidx(int r, int c) { return r * 64 + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3); }
+__device__ __forceinline__ float4 *srow4(float *sa, int r, int c4) {
+    return reinterpret_cast<float4 *>(sa + r * 64 + ((((c4 >> 2) ^ (r & 7))) << 2));
+}
 
 struct Unit {
     int n, h;
@@ -151,8 +156,8 @@ __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float 
     float arow[B], pt[B], y[B];
 #pragma unroll
     for (int l = 0; l < B; ++l) {
-        arow[l] = (l < jl) ? bj * expf(fminf(gj - gl[l], 0.f)) * ak[l] : 0.f;
-        pt[l] = aq[l] * expf(gend - gl[l]);
+        arow[l] = (l < jl) ? bj * exp2f(fminf(gj - gl[l], 0.f)) * ak[l] : 0.f;
+        pt[l] = aq[l] * exp2f(gend - gl[l]);
     }
     const int base = lane - jl;
 #pragma unroll
@@ -165,55 +170,40 @@ __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float 
 #pragma unroll
     for (int l = 0; l < B; ++l) {
         wcoef[l] = y[l] * bl[l];
-        ycoef[l] = wcoef[l] * expf(gl[l]);
+        ycoef[l] = wcoef[l] * exp2f(gl[l]);
     }
 }
 
-// Z row (in place of q~ row) and the W~V~ term into TMEM, for one 64-column half.
+// This thread's half (K columns [64ch, 64ch+64), i.e. the noisy rows of view ch) of the
+// block-diagonal row `sign * coef` of noisy row (view v, block start bs), stored into tensor
+// memory as bf16 pairs (low half = even k): an A operand for a tensor-memory MMA.
 template <int B>
-__device__ __forceinline__ void noisy_row_build(uint8_t *sm, uint32_t tb, int q, int ch, int rho, int j, int v,
-                                                const float (&ycoef)[B], const float (&wcoef)[B], float gend) {
-    const int bs = (j / B) * B;
-    const float Gend = expf(gend);
-    uint8_t *nq = sm + OFF_NQ + ch * 16384;
-    const uint8_t *nk = sm + OFF_NK + ch * 16384;
-    const uint8_t *nv = sm + OFF_NV + ch * 16384;
-#pragma unroll 1
-    for (int c8 = 0; c8 < 8; ++c8) {
-        float z[8], kv[8];
-        unpack8(*reinterpret_cast<const uint4 *>(nq + sw128_off(rho, c8)), z);
+__device__ __forceinline__ void store_block_row(uint32_t taddr, int ch, int v, int bs, const float (&coef)[B],
+                                                float sign) {
+    float w[32];
+    if constexpr (B == 1) {
+        __nv_bfloat162 pr = (bs & 1) ? __floats2bfloat162_rn(0.f, sign * coef[0]) : __floats2bfloat162_rn(sign * coef[0], 0.f);
+        const float pf = __uint_as_float(*reinterpret_cast<uint32_t *>(&pr));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) z[e] *= Gend;
+        for (int x = 0; x < 32; ++x) w[x] = (ch == v && x == (bs >> 1)) ? pf : 0.f;
+    } else {
+        constexpr int HB = B / 2;
 #pragma unroll
-        for (int l = 0; l < B; ++l) {
-            unpack8(*reinterpret_cast<const uint4 *>(nk + sw128_off(64 * v + bs + l, c8)), kv);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) z[e] = fmaf(-ycoef[l], kv[e], z[e]);
+        for (int x = 0; x < 32; ++x) {
+            const int l0 = 2 * (x % HB);
+            __nv_bfloat162 pr = __floats2bfloat162_rn(sign * coef[l0], sign * coef[l0 + 1]);
+            const float pf = __uint_as_float(*reinterpret_cast<uint32_t *>(&pr));
+            w[x] = (ch == v && (x / HB) == (bs / B)) ? pf : 0.f;
         }
-        *reinterpret_cast<uint4 *>(nq + sw128_off(rho, c8)) = pack8(z);
     }
-#pragma unroll 1
-    for (int hf = 0; hf < 2; ++hf) {
-        float acc[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int l = 0; l < B; ++l) {
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                float vv[8];
-                unpack8(*reinterpret_cast<const uint4 *>(nv + sw128_off(64 * v + bs + l, hf * 4 + c4)), vv);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[c4 * 8 + e] = fmaf(wcoef[l], vv[e], acc[c4 * 8 + e]);
-            }
-        }
-        tmem_st32(tmem_addr(tb, q * 32, TM_N + 64 * ch + 32 * hf), acc);
-    }
+    tmem_st32(taddr, w);
 }
 
+// Noisy rows, step 1: block coefficients of this thread's row from [q~;k~]k~^T (TMEM), then the
+// rows of W~ and -Y~ as tensor-memory A operands (TM_R0 columns [0,64) and [64,128)).
 template <int B>
-__device__ __forceinline__ void noisy_phase1(uint8_t *sm, uint32_t tb, int q, int ch, int lane, int rho,
-                                             const float *s_ngam, const float *s_nbeta) {
+__device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int lane, int rho,
+                                              const float *s_ngam, const float *s_nbeta) {
     float wq[32], wk[32];
     tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 32 * q), wq);
     tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 32 * q), wk);
@@ -221,65 +211,94 @@ __device__ __forceinline__ void noisy_phase1(uint8_t *sm, uint32_t tb, int q, in
     const int v = rho >> 6, j = rho & 63;
     float ycoef[B], wcoef[B], gend;
     noisy_coeffs<B>(wq, wk, lane, j, s_ngam + 64 * v, s_nbeta + 64 * v, ycoef, wcoef, gend);
-    noisy_row_build<B>(sm, tb, q, ch, rho, j, v, ycoef, wcoef, gend);
+    bar_math();   // all windows of TM_R0 / TM_R1 are read before TM_R0 is overwritten
+    const int bs = (j / B) * B;
+    store_block_row<B>(tmem_addr(tb, q * 32, TM_R0 + 32 * ch), ch, v, bs, wcoef, 1.f);
+    store_block_row<B>(tmem_addr(tb, q * 32, TM_R0 + 64 + 32 * ch), ch, v, bs, ycoef, -1.f);
+    return gend;
 }
 
-// T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch (in place), blocked in
-// 16x16 tiles: diagonal tiles by forward substitution, then block rows 1..3.
-__device__ void solve_T(float *sa, float *sw, int mw, int lane) {
-    // diagonal blocks: warp I (0..3), lane c < 16 owns column c of D_I = (I + A_II)^{-1}
-    if (mw < 4 && lane < 16) {
-        const int I = mw, c = lane;
-        float x[16];
+// Noisy rows, step 2: Z_j = Gammatil_B q~_j + (-Y~ K~)_j over the q~ row (d columns [64ch, 64ch+64)).
+__device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int ch, int rho, float gend) {
+    const float Gend = exp2f(gend);
+    uint8_t *nq = sm + OFF_NQ + ch * 16384;
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
+    for (int hf = 0; hf < 2; ++hf) {
+        float yk[32];
+        tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32 * hf), yk);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const uint32_t o = sw128_off(rho, 4 * hf + c4);
+            float z[8];
+            unpack8(*reinterpret_cast<const uint4 *>(nq + o), z);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) z[e] = fmaf(Gend, z[e], yk[8 * c4 + e]);
+            *reinterpret_cast<uint4 *>(nq + o) = pack8(z);
+        }
+    }
+}
+
+// One merge level of the triangular inverse: for every pair of S x S diagonal blocks at offset
+// o (already inverted), X = A[o+S.., o..] T[o.., o..] and T[o+S.., o..] = -T[o+S.., o+S..] X.
+template <int S>
+__device__ __forceinline__ void tri_merge(float *sa, float *xb, int tid) {
+    constexpr int NR = S / 8;                  // rows per thread: r0, r0+8, ...
+    const int c = tid % S, r0 = (tid / S) % 8, m = tid / (S * 8), o = m * 2 * S;
+    float *X = xb + m * S * S;
+    float acc[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < S; k += 4) {
+        const float t0 = sa[sidx(o + k, o + c)], t1 = sa[sidx(o + k + 1, o + c)];
+        const float t2 = sa[sidx(o + k + 2, o + c)], t3 = sa[sidx(o + k + 3, o + c)];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const float4 a = *srow4(sa, o + S + r0 + 8 * i, o + k);
+            acc[i] = fmaf(a.x, t0, fmaf(a.y, t1, fmaf(a.z, t2, fmaf(a.w, t3, acc[i]))));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NR; ++i) X[(r0 + 8 * i) * S + c] = acc[i];
+    bar_math();
+#pragma unroll
+    for (int i = 0; i < NR; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < S; k += 4) {
+        const float x0 = X[k * S + c], x1 = X[(k + 1) * S + c], x2 = X[(k + 2) * S + c], x3 = X[(k + 3) * S + c];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const float4 t = *srow4(sa, o + S + r0 + 8 * i, o + S + k);
+            acc[i] = fmaf(t.x, x0, fmaf(t.y, x1, fmaf(t.z, x2, fmaf(t.w, x3, acc[i]))));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NR; ++i) sa[sidx(o + S + r0 + 8 * i, o + c)] = -acc[i];
+    bar_math();
+}
+
+// T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch (in place): the eight
+// 8x8 diagonal blocks by forward substitution (one thread per column), then merges 8->16->32->64.
+__device__ void solve_T(float *sa, float *xb, int tid) {
+    if (tid < 64) {
+        const int o = (tid >> 3) * 8, c = tid & 7;
+        float x[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
             float acc = (jj == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int l = 0; l < jj; ++l) acc = fmaf(-sa[sidx(16 * I + jj, 16 * I + l)], x[l], acc);
+            for (int l = 0; l < jj; ++l) acc = fmaf(-sa[sidx(o + jj, o + l)], x[l], acc);
             x[jj] = acc;
         }
-        __syncwarp(0x0000ffffu);
+        __syncwarp();
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) sa[sidx(16 * I + jj, 16 * I + c)] = x[jj];
+        for (int jj = 0; jj < 8; ++jj) sa[sidx(o + jj, o + c)] = x[jj];
     }
     bar_math();
-    // block rows: T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ  (T_JJ = D_J), J < I
-    for (int I = 1; I < 4; ++I) {
-        float t8[8];
-        const int J = mw;
-        const int r = lane >> 1, c0 = (lane & 1) * 8;
-        if (J < I) {
-            float w8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = 0.f;
-            for (int K = J; K < I; ++K) {
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const float a = sa[sidx(16 * I + r, 16 * K + kk)];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) w8[e] = fmaf(a, sa[sidx(16 * K + kk, 16 * J + c0 + e)], w8[e]);
-                }
-            }
-            float *wst = sw + J * 256;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) wst[r * 16 + c0 + e] = w8[e];
-            __syncwarp();
-#pragma unroll
-            for (int e = 0; e < 8; ++e) t8[e] = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-                const float dik = sa[sidx(16 * I + r, 16 * I + kk)];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t8[e] = fmaf(-dik, wst[kk * 16 + c0 + e], t8[e]);
-            }
-        }
-        bar_math();
-        if (J < I) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sa[sidx(16 * I + r, 16 * J + c0 + e)] = t8[e];
-        }
-        bar_math();
-    }
+    tri_merge<8>(sa, xb, tid);
+    tri_merge<16>(sa, xb, tid);
+    tri_merge<32>(sa, xb, tid);
 }
 
 template <int B>
@@ -290,7 +309,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     __shared__ uint64_t bar_a, bar_b, bar_mma;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float s_g[CH], s_gam[CH], s_beta[CH];
+    __shared__ float s_g[CH], s_gam[CH], s_beta[CH], s_E[CH], s_F[CH];
+    __shared__ int s_okw[2];
     __shared__ float s_ng[2 * CH], s_ngam[2 * CH], s_nbeta[2 * CH];
 
     const int tid = threadIdx.x;
@@ -372,8 +392,45 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     const uint32_t a_s0 = smem_u32(sm + OFF_S0), a_qk = smem_u32(sm + OFF_QK), a_v = smem_u32(sm + OFF_V);
     const uint32_t a_kh = smem_u32(sm + OFF_KH), a_y = smem_u32(sm + OFF_Y), a_nq = smem_u32(sm + OFF_NQ);
     const uint32_t a_nk = smem_u32(sm + OFF_NK);
+    // Base shared-memory descriptors; an operand offset of `off` bytes adds off >> 4.
+    const uint64_t dK_qk = make_sdesc(a_qk, 16, 1024);           // [Q;K] K-major (A), K rows (B)
+    const uint64_t dK_nq = make_sdesc(a_nq, 16, 1024);           // [q~;.] / Z, K-major
+    const uint64_t dK_nk = make_sdesc(a_nk, 16, 1024);           // [k~;.] / M'_Z, K-major
+    const uint64_t dK_y = make_sdesc(a_y, 16, 1024);             // [P;T] / [PT;T], K-major A
+    const uint64_t dM_t = make_sdesc(a_y + 8192, 8192, 1024);    // T rows as MN-major B
+    const uint64_t dM_s0 = make_sdesc(a_s0, 16384, 1024);        // S0, MN-major B
+    const uint64_t dM_v = make_sdesc(a_v, 8192, 1024);           // R / U, MN-major B
+    const uint64_t dM_kh = make_sdesc(a_kh, 8192, 1024);         // Khat, MN-major A
+    const uint64_t dM_nv = make_sdesc(smem_u32(sm + OFF_NV), 16384, 1024);  // [v~0;v~1], MN-major B
+    const uint64_t dM_nk = make_sdesc(a_nk, 16384, 1024);        // [k~0;k~1], MN-major B
     float *scratch = reinterpret_cast<float *>(sm + OFF_Y);
     float *wstage = reinterpret_cast<float *>(sm + OFF_W);
+
+    constexpr float kLog2e = 1.4426950408889634f;
+    // gate (log2-scaled) and beta of this thread's row in chunk m of unit Uq: threads 0-63 the
+    // clean rows, threads 64-191 the noisy rows of both views (zero outside the document)
+    auto load_scalars = [&](const Unit &Uq, int mq, float &gv, float &bv) {
+        gv = 0.f;
+        bv = 0.f;
+        const int cst = Uq.s + Uq.prompt + CH * mq;
+        if (tid < CH) {
+            const int tok = cst + tid;
+            if (tok >= Uq.s && tok < Uq.s + Uq.len) {
+                gv = P.g[(int64_t)tok * H + Uq.h] * kLog2e;
+                bv = P.beta[(int64_t)tok * H + Uq.h];
+            }
+        } else if (mq >= 0 && V > 0 && tid < 3 * CH) {
+            const int idx = tid - CH, vw = idx >> 6, jj = idx & 63;
+            const int rr = CH * mq + jj;
+            if (vw < V && rr < Uq.R) {
+                const int64_t row = (int64_t)vw * TR + Uq.roff + rr;
+                gv = P.gn[row * H + Uq.h] * kLog2e;
+                bv = P.betan[row * H + Uq.h];
+            }
+        }
+    };
+    float pf_g = 0.f, pf_b = 0.f;
+    bool pf_valid = false;
 
     for (int u = blockIdx.x; u < P.num_units; u += gridDim.x) {
         const Unit U = make_unit(P, u);
@@ -402,32 +459,49 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             const bool noisy = (m >= 0) && V > 0;
             const bool last = ci == U.nchunks - 1;
             const int cstart = U.s + U.prompt + CH * m;   // global token of chunk row 0
-            // ---- per-chunk scalars: gates, betas, cumulative log-decays ----
+            // ---- per-chunk scalars: betas and cumulative log2-decays (gamma * log2 e) ----
             {
-                if (tid < CH) {
-                    const int tok = cstart + tid;
-                    const bool ok = tok >= U.s && tok < U.s + U.len;
-                    s_g[tid] = ok ? P.g[(int64_t)tok * H + U.h] : 0.f;
-                    s_beta[tid] = ok ? P.beta[(int64_t)tok * H + U.h] : 0.f;
-                } else if (noisy && tid < 3 * CH) {
-                    const int idx = tid - CH, vw = idx >> 6, jj = idx & 63;
-                    const int rr = CH * m + jj;
-                    const bool ok = vw < V && rr < U.R;
-                    const int64_t row = (int64_t)vw * TR + U.roff + rr;
-                    s_ng[idx] = ok ? P.gn[row * H + U.h] : 0.f;
-                    s_nbeta[idx] = ok ? P.betan[row * H + U.h] : 0.f;
+                float gv, bv;
+                if (pf_valid) {
+                    gv = pf_g;
+                    bv = pf_b;
+                } else {
+                    load_scalars(U, m, gv, bv);
+                }
+                pf_valid = false;
+                if (!last) {                          // gates of the next chunk: loads in flight meanwhile
+                    load_scalars(U, m + 1, pf_g, pf_b);
+                    pf_valid = true;
+                }
+                if (tid < CH) {                       // clean: inclusive scan over the chunk (2 warps)
+                    s_beta[tid] = bv;
+#pragma unroll
+                    for (int d = 1; d < 32; d <<= 1) {
+                        const float o2 = __shfl_up_sync(0xffffffffu, gv, d);
+                        if (lane >= d) gv += o2;
+                    }
+                    s_g[tid] = gv;                     // per-warp inclusive scan
+                } else if (noisy && tid < 3 * CH) {   // noisy: inclusive scan inside each block
+                    const int idx = tid - CH;
+                    s_nbeta[idx] = bv;
+                    const int jl = (idx & 63) % B;
+#pragma unroll
+                    for (int d = 1; d < 32; d <<= 1) {
+                        const float o2 = __shfl_up_sync(0xffffffffu, gv, d);
+                        if (d < B && jl >= d) gv += o2;
+                    }
+                    s_ngam[idx] = gv;
                 }
                 bar_math();
                 if (tid < CH) {
-                    float acc = 0.f;
-                    for (int i = 0; i <= tid; ++i) acc += s_g[i];
-                    s_gam[tid] = acc;
-                } else if (noisy && tid < 3 * CH) {
-                    const int idx = tid - CH, jj = idx & 63, base = idx - jj;
-                    const int bs = (jj / B) * B;
-                    float acc = 0.f;
-                    for (int i = bs; i <= jj; ++i) acc += s_ng[base + i];
-                    s_ngam[idx] = acc;
+                    const float gm = s_g[tid] + (tid >= 32 ? s_g[31] : 0.f);
+                    s_gam[tid] = gm;
+                    s_E[tid] = exp2f(gm);
+                    s_F[tid] = exp2f(-gm);
+                    // e^{gamma_t - gamma_i} = E_t F_i is used only while every |gamma| of the chunk is
+                    // far from the fp32 exponent range; otherwise the difference is exponentiated.
+                    const bool okf = __all_sync(0xffffffffu, fabsf(gm) < 100.f);
+                    if (lane == 0) s_okw[tid >> 5] = okf;
                 }
             }
             // ---- wait for this chunk's tiles ----
@@ -438,38 +512,66 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             __syncwarp();
             bar_all();
             if (s_abort) break;
+            const bool fact = s_okw[0] && s_okw[1];
+            // e^{gamma_t - gamma_i} (i <= t): a product of per-row factors when safe
+            auto decay = [&](auto F, int t, int i) -> float {
+                if constexpr (decltype(F)::value) return s_E[t] * s_F[i];
+                else return exp2f(fminf(s_gam[t] - s_gam[i], 0.f));
+            };
 
             // ================= PK1 =================
             if (tid == 0) {
                 tc_fence_after();
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tb + TM_TK, make_sdesc(a_qk + off, 16, 1024), make_sdesc(a_qk + 8192 + off, 16, 1024),
+                    mma_bf16(tb + TM_TK, dK_qk + (off >> 4), dK_qk + ((8192 + off) >> 4),
                              make_idesc_bf16(128, 64, 0, 0), kk > 0);
                 }
                 if (noisy) {
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_bf16(tb + TM_R0, make_sdesc(a_nq + off, 16, 1024), make_sdesc(a_nk + off, 16, 1024),
+                        mma_bf16(tb + TM_R0, dK_nq + (off >> 4), dK_nk + (off >> 4),
                                  make_idesc_bf16(128, 128, 0, 0), kk > 0);
-                        mma_bf16(tb + TM_R1, make_sdesc(a_nk + off, 16, 1024), make_sdesc(a_nk + off, 16, 1024),
+                        mma_bf16(tb + TM_R1, dK_nk + (off >> 4), dK_nk + (off >> 4),
                                  make_idesc_bf16(128, 128, 0, 0), kk > 0);
                     }
                 }
                 mma_commit(&bar_mma);
             }
             wait_mma(10);
-            // clean: P rows (lanes 0-63) into registers, A rows (lanes 64-127) into scratch
-            if (rho >= 64) {
+            // clean: P rows (lanes 0-63, bf16 packed in registers until the solve is done) and
+            // A rows (lanes 64-127) into the fp32 scratch
+            uint4 ppk[4];
+            {
                 float tk[32];
                 tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), tk);
                 tmem_wait_ld();
-                const int t = rho - 64;
-                const float gt = s_gam[t], bt = s_beta[t];
+                if (rho < 64) {
+                    const int t = rho;
+                    auto body = [&](auto F) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int i = 32 * ch + c;
-                    scratch[sidx(t, i)] = (i < t) ? bt * expf(fminf(gt - s_gam[i], 0.f)) * tk[c] : 0.f;
+                        for (int c = 0; c < 32; ++c) {
+                            const int i = 32 * ch + c;
+                            tk[c] = (i <= t) ? tk[c] * decay(F, t, i) : 0.f;
+                        }
+                    };
+                    if (fact) body(std::true_type{}); else body(std::false_type{});
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) ppk[c4] = pack8(tk + 8 * c4);
+                } else {
+                    const int t = rho - 64;
+                    const float bt = s_beta[t];
+                    auto body = [&](auto F) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int i = 32 * ch + c;
+                            tk[c] = (i < t) ? bt * decay(F, t, i) * tk[c] : 0.f;
+                        }
+                    };
+                    if (fact) body(std::true_type{}); else body(std::false_type{});
+#pragma unroll
+                    for (int g4 = 0; g4 < 8; ++g4)
+                        *srow4(scratch, t, 32 * ch + 4 * g4) = make_float4(tk[4 * g4], tk[4 * g4 + 1], tk[4 * g4 + 2], tk[4 * g4 + 3]);
                 }
             }
             // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout)
@@ -478,42 +580,46 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 const int t = it >> 4, c16 = it & 15, hf = c16 >> 3, c8 = c16 & 7;
                 float f[8];
                 unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QK + hf * 16384 + sw128_off(64 + t, c8)), f);
-                const float sc = expf(fminf(gC - s_gam[t], 0.f));
+                const float sc = fact ? s_E[CH - 1] * s_F[t] : exp2f(fminf(gC - s_gam[t], 0.f));
 #pragma unroll
                 for (int e = 0; e < 8; ++e) f[e] *= sc;
                 *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
             }
-            // noisy: block coefficients, Z rows (in place of q~) and W~V~ into TMEM
-            if (noisy) noisy_phase1<B>(sm, tb, q, ch, lane, rho, s_ngam, s_nbeta);
+            // noisy: block coefficients, then W~ and -Y~ rows into TMEM as A operands
+            float gend = 0.f;
+            if (noisy) gend = noisy_phase1<B>(tb, q, ch, lane, rho, s_ngam, s_nbeta);
+            tmem_wait_st();
+            tc_fence_before();
             bar_math();
-            solve_T(scratch, wstage, warp, lane);
+            // W~V~ -> TM_N and (-Y~)K~ -> TM_R1 on the tensor cores while the solve runs
+            if (noisy && tid == 0) {
+                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tb + TM_N, tb + TM_R0 + kk * 8, dM_nv + ((kk * 2048) >> 4),
+                                make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tb + TM_R1, tb + TM_R0 + 64 + kk * 8, dM_nk + ((kk * 2048) >> 4),
+                                make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                mma_commit(&bar_mma);
+            }
+            solve_T(scratch, wstage, tid);
             // [P ; T] as bf16 K-major A (128 rows x 64): this thread writes row rho, cols [32ch, 32ch+32)
-            float tv[32];
             if (rho >= 64) {
                 const int t = rho - 64;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) tv[c] = scratch[sidx(t, 32 * ch + c)];
+                for (int g4 = 0; g4 < 4; ++g4) {
+                    const float4 a = *srow4(scratch, t, 32 * ch + 8 * g4);
+                    const float4 b = *srow4(scratch, t, 32 * ch + 8 * g4 + 4);
+                    const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    ppk[g4] = pack8(f);
+                }
             }
             bar_math();
-            if (rho < 64) {
-                // P_ti = e^{gamma_t - gamma_i} q_t.k_i (i <= t), from [Q;K]K^T still in TMEM
-                float pv[32];
-                tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), pv);
-                tmem_wait_ld();
-                const int t = rho;
-                const float gt = s_gam[t];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int i = 32 * ch + c;
-                    pv[c] = (i <= t) ? pv[c] * expf(fminf(gt - s_gam[i], 0.f)) : 0.f;
-                }
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(pv + 8 * c4);
-            } else {
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(tv + 8 * c4);
+            for (int c4 = 0; c4 < 4; ++c4) *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = ppk[c4];
+            if (noisy) {
+                wait_mma(15);
+                z_epilogue(sm, tb, q, ch, rho, gend);
             }
             tmem_wait_st();
             fence_async_smem();
@@ -525,12 +631,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             if (tid == 0) {
                 tc_fence_after();
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tb + TM_TK, make_sdesc(a_y + kk * 32, 16, 1024),
-                             make_sdesc(a_y + 8192 + kk * 2048, 8192, 1024), make_idesc_bf16(128, 64, 0, 1), kk > 0);
+                    mma_bf16(tb + TM_TK, dK_y + ((kk * 32) >> 4),
+                             dM_t + ((kk * 2048) >> 4), make_idesc_bf16(128, 64, 0, 1), kk > 0);
                 if (noisy) {
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_bf16(tb + TM_ZK, make_sdesc(a_nq + off, 16, 1024), make_sdesc(a_qk + 8192 + off, 16, 1024),
+                        mma_bf16(tb + TM_ZK, dK_nq + (off >> 4), dK_qk + ((8192 + off) >> 4),
                                  make_idesc_bf16(128, 64, 0, 0), kk > 0);
                     }
                 }
@@ -552,15 +658,18 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 const int jj = rho & 63;
                 const int e = (jj / B) * B - 1;          // chunk-local boundary row (-1: S0)
                 const float ge = e >= 0 ? s_gam[e] : 0.f;
+                auto body = [&](auto F) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int i = 32 * ch + c;
-                    zk[c] = (i <= e) ? zk[c] * expf(fminf(ge - s_gam[i], 0.f)) : 0.f;
-                }
+                    for (int c = 0; c < 32; ++c) {
+                        const int i = 32 * ch + c;
+                        zk[c] = (i <= e) ? zk[c] * decay(F, e < 0 ? 0 : e, i) : 0.f;
+                    }
+                };
+                if (fact) body(std::true_type{}); else body(std::false_type{});
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
                     *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
-                const float Ge = expf(ge);        // Gamma_e (1 for e = -1)
+                const float Ge = e >= 0 ? s_E[e] : 1.f;        // Gamma_e (1 for e = -1)
                 uint8_t *zrow = sm + OFF_NQ + ch * 16384;
 #pragma unroll
                 for (int c8 = 0; c8 < 8; ++c8) {
@@ -581,13 +690,13 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 tc_fence_after();
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tb + TM_R0, make_sdesc(a_qk + off, 16, 1024), make_sdesc(a_s0 + kk * 2048, 16384, 1024),
+                    mma_bf16(tb + TM_R0, dK_qk + (off >> 4), dM_s0 + ((kk * 2048) >> 4),
                              make_idesc_bf16(128, 128, 0, 1), kk > 0);
                 }
                 if (noisy) {
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_bf16(tb + TM_N, make_sdesc(a_nq + off, 16, 1024), make_sdesc(a_s0 + kk * 2048, 16384, 1024),
+                        mma_bf16(tb + TM_N, dK_nq + (off >> 4), dM_s0 + ((kk * 2048) >> 4),
                                  make_idesc_bf16(128, 128, 0, 1), 1u);
                     }
                 }
@@ -601,7 +710,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             wait_mma(30);
             if (rho >= 64) {
                 const int t = rho - 64;
-                const float bt = s_beta[t], bg = bt * expf(s_gam[t]);
+                const float bt = s_beta[t], bg = bt * s_E[t];
                 uint8_t *vrow = sm + OFF_V + ch * 8192;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -628,7 +737,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             if (tid == 0) {
                 tc_fence_after();
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tb + TM_R1, make_sdesc(a_y + kk * 32, 16, 1024), make_sdesc(a_v + kk * 2048, 8192, 1024),
+                    mma_bf16(tb + TM_R1, dK_y + ((kk * 32) >> 4), dM_v + ((kk * 2048) >> 4),
                              make_idesc_bf16(128, 128, 0, 1), kk > 0);
                 mma_commit(&bar_mma);
             }
@@ -637,7 +746,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 const int t = rho;
                 const int tok = cstart + t;
                 const bool ok = tok >= U.s && tok < U.s + U.len;
-                const float Gt = expf(s_gam[t]);
+                const float Gt = s_E[t];
                 __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(P.out) + ((int64_t)tok * H + U.h) * D + 64 * ch;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -675,11 +784,11 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             if (tid == 0) {
                 tc_fence_after();
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tb + TM_R0, make_sdesc(a_kh + kk * 2048, 8192, 1024), make_sdesc(a_v + kk * 2048, 8192, 1024),
+                    mma_bf16(tb + TM_R0, dM_kh + ((kk * 2048) >> 4), dM_v + ((kk * 2048) >> 4),
                              make_idesc_bf16(128, 128, 1, 1), kk > 0);
                 if (noisy) {
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tb + TM_N, make_sdesc(a_nk + kk * 32, 16, 1024), make_sdesc(a_v + kk * 2048, 8192, 1024),
+                        mma_bf16(tb + TM_N, dK_nk + ((kk * 32) >> 4), dM_v + ((kk * 2048) >> 4),
                                  make_idesc_bf16(128, 128, 0, 1), 1u);
                 }
                 mma_commit(&bar_mma);
@@ -689,7 +798,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 }
             }
             wait_mma(50);
-            const float GC = expf(s_gam[CH - 1]);
+            const float GC = s_E[CH - 1];
             uint8_t *srow = sm + OFF_S0 + ch * 16384;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
