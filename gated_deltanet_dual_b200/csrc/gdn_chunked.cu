@@ -73,6 +73,8 @@ struct Maps {
 
 __device__ __forceinline__ void bar_all() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
 __device__ __forceinline__ void bar_math() { bar_all(); }
+// Warps 1..7 only: work overlapped with an MMA batch that thread 0 (warp 0) is issuing.
+__device__ __forceinline__ void bar_side() { asm volatile("bar.sync 3, %0;" ::"n"(kThreads - 32) : "memory"); }
 
 __device__ __forceinline__ uint4 pack8(const float *f) {
     uint4 r;
@@ -222,11 +224,13 @@ __device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int la
 __device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int ch, int rho, float gend) {
     const float Gend = exp2f(gend);
     uint8_t *nq = sm + OFF_NQ + ch * 16384;
+    float ykb[2][32];
+    tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch), ykb[0]);
+    tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32), ykb[1]);
+    tmem_wait_ld();
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-        float yk[32];
-        tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32 * hf), yk);
-        tmem_wait_ld();
+        float (&yk)[32] = ykb[hf];
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
             const uint32_t o = sw128_off(rho, 4 * hf + c4);
@@ -241,40 +245,54 @@ __device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int 
 
 // One merge level of the triangular inverse: for every pair of S x S diagonal blocks at offset
 // o (already inverted), X = A[o+S.., o..] T[o.., o..] and T[o+S.., o..] = -T[o+S.., o+S..] X.
+// Thread: column c, rows r0 + 8i.  T[o+S.., o+S..] is unit lower triangular, so the second
+// product of row r stops at k = r (the bound is uniform per warp when S = 32).
 template <int S>
 __device__ __forceinline__ void tri_merge(float *sa, float *xb, int tid) {
     constexpr int NR = S / 8;                  // rows per thread: r0, r0+8, ...
     const int c = tid % S, r0 = (tid / S) % 8, m = tid / (S * 8), o = m * 2 * S;
     float *X = xb + m * S * S;
-    float acc[NR];
+    float acc[NR], acc2[NR];
 #pragma unroll
-    for (int i = 0; i < NR; ++i) acc[i] = 0.f;
+    for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
 #pragma unroll
-    for (int k = 0; k < S; k += 4) {
-        const float t0 = sa[sidx(o + k, o + c)], t1 = sa[sidx(o + k + 1, o + c)];
-        const float t2 = sa[sidx(o + k + 2, o + c)], t3 = sa[sidx(o + k + 3, o + c)];
+    for (int k = 0; k < S; k += 8) {
+        float t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = sa[sidx(o + k + e, o + c)];
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
             const float4 a = *srow4(sa, o + S + r0 + 8 * i, o + k);
-            acc[i] = fmaf(a.x, t0, fmaf(a.y, t1, fmaf(a.z, t2, fmaf(a.w, t3, acc[i]))));
+            const float4 b = *srow4(sa, o + S + r0 + 8 * i, o + k + 4);
+            acc[i] = fmaf(a.x, t[0], fmaf(a.y, t[1], fmaf(a.z, t[2], fmaf(a.w, t[3], acc[i]))));
+            acc2[i] = fmaf(b.x, t[4], fmaf(b.y, t[5], fmaf(b.z, t[6], fmaf(b.w, t[7], acc2[i]))));
         }
     }
 #pragma unroll
-    for (int i = 0; i < NR; ++i) X[(r0 + 8 * i) * S + c] = acc[i];
+    for (int i = 0; i < NR; ++i) X[(r0 + 8 * i) * S + c] = acc[i] + acc2[i];
     bar_math();
+    const int rmax = r0 | (32 / S - 1);        // largest r0 in this warp
 #pragma unroll
-    for (int i = 0; i < NR; ++i) acc[i] = 0.f;
+    for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
 #pragma unroll
-    for (int k = 0; k < S; k += 4) {
-        const float x0 = X[k * S + c], x1 = X[(k + 1) * S + c], x2 = X[(k + 2) * S + c], x3 = X[(k + 3) * S + c];
+    for (int k = 0; k < S; k += 8) {
+        if (k <= rmax + 8 * (NR - 1)) {
+            float x[8];
 #pragma unroll
-        for (int i = 0; i < NR; ++i) {
-            const float4 t = *srow4(sa, o + S + r0 + 8 * i, o + S + k);
-            acc[i] = fmaf(t.x, x0, fmaf(t.y, x1, fmaf(t.z, x2, fmaf(t.w, x3, acc[i]))));
+            for (int e = 0; e < 8; ++e) x[e] = X[(k + e) * S + c];
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+                if (k <= rmax + 8 * i) {
+                    const float4 a = *srow4(sa, o + S + r0 + 8 * i, o + S + k);
+                    const float4 b = *srow4(sa, o + S + r0 + 8 * i, o + S + k + 4);
+                    acc[i] = fmaf(a.x, x[0], fmaf(a.y, x[1], fmaf(a.z, x[2], fmaf(a.w, x[3], acc[i]))));
+                    acc2[i] = fmaf(b.x, x[4], fmaf(b.y, x[5], fmaf(b.z, x[6], fmaf(b.w, x[7], acc2[i]))));
+                }
+            }
         }
     }
 #pragma unroll
-    for (int i = 0; i < NR; ++i) sa[sidx(o + S + r0 + 8 * i, o + c)] = -acc[i];
+    for (int i = 0; i < NR; ++i) sa[sidx(o + S + r0 + 8 * i, o + c)] = -(acc[i] + acc2[i]);
     bar_math();
 }
 
@@ -309,9 +327,13 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     __shared__ uint64_t bar_a, bar_b, bar_mma;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float s_g[CH], s_gam[CH], s_beta[CH], s_E[CH], s_F[CH];
-    __shared__ int s_okw[2];
-    __shared__ float s_ng[2 * CH], s_ngam[2 * CH], s_nbeta[2 * CH];
+    // Per-chunk scalars, double-buffered so the next chunk's are prepared while this chunk's
+    // state phases run: [buffer][gamma | beta | E = 2^gamma | F = 2^-gamma | noisy gamma | noisy beta]
+    constexpr int SC_GAM = 0, SC_BETA = CH, SC_E = 2 * CH, SC_F = 3 * CH, SC_NGAM = 4 * CH, SC_NBETA = 6 * CH;
+    __shared__ float s_sc[2][8 * CH];
+    __shared__ int s_okw[2][2];
+    __shared__ float s_g[CH];                 // scan scratch
+    __shared__ float s_raw[2][2][3 * CH];     // [buffer][gate, beta][row]: cp.async staging
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -407,30 +429,82 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     float *wstage = reinterpret_cast<float *>(sm + OFF_W);
 
     constexpr float kLog2e = 1.4426950408889634f;
-    // gate (log2-scaled) and beta of this thread's row in chunk m of unit Uq: threads 0-63 the
-    // clean rows, threads 64-191 the noisy rows of both views (zero outside the document)
-    auto load_scalars = [&](const Unit &Uq, int mq, float &gv, float &bv) {
-        gv = 0.f;
-        bv = 0.f;
-        const int cst = Uq.s + Uq.prompt + CH * mq;
-        if (tid < CH) {
-            const int tok = cst + tid;
+    // Stage (cp.async) the gate and beta of this thread's row in chunk mq of unit Uq into buffer
+    // `buf`: threads 0-63 the clean rows, threads 64-191 the noisy rows of both views; rows
+    // outside the document read as 0.
+    // Rows are handled by warps 1..6 (sr = tid - 32): sr 0-63 the clean rows, sr 64-191 the noisy
+    // rows of both views.
+    const int sr = tid - 32;
+    auto stage_scalars = [&](const Unit &Uq, int mq, int buf) {
+        if (sr < 0 || sr >= 3 * CH) return;
+        const float *gp = P.g, *bp = P.beta;
+        uint32_t nb = 0;
+        if (sr < CH) {
+            const int tok = Uq.s + Uq.prompt + CH * mq + sr;
             if (tok >= Uq.s && tok < Uq.s + Uq.len) {
-                gv = P.g[(int64_t)tok * H + Uq.h] * kLog2e;
-                bv = P.beta[(int64_t)tok * H + Uq.h];
+                gp = P.g + (int64_t)tok * H + Uq.h;
+                bp = P.beta + (int64_t)tok * H + Uq.h;
+                nb = 4;
             }
-        } else if (mq >= 0 && V > 0 && tid < 3 * CH) {
-            const int idx = tid - CH, vw = idx >> 6, jj = idx & 63;
+        } else if (mq >= 0 && V > 0) {
+            const int idx = sr - CH, vw = idx >> 6, jj = idx & 63;
             const int rr = CH * mq + jj;
             if (vw < V && rr < Uq.R) {
                 const int64_t row = (int64_t)vw * TR + Uq.roff + rr;
-                gv = P.gn[row * H + Uq.h] * kLog2e;
-                bv = P.betan[row * H + Uq.h];
+                gp = P.gn + row * H + Uq.h;
+                bp = P.betan + row * H + Uq.h;
+                nb = 4;
             }
         }
+        cp_async4(&s_raw[buf][0][sr], gp, nb);
+        cp_async4(&s_raw[buf][1][sr], bp, nb);
+        cp_async_commit();
     };
-    float pf_g = 0.f, pf_b = 0.f;
-    bool pf_valid = false;
+    int rb = 0;      // s_raw buffer holding the next chunk to prepare
+    int cb = 0;      // s_sc buffer of the current chunk
+    // Scan the staged gates of chunk mq into scalar buffer `buf` (cumulative log2-decays, betas,
+    // per-row factors) and stage the gates of chunk mq+1.  Called by all threads.
+    auto prep_scalars = [&](const Unit &Uq, int mq, int buf) {   // warps 1..7 only
+        cp_async_wait_all();
+        float gv = 0.f, bv = 0.f;
+        if (sr < 3 * CH) {
+            gv = s_raw[rb][0][sr] * kLog2e;
+            bv = s_raw[rb][1][sr];
+        }
+        rb ^= 1;
+        if (mq + 1 < Uq.m_first + Uq.nchunks) stage_scalars(Uq, mq + 1, rb);
+        float *sc = s_sc[buf];
+        if (sr < CH) {                        // clean: inclusive scan over the chunk (warps 1, 2)
+            sc[SC_BETA + sr] = bv;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const float o2 = __shfl_up_sync(0xffffffffu, gv, d);
+                if (lane >= d) gv += o2;
+            }
+            s_g[sr] = gv;                      // per-warp inclusive scan
+        } else if (mq >= 0 && V > 0 && sr < 3 * CH) {   // noisy: inclusive scan inside each block
+            const int idx = sr - CH;
+            sc[SC_NBETA + idx] = bv;
+            const int jl = (idx & 63) % B;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const float o2 = __shfl_up_sync(0xffffffffu, gv, d);
+                if (d < B && jl >= d) gv += o2;
+            }
+            sc[SC_NGAM + idx] = gv;
+        }
+        bar_side();
+        if (sr < CH) {
+            const float gm = s_g[sr] + (sr >= 32 ? s_g[31] : 0.f);
+            sc[SC_GAM + sr] = gm;
+            sc[SC_E + sr] = exp2f(gm);
+            sc[SC_F + sr] = exp2f(-gm);
+            // e^{gamma_t - gamma_i} = E_t F_i is used only while every |gamma| of the chunk is
+            // far from the fp32 exponent range; otherwise the difference is exponentiated.
+            const bool okf = __all_sync(0xffffffffu, fabsf(gm) < 100.f);
+            if (lane == 0) s_okw[buf][sr >> 5] = okf;
+        }
+    };
 
     for (int u = blockIdx.x; u < P.num_units; u += gridDim.x) {
         const Unit U = make_unit(P, u);
@@ -459,50 +533,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             const bool noisy = (m >= 0) && V > 0;
             const bool last = ci == U.nchunks - 1;
             const int cstart = U.s + U.prompt + CH * m;   // global token of chunk row 0
-            // ---- per-chunk scalars: betas and cumulative log2-decays (gamma * log2 e) ----
-            {
-                float gv, bv;
-                if (pf_valid) {
-                    gv = pf_g;
-                    bv = pf_b;
-                } else {
-                    load_scalars(U, m, gv, bv);
-                }
-                pf_valid = false;
-                if (!last) {                          // gates of the next chunk: loads in flight meanwhile
-                    load_scalars(U, m + 1, pf_g, pf_b);
-                    pf_valid = true;
-                }
-                if (tid < CH) {                       // clean: inclusive scan over the chunk (2 warps)
-                    s_beta[tid] = bv;
-#pragma unroll
-                    for (int d = 1; d < 32; d <<= 1) {
-                        const float o2 = __shfl_up_sync(0xffffffffu, gv, d);
-                        if (lane >= d) gv += o2;
-                    }
-                    s_g[tid] = gv;                     // per-warp inclusive scan
-                } else if (noisy && tid < 3 * CH) {   // noisy: inclusive scan inside each block
-                    const int idx = tid - CH;
-                    s_nbeta[idx] = bv;
-                    const int jl = (idx & 63) % B;
-#pragma unroll
-                    for (int d = 1; d < 32; d <<= 1) {
-                        const float o2 = __shfl_up_sync(0xffffffffu, gv, d);
-                        if (d < B && jl >= d) gv += o2;
-                    }
-                    s_ngam[idx] = gv;
-                }
-                bar_math();
-                if (tid < CH) {
-                    const float gm = s_g[tid] + (tid >= 32 ? s_g[31] : 0.f);
-                    s_gam[tid] = gm;
-                    s_E[tid] = exp2f(gm);
-                    s_F[tid] = exp2f(-gm);
-                    // e^{gamma_t - gamma_i} = E_t F_i is used only while every |gamma| of the chunk is
-                    // far from the fp32 exponent range; otherwise the difference is exponentiated.
-                    const bool okf = __all_sync(0xffffffffu, fabsf(gm) < 100.f);
-                    if (lane == 0) s_okw[tid >> 5] = okf;
-                }
+            float *s_gam = s_sc[cb] + SC_GAM, *s_beta = s_sc[cb] + SC_BETA;
+            float *s_E = s_sc[cb] + SC_E, *s_F = s_sc[cb] + SC_F;
+            float *s_ngam = s_sc[cb] + SC_NGAM, *s_nbeta = s_sc[cb] + SC_NBETA;
+            if (ci == 0 && warp > 0) {
+                stage_scalars(U, m, rb);
+                prep_scalars(U, m, cb);
             }
             // ---- wait for this chunk's tiles ----
             if (!mbar_wait(&bar_a, ph_a & 1, kWaitIters)) fail(1);
@@ -512,7 +548,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             __syncwarp();
             bar_all();
             if (s_abort) break;
-            const bool fact = s_okw[0] && s_okw[1];
+            const bool fact = s_okw[cb][0] && s_okw[cb][1];
             // e^{gamma_t - gamma_i} (i <= t): a product of per-row factors when safe
             auto decay = [&](auto F, int t, int i) -> float {
                 if constexpr (decltype(F)::value) return s_E[t] * s_F[i];
@@ -537,6 +573,17 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     }
                 }
                 mma_commit(&bar_mma);
+            }
+            // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout)
+            const float gC = s_gam[CH - 1];
+            for (int it = tid - 32; it >= 0 && it < 64 * 16; it += kMathThreads - 32) {   // warps 1..7
+                const int t = it >> 4, c16 = it & 15, hf = c16 >> 3, c8 = c16 & 7;
+                float f[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QK + hf * 16384 + sw128_off(64 + t, c8)), f);
+                const float sc = fact ? s_E[CH - 1] * s_F[t] : exp2f(fminf(gC - s_gam[t], 0.f));
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] *= sc;
+                *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
             }
             wait_mma(10);
             // clean: P rows (lanes 0-63, bf16 packed in registers until the solve is done) and
@@ -573,17 +620,6 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     for (int g4 = 0; g4 < 8; ++g4)
                         *srow4(scratch, t, 32 * ch + 4 * g4) = make_float4(tk[4 * g4], tk[4 * g4 + 1], tk[4 * g4 + 2], tk[4 * g4 + 3]);
                 }
-            }
-            // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout)
-            const float gC = s_gam[CH - 1];
-            for (int it = tid; it < 64 * 16; it += kMathThreads) {
-                const int t = it >> 4, c16 = it & 15, hf = c16 >> 3, c8 = c16 & 7;
-                float f[8];
-                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QK + hf * 16384 + sw128_off(64 + t, c8)), f);
-                const float sc = fact ? s_E[CH - 1] * s_F[t] : exp2f(fminf(gC - s_gam[t], 0.f));
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] *= sc;
-                *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
             }
             // noisy: block coefficients, then W~ and -Y~ rows into TMEM as A operands
             float gend = 0.f;
@@ -657,7 +693,6 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 tmem_wait_ld();
                 const int jj = rho & 63;
                 const int e = (jj / B) * B - 1;          // chunk-local boundary row (-1: S0)
-                const float ge = e >= 0 ? s_gam[e] : 0.f;
                 auto body = [&](auto F) {
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
@@ -707,16 +742,19 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     else issue_a(U, m + 1);
                 }
             }
+            if (!last && warp > 0) prep_scalars(U, m + 1, cb ^ 1);   // next chunk's scalars while S1 runs
             wait_mma(30);
             if (rho >= 64) {
                 const int t = rho - 64;
                 const float bt = s_beta[t], bg = bt * s_E[t];
                 uint8_t *vrow = sm + OFF_V + ch * 8192;
+                float ksb[2][32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch), ksb[0]);
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32), ksb[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    float ks[32];
-                    tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32 * hf), ks);
-                    tmem_wait_ld();
+                    float (&ks)[32] = ksb[hf];
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         float f[8];
@@ -765,11 +803,13 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             } else {
                 const int t = rho - 64;
                 uint8_t *vrow = sm + OFF_V + ch * 8192;
+                float uub[2][32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch), uub[0]);
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32), uub[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    float uu[32];
-                    tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32 * hf), uu);
-                    tmem_wait_ld();
+                    float (&uu)[32] = uub[hf];
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4)
                         *reinterpret_cast<uint4 *>(vrow + sw128_off(t, 4 * hf + c4)) = pack8(uu + 8 * c4);
@@ -800,13 +840,16 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             wait_mma(50);
             const float GC = s_E[CH - 1];
             uint8_t *srow = sm + OFF_S0 + ch * 16384;
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float ds[32];
-                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32 * hf), ds);
+            {
+                float ds0[32], ds1[32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch), ds0);
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32), ds1);
                 tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 32; ++x) S[32 * hf + x] = fmaf(GC, S[32 * hf + x], ds[x]);
+                for (int x = 0; x < 32; ++x) {
+                    S[x] = fmaf(GC, S[x], ds0[x]);
+                    S[32 + x] = fmaf(GC, S[32 + x], ds1[x]);
+                }
             }
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8)
@@ -823,11 +866,13 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 const bool ok = vw < V && rr < U.R;
                 __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(P.out_noisy) +
                                       (((int64_t)vw * TR + U.roff + rr) * H + U.h) * D + 64 * ch;
+                float onb[2][32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_N + 64 * ch), onb[0]);
+                tmem_ld32(tmem_addr(tb, q * 32, TM_N + 64 * ch + 32), onb[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    float on[32];
-                    tmem_ld32(tmem_addr(tb, q * 32, TM_N + 64 * ch + 32 * hf), on);
-                    tmem_wait_ld();
+                    float (&on)[32] = onb[hf];
 #pragma unroll
                     for (int x = 0; x < 32; ++x) on[x] *= scale;
                     if (ok) {
@@ -840,6 +885,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             fence_async_smem();
             tc_fence_before();
             bar_all();
+            cb ^= 1;
             if (s_abort) break;
         }
         if (s_abort) break;
