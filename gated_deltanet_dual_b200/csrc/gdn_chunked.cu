@@ -202,7 +202,7 @@ __device__ __forceinline__ void store_block_row(uint32_t taddr, int ch, int v, i
 }
 
 // Noisy rows, step 1: block coefficients of this thread's row from [q~;k~]k~^T (TMEM), then the
-// rows of W~ and -Y~ as tensor-memory A operands (TM_R0 columns [0,64) and [64,128)).
+// rows of W~ and -Y~ as tensor-memory A operands (columns [0,64) and [64,128) from TM_TK).
 template <int B>
 __device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int lane, int rho,
                                               const float *s_ngam, const float *s_nbeta) {
@@ -213,10 +213,10 @@ __device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int la
     const int v = rho >> 6, j = rho & 63;
     float ycoef[B], wcoef[B], gend;
     noisy_coeffs<B>(wq, wk, lane, j, s_ngam + 64 * v, s_nbeta + 64 * v, ycoef, wcoef, gend);
-    bar_math();   // all windows of TM_R0 / TM_R1 are read before TM_R0 is overwritten
+    bar_math();   // every warp has finished reading TM_TK before it is overwritten
     const int bs = (j / B) * B;
-    store_block_row<B>(tmem_addr(tb, q * 32, TM_R0 + 32 * ch), ch, v, bs, wcoef, 1.f);
-    store_block_row<B>(tmem_addr(tb, q * 32, TM_R0 + 64 + 32 * ch), ch, v, bs, ycoef, -1.f);
+    store_block_row<B>(tmem_addr(tb, q * 32, TM_TK + 32 * ch), ch, v, bs, wcoef, 1.f);
+    store_block_row<B>(tmem_addr(tb, q * 32, TM_TK + 64 + 32 * ch), ch, v, bs, ycoef, -1.f);
     return gend;
 }
 
@@ -245,78 +245,88 @@ __device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int 
 
 // One merge level of the triangular inverse: for every pair of S x S diagonal blocks at offset
 // o (already inverted), X = A[o+S.., o..] T[o.., o..] and T[o+S.., o..] = -T[o+S.., o+S..] X.
-// Thread: column c, rows r0 + 8i.  T[o+S.., o+S..] is unit lower triangular, so the second
-// product of row r stops at k = r (the bound is uniform per warp when S = 32).
-template <int S>
-__device__ __forceinline__ void tri_merge(float *sa, float *xb, int tid) {
-    constexpr int NR = S / 8;                  // rows per thread: r0, r0+8, ...
-    const int c = tid % S, r0 = (tid / S) % 8, m = tid / (S * 8), o = m * 2 * S;
+// NT threads (t = 0..NT-1 when `active`): column c, rows g + RG*i.  T[o+S.., o+S..] is unit lower
+// triangular, so the second product of row r stops at k = r.  `side`: barrier of warps 1..7.
+template <int S, int NT>
+__device__ __forceinline__ void tri_merge(float *sa, float *xb, int t, bool active, bool side) {
+    constexpr int RG = NT / 32;                // row groups per merge
+    constexpr int NR = S / RG;                 // rows per thread
+    const int c = t % S, g = (t / S) % RG, m = t / (S * RG), o = m * 2 * S;
     float *X = xb + m * S * S;
     float acc[NR], acc2[NR];
+    if (active) {
 #pragma unroll
-    for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
+        for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
 #pragma unroll
-    for (int k = 0; k < S; k += 8) {
-        float t[8];
+        for (int k = 0; k < S; k += 8) {
+            float tv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = sa[sidx(o + k + e, o + c)];
-#pragma unroll
-        for (int i = 0; i < NR; ++i) {
-            const float4 a = *srow4(sa, o + S + r0 + 8 * i, o + k);
-            const float4 b = *srow4(sa, o + S + r0 + 8 * i, o + k + 4);
-            acc[i] = fmaf(a.x, t[0], fmaf(a.y, t[1], fmaf(a.z, t[2], fmaf(a.w, t[3], acc[i]))));
-            acc2[i] = fmaf(b.x, t[4], fmaf(b.y, t[5], fmaf(b.z, t[6], fmaf(b.w, t[7], acc2[i]))));
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < NR; ++i) X[(r0 + 8 * i) * S + c] = acc[i] + acc2[i];
-    bar_math();
-    const int rmax = r0 | (32 / S - 1);        // largest r0 in this warp
-#pragma unroll
-    for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
-#pragma unroll
-    for (int k = 0; k < S; k += 8) {
-        if (k <= rmax + 8 * (NR - 1)) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = X[(k + e) * S + c];
+            for (int e = 0; e < 8; ++e) tv[e] = sa[sidx(o + k + e, o + c)];
 #pragma unroll
             for (int i = 0; i < NR; ++i) {
-                if (k <= rmax + 8 * i) {
-                    const float4 a = *srow4(sa, o + S + r0 + 8 * i, o + S + k);
-                    const float4 b = *srow4(sa, o + S + r0 + 8 * i, o + S + k + 4);
-                    acc[i] = fmaf(a.x, x[0], fmaf(a.y, x[1], fmaf(a.z, x[2], fmaf(a.w, x[3], acc[i]))));
-                    acc2[i] = fmaf(b.x, x[4], fmaf(b.y, x[5], fmaf(b.z, x[6], fmaf(b.w, x[7], acc2[i]))));
+                const float4 a = *srow4(sa, o + S + g + RG * i, o + k);
+                const float4 b = *srow4(sa, o + S + g + RG * i, o + k + 4);
+                acc[i] = fmaf(a.x, tv[0], fmaf(a.y, tv[1], fmaf(a.z, tv[2], fmaf(a.w, tv[3], acc[i]))));
+                acc2[i] = fmaf(b.x, tv[4], fmaf(b.y, tv[5], fmaf(b.z, tv[6], fmaf(b.w, tv[7], acc2[i]))));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < NR; ++i) X[(g + RG * i) * S + c] = acc[i] + acc2[i];
+    }
+    if (side) bar_side(); else bar_math();
+    if (active) {
+        const int gmax = g | (32 / S - 1);     // largest row group in this warp
+#pragma unroll
+        for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < S; k += 8) {
+            if (k <= gmax + RG * (NR - 1)) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = X[(k + e) * S + c];
+#pragma unroll
+                for (int i = 0; i < NR; ++i) {
+                    if (k <= gmax + RG * i) {
+                        const float4 a = *srow4(sa, o + S + g + RG * i, o + S + k);
+                        const float4 b = *srow4(sa, o + S + g + RG * i, o + S + k + 4);
+                        acc[i] = fmaf(a.x, x[0], fmaf(a.y, x[1], fmaf(a.z, x[2], fmaf(a.w, x[3], acc[i]))));
+                        acc2[i] = fmaf(b.x, x[4], fmaf(b.y, x[5], fmaf(b.z, x[6], fmaf(b.w, x[7], acc2[i]))));
+                    }
                 }
             }
         }
-    }
 #pragma unroll
-    for (int i = 0; i < NR; ++i) sa[sidx(o + S + r0 + 8 * i, o + c)] = -(acc[i] + acc2[i]);
-    bar_math();
+        for (int i = 0; i < NR; ++i) sa[sidx(o + S + g + RG * i, o + c)] = -(acc[i] + acc2[i]);
+    }
+    if (side) bar_side(); else bar_math();
 }
 
 // T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch (in place): the eight
-// 8x8 diagonal blocks by forward substitution (one thread per column), then merges 8->16->32->64.
-__device__ void solve_T(float *sa, float *xb, int tid) {
-    if (tid < 64) {
-        const int o = (tid >> 3) * 8, c = tid & 7;
-        float x[8];
+// 8x8 diagonal blocks by forward substitution (one thread per column) and the 8- and 16-merges on
+// warps 1..7 (warp 0 is issuing an MMA batch meanwhile), then the 32-merge on all warps.
+__device__ void solve_T(float *sa, float *xb, int tid, int warp) {
+    if (warp > 0) {
+        const int t = tid - 32;
+        if (t < 64) {
+            const int o = (t >> 3) * 8, c = t & 7;
+            float x[8];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-            float acc = (jj == c) ? 1.f : 0.f;
+            for (int jj = 0; jj < 8; ++jj) {
+                float acc = (jj == c) ? 1.f : 0.f;
 #pragma unroll
-            for (int l = 0; l < jj; ++l) acc = fmaf(-sa[sidx(o + jj, o + l)], x[l], acc);
-            x[jj] = acc;
+                for (int l = 0; l < jj; ++l) acc = fmaf(-sa[sidx(o + jj, o + l)], x[l], acc);
+                x[jj] = acc;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) sa[sidx(o + jj, o + c)] = x[jj];
         }
-        __syncwarp();
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) sa[sidx(o + jj, o + c)] = x[jj];
+        bar_side();
+        tri_merge<8, 128>(sa, xb, t, t < 128, true);
+        tri_merge<16, 128>(sa, xb, t, t < 128, true);
     }
     bar_math();
-    tri_merge<8>(sa, xb, tid);
-    tri_merge<16>(sa, xb, tid);
-    tri_merge<32>(sa, xb, tid);
+    tri_merge<32, 256>(sa, xb, tid, true, false);
 }
 
 template <int B>
@@ -324,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps M) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_a, bar_b, bar_mma;
+    __shared__ uint64_t bar_a, bar_b, bar_mma, bar_mma2;   // bar_mma2: the noisy half of PK1 only
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     // Per-chunk scalars, double-buffered so the next chunk's are prepared while this chunk's
@@ -346,6 +356,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
         mbar_init(&bar_mma, 1);
+        mbar_init(&bar_mma2, 1);
         fence_mbar_init();
         s_abort = 0;
     }
@@ -362,7 +373,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     __syncthreads();
     tc_fence_after();
     const uint32_t tb = s_tmem;
-    uint32_t ph_a = 0, ph_b = 0, ph_mma = 0;
+    // Every mbarrier has at most one outstanding phase when it is waited on, so parities never alias.
+    uint32_t ph_a = 0, ph_b = 0, ph_mma = 0, ph_mma2 = 0;
 
     auto fail = [&](int where) {
         if (atomicExch(&s_abort, 1) == 0) {
@@ -374,6 +386,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(where);
         ++ph_mma;
         __syncwarp();            // reconverge before warp-collective tcgen05.ld/st
+        tc_fence_after();
+    };
+    auto wait_mma2 = [&](int where) {
+        if (!mbar_wait(&bar_mma2, ph_mma2 & 1, kWaitIters)) fail(where);
+        ++ph_mma2;
+        __syncwarp();
         tc_fence_after();
     };
 
@@ -543,8 +561,6 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // ---- wait for this chunk's tiles ----
             if (!mbar_wait(&bar_a, ph_a & 1, kWaitIters)) fail(1);
             ++ph_a;
-            if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
-            ++ph_b;
             __syncwarp();
             bar_all();
             if (s_abort) break;
@@ -555,7 +571,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 else return exp2f(fminf(s_gam[t] - s_gam[i], 0.f));
             };
 
-            // ================= PK1 =================
+            // ================= PK1: [Q;K]K^T now, the noisy products once group B is in ========
             if (tid == 0) {
                 tc_fence_after();
                 for (int kk = 0; kk < 8; ++kk) {
@@ -563,17 +579,9 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     mma_bf16(tb + TM_TK, dK_qk + (off >> 4), dK_qk + ((8192 + off) >> 4),
                              make_idesc_bf16(128, 64, 0, 0), kk > 0);
                 }
-                if (noisy) {
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_bf16(tb + TM_R0, dK_nq + (off >> 4), dK_nk + (off >> 4),
-                                 make_idesc_bf16(128, 128, 0, 0), kk > 0);
-                        mma_bf16(tb + TM_R1, dK_nk + (off >> 4), dK_nk + (off >> 4),
-                                 make_idesc_bf16(128, 128, 0, 0), kk > 0);
-                    }
-                }
                 mma_commit(&bar_mma);
             }
+            __syncwarp();
             // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout)
             const float gC = s_gam[CH - 1];
             for (int it = tid - 32; it >= 0 && it < 64 * 16; it += kMathThreads - 32) {   // warps 1..7
@@ -585,6 +593,20 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 for (int e = 0; e < 8; ++e) f[e] *= sc;
                 *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
             }
+            if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);   // V and [k~0;k~1]
+            ++ph_b;
+            __syncwarp();
+            if (noisy && tid == 0) {
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_bf16(tb + TM_R0, dK_nq + (off >> 4), dK_nk + (off >> 4),
+                             make_idesc_bf16(128, 128, 0, 0), kk > 0);
+                    mma_bf16(tb + TM_R1, dK_nk + (off >> 4), dK_nk + (off >> 4),
+                             make_idesc_bf16(128, 128, 0, 0), kk > 0);
+                }
+                mma_commit(&bar_mma2);
+            }
+            __syncwarp();
             wait_mma(10);
             // clean: P rows (lanes 0-63, bf16 packed in registers until the solve is done) and
             // A rows (lanes 64-127) into the fp32 scratch
@@ -621,24 +643,34 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                         *srow4(scratch, t, 32 * ch + 4 * g4) = make_float4(tk[4 * g4], tk[4 * g4 + 1], tk[4 * g4 + 2], tk[4 * g4 + 3]);
                 }
             }
+            if (noisy) wait_mma2(11);                   // noisy block products of PK1
             // noisy: block coefficients, then W~ and -Y~ rows into TMEM as A operands
             float gend = 0.f;
             if (noisy) gend = noisy_phase1<B>(tb, q, ch, lane, rho, s_ngam, s_nbeta);
             tmem_wait_st();
             tc_fence_before();
             bar_math();
-            // W~V~ -> TM_N and (-Y~)K~ -> TM_R1 on the tensor cores while the solve runs
-            if (noisy && tid == 0) {
+            // On the tensor cores while the solve runs: [Q;K] S0 -> TM_R0 and, for the noisy rows,
+            // W~V~ -> TM_N and (-Y~)K~ -> TM_R1 (A operands in TMEM).
+            if (tid == 0) {
                 tc_fence_after();
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tb + TM_N, tb + TM_R0 + kk * 8, dM_nv + ((kk * 2048) >> 4),
-                                make_idesc_bf16(128, 128, 0, 1), kk > 0);
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tb + TM_R1, tb + TM_R0 + 64 + kk * 8, dM_nk + ((kk * 2048) >> 4),
-                                make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_bf16(tb + TM_R0, dK_qk + (off >> 4), dM_s0 + ((kk * 2048) >> 4),
+                             make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                }
+                if (noisy) {
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tb + TM_N, tb + TM_TK + kk * 8, dM_nv + ((kk * 2048) >> 4),
+                                    make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tb + TM_R1, tb + TM_TK + 64 + kk * 8, dM_nk + ((kk * 2048) >> 4),
+                                    make_idesc_bf16(128, 128, 0, 1), kk > 0);
+                }
                 mma_commit(&bar_mma);
             }
-            solve_T(scratch, wstage, tid);
+            __syncwarp();
+            solve_T(scratch, wstage, tid, warp);
             // [P ; T] as bf16 K-major A (128 rows x 64): this thread writes row rho, cols [32ch, 32ch+32)
             if (rho >= 64) {
                 const int t = rho - 64;
@@ -653,10 +685,31 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             bar_math();
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = ppk[c4];
-            if (noisy) {
-                wait_mma(15);
-                z_epilogue(sm, tb, q, ch, rho, gend);
+            wait_mma(15);
+            // R = beta V - beta Gamma (K S0), over V (K S0 are rows 64..127 of TM_R0)
+            if (rho >= 64) {
+                const int t = rho - 64;
+                const float bt = s_beta[t], bg = bt * s_E[t];
+                uint8_t *vrow = sm + OFF_V + ch * 8192;
+                float ksb[2][32];
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch), ksb[0]);
+                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32), ksb[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    float (&ks)[32] = ksb[hf];
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        float f[8];
+                        const uint32_t o = sw128_off(t, 4 * hf + c4);
+                        unpack8(*reinterpret_cast<const uint4 *>(vrow + o), f);
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) f[x] = bt * f[x] - bg * ks[8 * c4 + x];
+                        *reinterpret_cast<uint4 *>(vrow + o) = pack8(f);
+                    }
+                }
             }
+            if (noisy) z_epilogue(sm, tb, q, ch, rho, gend);
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
@@ -678,6 +731,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 }
                 mma_commit(&bar_mma);
             }
+            __syncwarp();
             wait_mma(20);
             if (rho < 64) {
                 float pt[32];
@@ -720,14 +774,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             bar_all();
             if (s_abort) break;
 
-            // ================= S1 =================
+            // ================= S2: [PT;T] R and the noisy rows' state product =================
             if (tid == 0) {
                 tc_fence_after();
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_bf16(tb + TM_R0, dK_qk + (off >> 4), dM_s0 + ((kk * 2048) >> 4),
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tb + TM_R1, dK_y + ((kk * 32) >> 4), dM_v + ((kk * 2048) >> 4),
                              make_idesc_bf16(128, 128, 0, 1), kk > 0);
-                }
                 if (noisy) {
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -736,49 +788,14 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     }
                 }
                 mma_commit(&bar_mma);
-                // prefetch group A of the next chunk once S1 has consumed [Q;K] and Z
+                // prefetch group A of the next chunk once [Q;K] and Z are consumed
                 if (!last) {
-                    if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(30);
+                    if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(40);
                     else issue_a(U, m + 1);
                 }
             }
-            if (!last && warp > 0) prep_scalars(U, m + 1, cb ^ 1);   // next chunk's scalars while S1 runs
-            wait_mma(30);
-            if (rho >= 64) {
-                const int t = rho - 64;
-                const float bt = s_beta[t], bg = bt * s_E[t];
-                uint8_t *vrow = sm + OFF_V + ch * 8192;
-                float ksb[2][32];
-                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch), ksb[0]);
-                tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32), ksb[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float (&ks)[32] = ksb[hf];
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        float f[8];
-                        const uint32_t o = sw128_off(t, 4 * hf + c4);
-                        unpack8(*reinterpret_cast<const uint4 *>(vrow + o), f);
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) f[x] = bt * f[x] - bg * ks[8 * c4 + x];
-                        *reinterpret_cast<uint4 *>(vrow + o) = pack8(f);
-                    }
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            bar_all();
-            if (s_abort) break;
-
-            // ================= S2 =================
-            if (tid == 0) {
-                tc_fence_after();
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tb + TM_R1, dK_y + ((kk * 32) >> 4), dM_v + ((kk * 2048) >> 4),
-                             make_idesc_bf16(128, 128, 0, 1), kk > 0);
-                mma_commit(&bar_mma);
-            }
+            __syncwarp();
+            if (!last && warp > 0) prep_scalars(U, m + 1, cb ^ 1);   // next chunk's scalars meanwhile
             wait_mma(40);
             if (rho < 64) {
                 const int t = rho;
@@ -837,6 +854,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     else issue_b(U, m + 1);
                 }
             }
+            __syncwarp();
             wait_mma(50);
             const float GC = s_E[CH - 1];
             uint8_t *srow = sm + OFF_S0 + ch * 16384;
