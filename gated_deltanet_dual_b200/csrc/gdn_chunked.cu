@@ -329,6 +329,128 @@ __device__ void solve_T(float *sa, float *xb, int tid, int warp) {
     tri_merge<32, 256>(sa, xb, tid, true, false);
 }
 
+// ----------------------------------------------------------------------------- ShortConv
+// Width-4 depthwise causal conv on q, k, v (Key design 3 of the FLARE notes), applied in place to
+// the chunk's tiles before anything reads them.  Tap 3 is the current token.  Clean taps before
+// the document start read 0; a noisy tap that reaches before its block start reads the clean raw
+// input (rows of this chunk, or the three raw rows carried over from the previous chunk).
+constexpr int OFF_CW = OFF_KH;   // conv weights [q,k,v][128][4] fp32 (6 KB) until K-hat is built
+
+__device__ __forceinline__ uint8_t *clean_at(uint8_t *sm, int X, int r, int cc) {
+    const int hf = cc >> 3, c8 = cc & 7;
+    if (X == 0) return sm + OFF_QK + hf * 16384 + sw128_off(r, c8);
+    if (X == 1) return sm + OFF_QK + hf * 16384 + 8192 + sw128_off(r, c8);
+    return sm + OFF_V + hf * 8192 + sw128_off(r, c8);
+}
+__device__ __forceinline__ uint8_t *noisy_at(uint8_t *sm, int X, int v, int r, int cc) {
+    const int hf = cc >> 3, c8 = cc & 7;
+    const int base = X == 0 ? OFF_NQ : (X == 1 ? OFF_NK : OFF_NV);
+    return sm + base + hf * 16384 + v * 8192 + sw128_off(r, c8);
+}
+// Raw clean row src (>= 0) of the chunk: zero before the document start.
+__device__ __forceinline__ uint4 clean_raw(uint8_t *sm, int X, int src, int cc, int cstart, int s_doc) {
+    return (cstart + src >= s_doc) ? *reinterpret_cast<const uint4 *>(clean_at(sm, X, src, cc)) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Convolve rows r0+15 .. r0 of one 8-channel column in place (descending, a 4-row window).
+// noisy: rows of view v; taps before the row's block start read clean raw rows / the halo.
+template <int B, bool NOISY>
+__device__ __forceinline__ void conv_rows(uint8_t *sm, const float *cw, const uint4 (*halo)[3][16], bool first,
+                                          int X, int v, int cc, int r0, const uint4 (&pre)[3], int cstart,
+                                          int s_doc) {
+    float w[8][4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float4 t = *reinterpret_cast<const float4 *>(cw + (X * 128 + 8 * cc + e) * 4);
+        w[e][0] = t.x; w[e][1] = t.y; w[e][2] = t.z; w[e][3] = t.w;
+    }
+    auto own = [&](int r) -> uint4 {
+        if (NOISY) return *reinterpret_cast<const uint4 *>(noisy_at(sm, X, v, r, cc));
+        return clean_raw(sm, X, r, cc, cstart, s_doc);
+    };
+    auto clean_or_halo = [&](int src) -> uint4 {
+        if (src >= 0) return clean_raw(sm, X, src, cc, cstart, s_doc);
+        return first ? make_uint4(0u, 0u, 0u, 0u) : halo[X][3 + src][cc];
+    };
+    float x[4][8];                 // raw rows t, t-1, t-2, t-3
+#pragma unroll
+    for (int i = 0; i < 4; ++i) unpack8(own(r0 + 15 - i), x[i]);
+#pragma unroll
+    for (int jj = 15; jj >= 0; --jj) {
+        const int t = r0 + jj;
+        float tap[4][8];
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) tap[l][e] = x[l][e];
+        }
+        if (NOISY) {
+            const int bs = t - (t % B);
+#pragma unroll
+            for (int l = 1; l < 4; ++l) {
+                if (t - l < bs) unpack8(clean_or_halo(t - l), tap[l]);
+            }
+        }
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            o[e] = fmaf(w[e][3], tap[0][e], fmaf(w[e][2], tap[1][e], fmaf(w[e][1], tap[2][e], w[e][0] * tap[3][e])));
+        uint8_t *dst = NOISY ? noisy_at(sm, X, v, t, cc) : clean_at(sm, X, t, cc);
+        *reinterpret_cast<uint4 *>(dst) = pack8(o);
+        if (jj > 0) {
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[l][e] = x[l + 1][e];
+            }
+            if (jj - 4 >= 0) unpack8(own(r0 + jj - 4), x[3]);
+            else unpack8(pre[jj - 1], x[3]);
+        }
+    }
+}
+
+// The whole prologue for one chunk (all threads; barriers inside).  Noisy tiles first (they
+// read raw clean rows), then the clean tiles, whose last three raw rows become the next halo.
+template <int B>
+__device__ __noinline__ void conv_chunk(uint8_t *sm, uint4 (*halo)[3][16], bool first, bool noisy, int cstart,
+                                        int s_doc, int tid) {
+    const float *cw = reinterpret_cast<const float *>(sm + OFF_CW);
+    if (noisy) {
+        for (int round = 0; round < 2; ++round) {    // 384 items: (tensor, view, column chunk, segment)
+            const int it = tid + 256 * round;
+            const bool act = it < 384;
+            const int X = it / 128, rem = it % 128, v = rem / 64, cc = (rem % 64) / 4, r0 = 16 * (rem % 4);
+            uint4 pre[3];
+#pragma unroll
+            for (int l = 0; l < 3; ++l)
+                pre[l] = (act && r0 > 0) ? *reinterpret_cast<const uint4 *>(noisy_at(sm, X, v, r0 - 3 + l, cc))
+                                         : make_uint4(0u, 0u, 0u, 0u);
+            bar_math();
+            if (act) conv_rows<B, true>(sm, cw, halo, first, X, v, cc, r0, pre, cstart, s_doc);
+            bar_math();
+        }
+    }
+    const bool act = tid < 192;                         // 192 items: (tensor, column chunk, segment)
+    const int X = tid / 64, cc = (tid % 64) / 4, r0 = 16 * (tid % 4);
+    uint4 pre[3];
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+        const int src = r0 - 3 + l;
+        pre[l] = !act ? make_uint4(0u, 0u, 0u, 0u)
+                      : (src >= 0 ? clean_raw(sm, X, src, cc, cstart, s_doc)
+                                  : (first ? make_uint4(0u, 0u, 0u, 0u) : halo[X][3 + src][cc]));
+    }
+    bar_math();
+    if (act) {
+        if (r0 == 48) {
+#pragma unroll
+            for (int l = 0; l < 3; ++l) halo[X][l][cc] = clean_raw(sm, X, 61 + l, cc, cstart, s_doc);
+        }
+        conv_rows<B, false>(sm, cw, halo, first, X, 0, cc, r0, pre, cstart, s_doc);
+    }
+    bar_math();
+}
+
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps M) {
@@ -343,7 +465,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     __shared__ float s_sc[2][8 * CH];
     __shared__ int s_okw[2][2];
     __shared__ float s_g[CH];                 // scan scratch
-    __shared__ float s_raw[2][2][3 * CH];     // [buffer][gate, beta][row]: cp.async staging
+    __shared__ float s_raw[2][3 * CH];        // [gate, beta][row]: cp.async staging (read before restaged)
+    __shared__ uint4 s_halo[3][3][16];        // ShortConv: raw clean rows cstart-3..cstart-1 [q,k,v][row][chunk]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -351,6 +474,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     const int H = P.H, V = P.V;
     const int64_t TR = P.TR;
     const float scale = P.scale;
+    const bool conv = P.conv_width > 0;
 
     if (tid == 0) {
         mbar_init(&bar_a, 1);
@@ -474,8 +598,9 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 nb = 4;
             }
         }
-        cp_async4(&s_raw[buf][0][sr], gp, nb);
-        cp_async4(&s_raw[buf][1][sr], bp, nb);
+        (void)buf;
+        cp_async4(&s_raw[0][sr], gp, nb);
+        cp_async4(&s_raw[1][sr], bp, nb);
         cp_async_commit();
     };
     int rb = 0;      // s_raw buffer holding the next chunk to prepare
@@ -486,8 +611,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         cp_async_wait_all();
         float gv = 0.f, bv = 0.f;
         if (sr < 3 * CH) {
-            gv = s_raw[rb][0][sr] * kLog2e;
-            bv = s_raw[rb][1][sr];
+            gv = s_raw[0][sr] * kLog2e;
+            bv = s_raw[1][sr];
         }
         rb ^= 1;
         if (mq + 1 < Uq.m_first + Uq.nchunks) stage_scalars(Uq, mq + 1, rb);
@@ -558,9 +683,25 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 stage_scalars(U, m, rb);
                 prep_scalars(U, m, cb);
             }
+            // ---- conv weights of this head (cp.async into the K-hat buffer, free until PE1) ----
+            if (conv) {
+                for (int it = tid; it < 3 * 128 * 4 / 4; it += kThreads) {
+                    const int X = it / 128, c = it % 128;
+                    cp_async16(sm + OFF_CW + it * 16, P.conv_w + (((int64_t)X * H + U.h) * 128 + c) * 4);
+                }
+                cp_async_commit();
+            }
             // ---- wait for this chunk's tiles ----
             if (!mbar_wait(&bar_a, ph_a & 1, kWaitIters)) fail(1);
             ++ph_a;
+            if (conv) {
+                if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
+                ++ph_b;
+                cp_async_wait_all();
+                __syncwarp();
+                bar_all();
+                conv_chunk<B>(sm, s_halo, ci == 0, noisy, cstart, U.s, tid);
+            }
             __syncwarp();
             bar_all();
             if (s_abort) break;
@@ -593,8 +734,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 for (int e = 0; e < 8; ++e) f[e] *= sc;
                 *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
             }
-            if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);   // V and [k~0;k~1]
-            ++ph_b;
+            if (!conv) {                                  // V and [k~0;k~1]
+                if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
+                ++ph_b;
+            }
             __syncwarp();
             if (noisy && tid == 0) {
                 for (int kk = 0; kk < 8; ++kk) {
@@ -942,7 +1085,7 @@ bool encode_map(CUtensorMap *m, const void *ptr, int H, int64_t rows) {
 }  // namespace
 
 bool chunked_supported(int dtype, int d, int B, int conv_width) {
-    return dtype == GDN_BF16 && d == D && conv_width == 0 && B >= 1 && B <= 32 && (32 % B) == 0;
+    return dtype == GDN_BF16 && d == D && (conv_width == 0 || conv_width == 4) && B >= 1 && B <= 32 && (32 % B) == 0;
 }
 
 cudaError_t launch_chunked(const Params &p, cudaStream_t stream) {

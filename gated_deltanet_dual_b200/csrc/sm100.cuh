@@ -63,6 +63,10 @@ __device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t s
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
                  ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
 }
+// 16-byte global -> shared asynchronous copy (both addresses 16-byte aligned).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 

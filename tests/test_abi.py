@@ -173,7 +173,7 @@ def test_valid_arguments_without_device_report_cuda_error():
 def test_auto_selects_tensor_core_kernel_where_supported():
     assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 4, b.GDN_BF16)) == b.ALGO_CHUNKED
     assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 32, b.GDN_BF16)) == b.ALGO_CHUNKED
-    assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 4, b.GDN_BF16, conv_width=4)) == b.ALGO_SEQUENTIAL
+    assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 4, b.GDN_BF16, conv_width=4)) == b.ALGO_CHUNKED
     assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 64, b.GDN_BF16)) == b.ALGO_SEQUENTIAL
     assert b.select_algo(b.make_desc(2, 16, 64, 64, 2, 4, b.GDN_BF16)) == b.ALGO_SEQUENTIAL
     assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 4, b.GDN_FP32)) == b.ALGO_SEQUENTIAL
