@@ -334,121 +334,209 @@ __device__ void solve_T(float *sa, float *xb, int tid, int warp) {
 // the chunk's tiles before anything reads them.  Tap 3 is the current token.  Clean taps before
 // the document start read 0; a noisy tap that reaches before its block start reads the clean raw
 // input (rows of this chunk, or the three raw rows carried over from the previous chunk).
-constexpr int OFF_CW = OFF_KH;   // conv weights [q,k,v][128][4] fp32 (6 KB) until K-hat is built
+//
+// Work item: a few rows (a segment) of one 8-channel column of one tensor.  Lane bits 0-3 pick
+// the column, so the 8 lanes of a shared-memory phase touch 8 distinct 16-byte chunks of one row.
+// Every item reads all its rows into registers before any item of the same round writes, so the
+// in-place update needs one barrier per round at most.  Arithmetic is fp32, two channels per
+// instruction (packed FFMA2), rounded once to bf16.
+constexpr int OFF_CW = OFF_KH;   // conv weights (6 KB) until K-hat is built
 
-__device__ __forceinline__ uint8_t *clean_at(uint8_t *sm, int X, int r, int cc) {
-    const int hf = cc >> 3, c8 = cc & 7;
-    if (X == 0) return sm + OFF_QK + hf * 16384 + sw128_off(r, c8);
-    if (X == 1) return sm + OFF_QK + hf * 16384 + 8192 + sw128_off(r, c8);
-    return sm + OFF_V + hf * 8192 + sw128_off(r, c8);
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
 }
-__device__ __forceinline__ uint8_t *noisy_at(uint8_t *sm, int X, int v, int r, int cc) {
-    const int hf = cc >> 3, c8 = cc & 7;
-    const int base = X == 0 ? OFF_NQ : (X == 1 ? OFF_NK : OFF_NV);
-    return sm + base + hf * 16384 + v * 8192 + sw128_off(r, c8);
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
 }
-// Raw clean row src (>= 0) of the chunk: zero before the document start.
-__device__ __forceinline__ uint4 clean_raw(uint8_t *sm, int X, int src, int cc, int cstart, int s_doc) {
-    return (cstart + src >= s_doc) ? *reinterpret_cast<const uint4 *>(clean_at(sm, X, src, cc)) : make_uint4(0u, 0u, 0u, 0u);
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ float2 bf2_lo_hi(uint32_t w) {   // bf16 pair -> (even channel, odd channel)
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float2 f) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ uint32_t &word_of(uint4 &u, int i) {
+    return i == 0 ? u.x : (i == 1 ? u.y : (i == 2 ? u.z : u.w));
+}
+// Shared address of row r of 8-channel column c8 in a 64-row, 128-byte-swizzled half tile.
+__device__ __forceinline__ uint32_t conv_row(uint32_t half, int r, int c8) {
+    return half + r * 128 + ((c8 ^ (r & 7)) << 4);
+}
+// Byte offset of the half tile (64 channels) holding column half hf of clean tensor X / noisy
+// tensor X of view v.
+__device__ __forceinline__ int clean_half(int X, int hf) {
+    return X == 2 ? OFF_V + hf * 8192 : OFF_QK + hf * 16384 + X * 8192;
+}
+__device__ __forceinline__ int noisy_half(int X, int v, int hf) {
+    return (X == 0 ? OFF_NQ : (X == 1 ? OFF_NK : OFF_NV)) + hf * 16384 + v * 8192;
+}
+// Noisy segment of LEN rows that starts on a block boundary (B <= LEN): is clean row d (relative
+// to the segment start, -3 <= d < LEN - 1) a tap of one of its rows?
+__host__ __device__ constexpr bool conv_clean_tap(int B, int LEN, int d) {
+    for (int t = 0; t < LEN; ++t)
+        for (int l = 1; l <= 3; ++l)
+            if (t - l == d && d < t - t % B) return true;
+    return false;
 }
 
-// Convolve rows r0+15 .. r0 of one 8-channel column in place (descending, a 4-row window).
-// noisy: rows of view v; taps before the row's block start read clean raw rows / the halo.
-template <int B, bool NOISY>
-__device__ __forceinline__ void conv_rows(uint8_t *sm, const float *cw, const uint4 (*halo)[3][16], bool first,
-                                          int X, int v, int cc, int r0, const uint4 (&pre)[3], int cstart,
-                                          int s_doc) {
-    float w[8][4];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const float4 t = *reinterpret_cast<const float4 *>(cw + (X * 128 + 8 * cc + e) * 4);
-        w[e][0] = t.x; w[e][1] = t.y; w[e][2] = t.z; w[e][3] = t.w;
+// One work item: the LEN rows r0.. of one 8-channel column of one tensor, convolved in place;
+// a noisy item covers both views.  own[v][t] = raw row r0 + t of view v; ini = the raw rows
+// before them: for a noisy segment that starts on a block boundary (B <= LEN) every clean row
+// d (relative to r0, -3 <= d < LEN - 1) that a block start taps, shared by the views; otherwise
+// rows r0-3..r0-1 per view (clean, or the noisy rows of the view when r0 is inside a block).
+// All reads happen in load(); the caller puts a barrier between the loads and the stores.
+template <int B, bool NOISY, int LEN>
+struct ConvSeg {
+    static constexpr int NV = NOISY ? 2 : 1;
+    static constexpr bool TAPS = NOISY && B <= LEN;
+    static constexpr int NI = TAPS ? LEN + 2 : 3;
+    static constexpr int NIV = (NOISY && !TAPS) ? NV : 1;
+    uint4 own[NV][LEN];
+    uint4 ini[NIV][NI];
+
+    // own0: half tile of the tensor (view 0; view 1 follows 8 KB later); cln: half tile of the
+    // clean tensor; halo: carried raw clean rows [row][column] (rows cstart-3..cstart-1); zr:
+    // chunk rows r < zr lie before the document start and read 0 when clean; bstart: r0 starts
+    // a block (noisy items).
+    __device__ __forceinline__ uint4 clean_row(uint32_t cln, const uint4 (*halo)[16], int cc, int r, int c8,
+                                               int zr) {
+        if (r < zr) return make_uint4(0u, 0u, 0u, 0u);
+        if (r < 0) return halo[3 + r][cc];
+        return lds128(conv_row(cln, r, c8));
     }
-    auto own = [&](int r) -> uint4 {
-        if (NOISY) return *reinterpret_cast<const uint4 *>(noisy_at(sm, X, v, r, cc));
-        return clean_raw(sm, X, r, cc, cstart, s_doc);
-    };
-    auto clean_or_halo = [&](int src) -> uint4 {
-        if (src >= 0) return clean_raw(sm, X, src, cc, cstart, s_doc);
-        return first ? make_uint4(0u, 0u, 0u, 0u) : halo[X][3 + src][cc];
-    };
-    float x[4][8];                 // raw rows t, t-1, t-2, t-3
+    __device__ __forceinline__ void load(uint32_t own0, uint32_t cln, const uint4 (*halo)[16], int cc, int r0,
+                                         int c8, int zr, bool bstart) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) unpack8(own(r0 + 15 - i), x[i]);
+        for (int v = 0; v < NV; ++v) {
 #pragma unroll
-    for (int jj = 15; jj >= 0; --jj) {
-        const int t = r0 + jj;
-        float tap[4][8];
-#pragma unroll
-        for (int l = 0; l < 4; ++l) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) tap[l][e] = x[l][e];
+            for (int t = 0; t < LEN; ++t) own[v][t] = lds128(conv_row(own0 + v * 8192, r0 + t, c8));
         }
-        if (NOISY) {
-            const int bs = t - (t % B);
+        if (!NOISY && zr > r0) {
 #pragma unroll
-            for (int l = 1; l < 4; ++l) {
-                if (t - l < bs) unpack8(clean_or_halo(t - l), tap[l]);
+            for (int t = 0; t < LEN; ++t)
+                if (r0 + t < zr) own[0][t] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (TAPS) {
+#pragma unroll
+            for (int k = 0; k < NI; ++k)
+                ini[0][k] = conv_clean_tap(B, LEN, k - 3) ? clean_row(cln, halo, cc, r0 + k - 3, c8, zr)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
+        } else if (!NOISY) {
+#pragma unroll
+            for (int k = 0; k < 3; ++k) ini[0][k] = clean_row(cln, halo, cc, r0 + k - 3, c8, zr);
+        } else if (bstart) {
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+                ini[0][k] = clean_row(cln, halo, cc, r0 + k - 3, c8, zr);
+                ini[NIV - 1][k] = ini[0][k];
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < NIV; ++v) {
+#pragma unroll
+                for (int k = 0; k < 3; ++k) ini[v][k] = lds128(conv_row(own0 + v * 8192, r0 + k - 3, c8));
             }
         }
-        float o[8];
+    }
+
+    // Convolve and write over the rows.  w: weights of this (tensor, column).
+    __device__ __forceinline__ void store(uint32_t own0, uint32_t w, int r0, int c8) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            o[e] = fmaf(w[e][3], tap[0][e], fmaf(w[e][2], tap[1][e], fmaf(w[e][1], tap[2][e], w[e][0] * tap[3][e])));
-        uint8_t *dst = NOISY ? noisy_at(sm, X, v, t, cc) : clean_at(sm, X, t, cc);
-        *reinterpret_cast<uint4 *>(dst) = pack8(o);
-        if (jj > 0) {
+        for (int i = 0; i < 4; ++i) {                 // channel pair (2i, 2i+1)
+            const float4 wa = lds128f(w + i * 512), wb = lds128f(w + i * 512 + 256);
+            const float2 w0 = make_float2(wa.x, wa.y), w1 = make_float2(wa.z, wa.w);
+            const float2 w2 = make_float2(wb.x, wb.y), w3 = make_float2(wb.z, wb.w);
 #pragma unroll
-            for (int l = 0; l < 3; ++l) {
+            for (int v = 0; v < NV; ++v) {
+                uint4 (&in)[NI] = ini[TAPS ? 0 : (NIV > 1 ? v : 0)];
+                float2 x1 = bf2_lo_hi(word_of(in[2], i)), x2 = bf2_lo_hi(word_of(in[1], i)),
+                       x3 = bf2_lo_hi(word_of(in[0], i));
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[l][e] = x[l + 1][e];
+                for (int t = 0; t < LEN; ++t) {
+                    if (TAPS && t > 0 && t % B == 0) {   // block start: clean taps
+                        x1 = bf2_lo_hi(word_of(in[t + 2], i));
+                        x2 = bf2_lo_hi(word_of(in[t + 1], i));
+                        x3 = bf2_lo_hi(word_of(in[t], i));
+                    }
+                    const float2 x0 = bf2_lo_hi(word_of(own[v][t], i));
+                    float2 acc = __fmul2_rn(w3, x0);
+                    acc = __ffma2_rn(w2, x1, acc);
+                    acc = __ffma2_rn(w1, x2, acc);
+                    acc = __ffma2_rn(w0, x3, acc);
+                    word_of(own[v][t], i) = f2_to_bf2(acc);   // the raw word is dead once unpacked
+                    x3 = x2; x2 = x1; x1 = x0;
+                }
             }
-            if (jj - 4 >= 0) unpack8(own(r0 + jj - 4), x[3]);
-            else unpack8(pre[jj - 1], x[3]);
+        }
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+#pragma unroll
+            for (int t = 0; t < LEN; ++t) sts128(conv_row(own0 + v * 8192, r0 + t, c8), own[v][t]);
         }
     }
+};
+
+// Weights of (tensor X, column cc): fp32 [channel pair i][taps 0-1 | taps 2-3][cc][tap][pair], so
+// the eight lanes of a shared-memory phase read eight consecutive 16-byte words and every word
+// is an operand pair of a packed FFMA2.
+__device__ __forceinline__ uint32_t conv_weights(uint32_t s, int X, int cc) {
+    return s + OFF_CW + (X * 128 + cc) * 16;
+}
+// Noisy item (both views): tensor X, rows r0..r0+LEN-1.  BAR: barrier between loads and stores.
+template <int B, int LEN, bool BAR>
+__device__ __forceinline__ void conv_noisy_item(uint32_t s, uint4 (*halo)[3][16], int X, int cc, int r0, int zr) {
+    const int hf = cc >> 3, c8 = cc & 7;
+    const uint32_t own = s + noisy_half(X, 0, hf);
+    ConvSeg<B, true, LEN> sg;
+    sg.load(own, s + clean_half(X, hf), halo[X], cc, r0, c8, zr, (r0 % B) == 0);
+    if (BAR) bar_math();
+    sg.store(own, conv_weights(s, X, cc), r0, c8);
+}
+// Clean item: tensor X, rows r0..r0+LEN-1; the item ending at row 63 carries rows 61..63 (raw)
+// to the next chunk.
+template <int B, int LEN>
+__device__ __forceinline__ void conv_clean_item(uint32_t s, uint4 (*halo)[3][16], int X, int cc, int r0, int zr) {
+    const int hf = cc >> 3, c8 = cc & 7;
+    const uint32_t own = s + clean_half(X, hf);
+    ConvSeg<B, false, LEN> sg;
+    sg.load(own, own, halo[X], cc, r0, c8, zr, true);
+    bar_math();
+    if (r0 + LEN == CH) {
+#pragma unroll
+        for (int l = 0; l < 3; ++l) halo[X][l][cc] = sg.own[0][LEN - 3 + l];
+    }
+    sg.store(own, conv_weights(s, X, cc), r0, c8);
 }
 
-// The whole prologue for one chunk (all threads; barriers inside).  Noisy tiles first (they
-// read raw clean rows), then the clean tiles, whose last three raw rows become the next halo.
+// The whole prologue for one chunk (all threads; a barrier between the reads and the writes of
+// each round that rewrites rows another item reads).  A noisy tile is convolved before the clean
+// tile of the same tensor is overwritten (its block-start taps read the raw clean rows); a halo
+// is read before the round that rewrites it.  Rounds of 256 items, 36 output rows per thread:
+//   1  noisy q, k (8-row items, both views)
+//   2  noisy v (8-row items, both views) | clean q, k (16-row items)
+//   3  clean v (4-row items)
+// A chunk without noisy rows runs clean q, k as 8-row items, then round 3.
+// zr = document start - chunk start.
 template <int B>
-__device__ __noinline__ void conv_chunk(uint8_t *sm, uint4 (*halo)[3][16], bool first, bool noisy, int cstart,
-                                        int s_doc, int tid) {
-    const float *cw = reinterpret_cast<const float *>(sm + OFF_CW);
+__device__ __noinline__ void conv_chunk(uint8_t *sm, uint4 (*halo)[3][16], bool noisy, int zr, int tid) {
+    const uint32_t s = smem_u32(sm);
+    const int cc = tid & 15;
     if (noisy) {
-        for (int round = 0; round < 2; ++round) {    // 384 items: (tensor, view, column chunk, segment)
-            const int it = tid + 256 * round;
-            const bool act = it < 384;
-            const int X = it / 128, rem = it % 128, v = rem / 64, cc = (rem % 64) / 4, r0 = 16 * (rem % 4);
-            uint4 pre[3];
-#pragma unroll
-            for (int l = 0; l < 3; ++l)
-                pre[l] = (act && r0 > 0) ? *reinterpret_cast<const uint4 *>(noisy_at(sm, X, v, r0 - 3 + l, cc))
-                                         : make_uint4(0u, 0u, 0u, 0u);
-            bar_math();
-            if (act) conv_rows<B, true>(sm, cw, halo, first, X, v, cc, r0, pre, cstart, s_doc);
-            bar_math();
-        }
+        conv_noisy_item<B, 8, (B > 8)>(s, halo, tid >> 7, cc, 8 * ((tid >> 4) & 7), zr);
+        if (tid < 128) conv_noisy_item<B, 8, true>(s, halo, 2, cc, 8 * ((tid >> 4) & 7), zr);
+        else conv_clean_item<B, 16>(s, halo, (tid >> 6) & 1, cc, 16 * ((tid >> 4) & 3), zr);
+    } else {
+        conv_clean_item<B, 8>(s, halo, tid >> 7, cc, 8 * ((tid >> 4) & 7), zr);
     }
-    const bool act = tid < 192;                         // 192 items: (tensor, column chunk, segment)
-    const int X = tid / 64, cc = (tid % 64) / 4, r0 = 16 * (tid % 4);
-    uint4 pre[3];
-#pragma unroll
-    for (int l = 0; l < 3; ++l) {
-        const int src = r0 - 3 + l;
-        pre[l] = !act ? make_uint4(0u, 0u, 0u, 0u)
-                      : (src >= 0 ? clean_raw(sm, X, src, cc, cstart, s_doc)
-                                  : (first ? make_uint4(0u, 0u, 0u, 0u) : halo[X][3 + src][cc]));
-    }
-    bar_math();
-    if (act) {
-        if (r0 == 48) {
-#pragma unroll
-            for (int l = 0; l < 3; ++l) halo[X][l][cc] = clean_raw(sm, X, 61 + l, cc, cstart, s_doc);
-        }
-        conv_rows<B, false>(sm, cw, halo, first, X, 0, cc, r0, pre, cstart, s_doc);
-    }
-    bar_math();
+    conv_clean_item<B, 4>(s, halo, 2, cc, 4 * (tid >> 4), zr);
+    fence_async_smem();                      // the tiles are next read by the tensor cores
 }
 
 template <int B>
@@ -685,9 +773,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             }
             // ---- conv weights of this head (cp.async into the K-hat buffer, free until PE1) ----
             if (conv) {
-                for (int it = tid; it < 3 * 128 * 4 / 4; it += kThreads) {
-                    const int X = it / 128, c = it % 128;
-                    cp_async16(sm + OFF_CW + it * 16, P.conv_w + (((int64_t)X * H + U.h) * 128 + c) * 4);
+                for (int it = tid; it < 3 * 128 * 4; it += kThreads) {   // (tensor X, channel c, tap j)
+                    const int X = it >> 9, c = (it >> 2) & 127, j = it & 3;
+                    const int dst = (X * 128 + ((c & 7) >> 1) * 32 + (j >> 1) * 16 + (c >> 3)) * 4 + (j & 1) * 2 + (c & 1);
+                    cp_async4(sm + OFF_CW + dst * 4, P.conv_w + (((int64_t)X * H + U.h) * 128 + c) * 4 + j, 4);
                 }
                 cp_async_commit();
             }
@@ -698,9 +787,27 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
                 ++ph_b;
                 cp_async_wait_all();
+                // The state rows wait in tensor memory (columns free until the batch MMAs) while
+                // the conv needs the registers.
+                {
+                    float t0[32], t1[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) { t0[c] = S[c]; t1[c] = S[32 + c]; }
+                    tmem_st32(tmem_addr(tb, q * 32, TM_N + 64 * ch), t0);
+                    tmem_st32(tmem_addr(tb, q * 32, TM_N + 64 * ch + 32), t1);
+                    tmem_wait_st();
+                }
                 __syncwarp();
                 bar_all();
-                conv_chunk<B>(sm, s_halo, ci == 0, noisy, cstart, U.s, tid);
+                conv_chunk<B>(sm, s_halo, noisy, U.s - cstart, tid);
+                {
+                    float t0[32], t1[32];
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_N + 64 * ch), t0);
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_N + 64 * ch + 32), t1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) { S[c] = t0[c]; S[32 + c] = t1[c]; }
+                }
             }
             __syncwarp();
             bar_all();
