@@ -98,59 +98,108 @@ def profiled_traffic(algo, workload):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clock and throttle-reason samples taken DURING the timed region.
+
+    NVML is polled from a thread about every millisecond between mark_start() and mark_stop(),
+    so even a timed region of a few milliseconds gets samples; without NVML, nvidia-smi is run
+    in the background (100 ms period) and its lines are kept."""
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device: int):
+        self.device = device
+        self.samples = []          # (sm_mhz, max_mhz, {reason names})
+        self.source = None
+        self._on = threading.Event()
+        self._quit = threading.Event()
+        self._thread = None
+        self._proc = None
+        self._lines = []
+
+    # -- NVML
+    def _nvml_handle(self, nv):
+        try:
+            props = torch.cuda.get_device_properties(self.device)
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.device)
+
+    def _nvml_loop(self, nv, h):
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self._quit.is_set():
+            if self._on.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h) if hasattr(
+                        nv, "nvmlDeviceGetCurrentClocksEventReasons") else nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                    self.samples.append((float(sm), float(mx), {n for n, m in self.REASONS.items() if bits & m}))
+                except Exception:
+                    pass
+            time.sleep(0.001)
+
+    # -- nvidia-smi fallback
+    def _smi_read(self):
+        for line in self._proc.stdout:
+            if self._on.is_set():
+                self._lines.append(line.strip())
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "100", "-i", str(self.gpu)],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except (FileNotFoundError, OSError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._nvml_handle(nv)
+            self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self._thread.start()
+            self.source = "nvml"
+        except Exception:
+            try:
+                self._proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                               "-lms", "100", "-i", str(self.device)],
+                                              stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self._thread = threading.Thread(target=self._smi_read, daemon=True)
+                self._thread.start()
+                self.source = "nvidia-smi"
+            except (FileNotFoundError, OSError):
+                self.source = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def mark_start(self):
+        self._on.set()
+
+    def mark_stop(self):
+        self._on.clear()
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        self._quit.set()
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.thread.join(timeout=2)
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        samples = list(self.samples)
+        for ln in self._lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                rs = {n for n, v in zip(["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"],
+                                        parts[5:9]) if v.lower().startswith("active")}
+                samples.append((float(parts[1]), float(parts[2]), rs))
             except ValueError:
                 continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
+        if not samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set().union(*[r for _, _, r in samples])
+        return {"sm_mhz": statistics.median(s for s, _, _ in samples), "sm_max_mhz": max(m for _, m, _ in samples),
+                "reasons": sorted(reasons), "samples": len(samples), "source": self.source}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -279,6 +328,7 @@ def main():
     with ClockSampler(local) as clocks:
         barrier()
         torch.cuda.synchronize()
+        clocks.mark_start()
         start.record(stream)
         for i in range(args.steps):
             evs[i][0].record(stream)
@@ -286,6 +336,7 @@ def main():
             evs[i][1].record(stream)
         stop.record(stream)
         torch.cuda.synchronize()
+        clocks.mark_stop()
         barrier()
     elapsed_ms = max_over_ranks(start.elapsed_time(stop))
     launch_ms = [a.elapsed_time(b) for a, b in evs]
