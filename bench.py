@@ -151,6 +151,8 @@ class ClockSampler:
             import pynvml as nv
             nv.nvmlInit()
             h = self._nvml_handle(nv)
+            self._nv, self._h = nv, h
+            self._mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
             self._thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
             self._thread.start()
             self.source = "nvml"
@@ -168,6 +170,21 @@ class ClockSampler:
 
     def mark_start(self):
         self._on.set()
+
+    def poll_until(self, event):
+        """Sample from the calling thread until `event` (a CUDA event recorded after the timed
+        work) has completed, so a short timed region still gets samples under load."""
+        nv, h = getattr(self, "_nv", None), getattr(self, "_h", None)
+        while not event.query():
+            if nv is not None:
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h) if hasattr(
+                        nv, "nvmlDeviceGetCurrentClocksEventReasons") else nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                    self.samples.append((float(sm), float(self._mx), {n for n, m in self.REASONS.items() if bits & m}))
+                except Exception:
+                    pass
+            time.sleep(0.0005)
 
     def mark_stop(self):
         self._on.clear()
@@ -335,6 +352,7 @@ def main():
             step()
             evs[i][1].record(stream)
         stop.record(stream)
+        clocks.poll_until(stop)
         torch.cuda.synchronize()
         clocks.mark_stop()
         barrier()

@@ -161,13 +161,14 @@ __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float 
         arow[l] = (l < jl) ? bj * exp2f(fminf(gj - gl[l], 0.f)) * ak[l] : 0.f;
         pt[l] = aq[l] * exp2f(gend - gl[l]);
     }
+    // Right-looking back substitution: once y_mm is final it is taken out of every earlier
+    // position at once, so the dependent chain is B steps of one FMA each.
     const int base = lane - jl;
 #pragma unroll
-    for (int l = B - 1; l >= 0; --l) {
-        float acc = pt[l];
+    for (int mm = B - 1; mm >= 0; --mm) {
+        y[mm] = pt[mm];
 #pragma unroll
-        for (int mm = l + 1; mm < B; ++mm) acc -= y[mm] * __shfl_sync(0xffffffffu, arow[l], base + mm);
-        y[l] = acc;
+        for (int l = 0; l < mm; ++l) pt[l] = fmaf(-y[mm], __shfl_sync(0xffffffffu, arow[l], base + mm), pt[l]);
     }
 #pragma unroll
     for (int l = 0; l < B; ++l) {
@@ -309,13 +310,20 @@ __device__ void solve_T(float *sa, float *xb, int tid, int warp) {
         const int t = tid - 32;
         if (t < 64) {
             const int o = (t >> 3) * 8, c = t & 7;
-            float x[8];
+            // column c of the block's inverse, right-looking: x_l is final once every earlier
+            // x has been taken out of it
+            float a[8][8], x[8];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                float acc = (jj == c) ? 1.f : 0.f;
+            for (int jj = 1; jj < 8; ++jj) {
 #pragma unroll
-                for (int l = 0; l < jj; ++l) acc = fmaf(-sa[sidx(o + jj, o + l)], x[l], acc);
-                x[jj] = acc;
+                for (int l = 0; l < jj; ++l) a[jj][l] = sa[sidx(o + jj, o + l)];
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) x[jj] = (jj == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int l = 0; l < 8; ++l) {
+#pragma unroll
+                for (int jj = l + 1; jj < 8; ++jj) x[jj] = fmaf(-a[jj][l], x[l], x[jj]);
             }
             __syncwarp();
 #pragma unroll
