@@ -56,7 +56,7 @@ constexpr int OFF_Y = 98304;       // 16 KB  fp32 solve scratch, then [P;T] -> [
 constexpr int OFF_NQ = 114688;     // 32 KB  [q~0;q~1] -> Z -> Gamma_e Z, K-major
 constexpr int OFF_NK = 147456;     // 32 KB  [k~0;k~1] K-major; d-half 0 later holds M'_Z
 constexpr int OFF_NV = 180224;     // 32 KB  [v~0;v~1] per v-half (row-major, swizzled)
-constexpr int OFF_W = 212992;      //  4 KB  triangular-solve staging (one 32x32 fp32 block)
+constexpr int OFF_W = 212992;      //  4 KB  the triangular solve's 32-merge result (32x32 fp32)
 constexpr int SMEM_USED = 217088;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;   // alignment slack
 
@@ -244,6 +244,60 @@ __device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int 
     }
 }
 
+// 32 x 32 fp32 staging block (the 32-merge's result): 128-byte rows, 16-byte chunks swizzled by
+// the row like the solve scratch.
+__device__ __forceinline__ int widx(int r, int c) { return r * 32 + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3); }
+__device__ __forceinline__ float4 *wrow4(float *w, int r, int c4) {
+    return reinterpret_cast<float4 *>(w + r * 32 + ((((c4 >> 2) ^ (r & 7))) << 2));
+}
+
+// One merge of the triangular inverse by one warp that owns NC consecutive output columns
+// [cb, cb + NC) of the S x S block below the diagonal at offset o.  With T11 = T[o.., o..] and
+// T22 = T[o+S.., o+S..] already inverted (unit lower, zeros above the diagonal):
+//   X = A[o+S.., o..] T11,   T[o+S.., o..] = -T22 X.
+// Lane (g = lane / NC, cl = lane % NC) holds column cb + cl for the rows g + RG*i.  X moves between
+// the lanes by shuffles, so the warp needs no barrier; T11[k][c] = 0 for k < c lets the first
+// product start at k = cb, and the second product of row r stops at k = r (warp-uniform bounds).
+// The result goes to dst[(row, col)] via `store` (block-local row and column).
+template <int S, int NC, typename Store>
+__device__ __forceinline__ void warp_merge(const float *sa, int o, int cb, int lane, Store store) {
+    constexpr int RG = 32 / NC, NR = S / RG;
+    const int cl = lane % NC, g = lane / NC, c = cb + cl;
+    float x[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) x[i] = 0.f;
+#pragma unroll
+    for (int k4 = 0; k4 < S; k4 += 4) {
+        if (k4 < (cb & ~3)) continue;
+        float tv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tv[e] = sa[sidx(o + k4 + e, o + c)];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const float4 a = *srow4(const_cast<float *>(sa), o + S + g + RG * i, o + k4);
+            x[i] = fmaf(a.w, tv[3], fmaf(a.z, tv[2], fmaf(a.y, tv[1], fmaf(a.x, tv[0], x[i]))));
+        }
+    }
+    float y[NR];
+#pragma unroll
+    for (int i = 0; i < NR; ++i) y[i] = 0.f;
+#pragma unroll
+    for (int k4 = 0; k4 < S; k4 += 4) {
+        float xk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) xk[e] = __shfl_sync(0xffffffffu, x[(k4 + e) / RG], ((k4 + e) % RG) * NC + cl);
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            if (k4 <= RG * i + RG - 1) {
+                const float4 a = *srow4(const_cast<float *>(sa), o + S + g + RG * i, o + S + k4);
+                y[i] = fmaf(a.w, xk[3], fmaf(a.z, xk[2], fmaf(a.y, xk[1], fmaf(a.x, xk[0], y[i]))));
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NR; ++i) store(g + RG * i, c, -y[i]);
+}
+
 // One merge level of the triangular inverse: for every pair of S x S diagonal blocks at offset
 // o (already inverted), X = A[o+S.., o..] T[o.., o..] and T[o+S.., o..] = -T[o+S.., o+S..] X.
 // NT threads (t = 0..NT-1 when `active`): column c, rows g + RG*i.  T[o+S.., o+S..] is unit lower
@@ -302,10 +356,13 @@ __device__ __forceinline__ void tri_merge(float *sa, float *xb, int t, bool acti
     if (side) bar_side(); else bar_math();
 }
 
-// T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch (in place): the eight
-// 8x8 diagonal blocks by forward substitution (one thread per column) and the 8- and 16-merges on
-// warps 1..7 (warp 0 is issuing an MMA batch meanwhile), then the 32-merge on all warps.
-__device__ void solve_T(float *sa, float *xb, int tid, int warp) {
+// T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch, while warp 0 issues an MMA
+// batch: warps 1-7 invert the eight 8x8 diagonal blocks (one thread per column, right-looking
+// forward substitution) and run the 8- and 16-merges; then all warps run the 32-merge
+// (warp-local, no barrier inside), whose lower-left block goes to the 32 x 32 staging block `wb`
+// (rows 32..63, columns 0..31 of T) so that no warp overwrites A while another still reads it.
+__device__ void solve_T(float *sa, float *wb, int tid, int warp) {
+    const int lane = tid & 31;
     if (warp > 0) {
         const int t = tid - 32;
         if (t < 64) {
@@ -330,11 +387,13 @@ __device__ void solve_T(float *sa, float *xb, int tid, int warp) {
             for (int jj = 0; jj < 8; ++jj) sa[sidx(o + jj, o + c)] = x[jj];
         }
         bar_side();
-        tri_merge<8, 128>(sa, xb, t, t < 128, true);
-        tri_merge<16, 128>(sa, xb, t, t < 128, true);
+        tri_merge<8, 128>(sa, wb, t, t < 128, true);
+        tri_merge<16, 128>(sa, wb, t, t < 128, true);
     }
     bar_math();
-    tri_merge<32, 256>(sa, xb, tid, true, false);
+    // warp 0 arrives last (it issued the MMA batch): it takes the columns with the least work
+    warp_merge<32, 4>(sa, 0, 4 * (7 - warp), lane, [&](int r, int c, float v) { wb[widx(r, c)] = v; });
+    bar_math();
 }
 
 // ----------------------------------------------------------------------------- ShortConv
@@ -932,10 +991,11 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // [P ; T] as bf16 K-major A (128 rows x 64): this thread writes row rho, cols [32ch, 32ch+32)
             if (rho >= 64) {
                 const int t = rho - 64;
+                const bool lowleft = t >= 32 && ch == 0;          // the 32-merge's block
 #pragma unroll
                 for (int g4 = 0; g4 < 4; ++g4) {
-                    const float4 a = *srow4(scratch, t, 32 * ch + 8 * g4);
-                    const float4 b = *srow4(scratch, t, 32 * ch + 8 * g4 + 4);
+                    const float4 a = lowleft ? *wrow4(wstage, t - 32, 8 * g4) : *srow4(scratch, t, 32 * ch + 8 * g4);
+                    const float4 b = lowleft ? *wrow4(wstage, t - 32, 8 * g4 + 4) : *srow4(scratch, t, 32 * ch + 8 * g4 + 4);
                     const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
                     ppk[g4] = pack8(f);
                 }
