@@ -44,6 +44,8 @@ def open_library(path: str):
     lib.gdn_oracle_forward.argtypes = ([ctypes.c_int] * 7 + [ip, ip] + [dp] * 10 + [dp]
                                        + [dp, dp, dp, dp] + [ctypes.c_int])
     lib.gdn_oracle_max_threads.restype = ctypes.c_int
+    lib.gdn_oracle_decode_steps.restype = ctypes.c_int
+    lib.gdn_oracle_decode_steps.argtypes = [ctypes.c_int] * 5 + [dp] * 9 + [ctypes.c_int]
     return lib
 
 
@@ -122,3 +124,38 @@ def forward_problem(prob, num_threads: int = 0, return_noisy_state: bool = False
                    prob.gn, prob.betan, prob.doc_offsets, prob.prompt_len, prob.block_size,
                    conv_w=prob.conv_w, num_threads=num_threads,
                    return_noisy_state=return_noisy_state, _lib=_lib)
+
+
+def decode_steps(S0, q, k, v, g, beta, record_states: bool = False, num_threads: int = 0, _lib=None):
+    """Decode-side clean steps from given states (the serving paragraph of the FLARE notes:
+    Diffusion-Trust causal replay of a committed block; AR-Trust verify forward with every
+    step's state kept for the rollback).  S0 [Nseq,H,dk,dv]; q,k [Nseq,L,H,dk]; v [Nseq,L,H,dv];
+    g, beta [Nseq,L,H].  Returns dict(out=[Nseq,L,H,dv], final_state=[Nseq,H,dk,dv]
+    [, states=[Nseq,L,H,dk,dv]]) as fp64 arrays."""
+    lib = _lib if _lib is not None else _load()
+    S0, q, k, v, g, beta = (_f64(x) for x in (S0, q, k, v, g, beta))
+    Nseq, L, H, dk = q.shape
+    dv = v.shape[3]
+    out = np.zeros((Nseq, L, H, dv))
+    fin = np.zeros((Nseq, H, dk, dv))
+    st = np.zeros((Nseq, L, H, dk, dv)) if record_states else None
+    rc = lib.gdn_oracle_decode_steps(Nseq, H, L, dk, dv, _ptr(S0), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                     _ptr(beta), _ptr(out), _ptr(fin), _ptr(st), int(num_threads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the inputs (code {rc})")
+    res = dict(out=out, final_state=fin)
+    if record_states:
+        res["states"] = st
+    return res
+
+
+def commit(pool, slots, states, accepted):
+    """AR-Trust rollback by gather-scatter (the serving paragraph of the FLARE notes): for every
+    sequence i with accepted[i] = r >= 1, pool[slots[i]] := states[i, r - 1] (the state after the
+    r accepted candidates); r = 0 leaves the pool row as it was.  Returns a new fp64 array."""
+    pool = _f64(pool).copy()
+    states = _f64(states)
+    for i, (slot, r) in enumerate(zip(np.asarray(slots), np.asarray(accepted))):
+        if r >= 1:
+            pool[int(slot)] = states[i, int(r) - 1]
+    return pool

@@ -255,6 +255,55 @@ int gdn_oracle_forward(int N, int H, int dk, int dv, int V, int B, int conv_widt
     return status;
 }
 
+/*
+ * Decode-side steps (the serving paragraph of the same notes: Diffusion-Trust commits a finished
+ * block with one causal replay that writes its final state into the state pool; AR-Trust's
+ * verify forward runs the clean stream over the K candidate tokens and keeps every step's state
+ * so that accepting the first r candidates is a gather of state r).  Per sequence n and head h:
+ *   S := S0[n, h];  for t = 0..L-1:  S <- alpha_t (I - beta_t k_t k_t^T) S + beta_t k_t v_t^T,
+ *                                     o_t = S^T q_t / sqrt(dk),  states[n, t, h] = S (optional);
+ *   S_final[n, h] := S.
+ * Shapes: S0, S_final [Nseq, H, dk, dv]; q,k [Nseq, L, H, dk]; v [Nseq, L, H, dv];
+ *         g, beta [Nseq, L, H]; out [Nseq, L, H, dv]; states (may be NULL) [Nseq, L, H, dk, dv].
+ */
+int gdn_oracle_decode_steps(int Nseq, int H, int L, int dk, int dv,
+                            const double *S0, const double *q, const double *k, const double *v,
+                            const double *g, const double *beta,
+                            double *out, double *S_final, double *states, int num_threads)
+{
+    if (Nseq < 0 || H < 1 || L < 0 || dk < 1 || dv < 1) return ORACLE_BAD_ARG;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+    int status = ORACLE_OK;
+    const long units = (long)Nseq * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long unit = 0; unit < units; ++unit) {
+        const long n = unit / H, h = unit % H;
+        const long sz = (long)dk * dv;
+        double *S = (double *)malloc(sizeof(double) * (size_t)sz);
+        double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (!S || !u) {
+            free(S); free(u);
+#pragma omp atomic write
+            status = ORACLE_NOMEM;
+            continue;
+        }
+        memcpy(S, S0 + unit * sz, sizeof(double) * (size_t)sz);
+        for (int t = 0; t < L; ++t) {
+            const long row = (n * L + t) * H + h;          /* (n, t, h) */
+            delta_step(S, u, dk, dv, k + row * dk, v + row * dv, exp(g[row]), beta[row]);
+            readout(S, dk, dv, q + row * dk, out + row * dv);
+            if (states) memcpy(states + row * sz, S, sizeof(double) * (size_t)sz);
+        }
+        memcpy(S_final + unit * sz, S, sizeof(double) * (size_t)sz);
+        free(S); free(u);
+    }
+    return status;
+}
+
 /* Threads the oracle would use (for reporting). */
 int gdn_oracle_max_threads(void)
 {
