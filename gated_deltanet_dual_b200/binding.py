@@ -21,7 +21,8 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_ALIGNMENT, GDN_ERR_UNSUPPORTED, GDN_ERR_CUD
 GDN_BF16, GDN_FP32 = 0, 1
 ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED = 0, 1, 2
 EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device_status",
-            "gdn_status_string", "gdn_dual_version", "gdn_dual_select_algo")
+            "gdn_status_string", "gdn_dual_version", "gdn_dual_select_algo",
+            "gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit")
 
 
 class GdnError(RuntimeError):
@@ -33,6 +34,12 @@ class GdnError(RuntimeError):
 class Desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("num_docs", "num_heads", "d_k", "d_v", "num_views",
                                                "block_size", "dtype", "conv_width", "algo", "reserved")]
+
+
+class DecodeDesc(ctypes.Structure):
+    """gdn_decode_desc of include/gdn_decode.h."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("num_seqs", "num_heads", "d_k", "d_v", "num_tokens",
+                                               "pool_slots", "dtype", "reserved")]
 
 
 _lock = threading.Lock()
@@ -60,6 +67,12 @@ def load_library(path: str = LIB_PATH):
             lib.gdn_dual_version.restype = ctypes.c_int32
             lib.gdn_dual_select_algo.restype = ctypes.c_int32
             lib.gdn_dual_select_algo.argtypes = [ctypes.POINTER(Desc)]
+            dd = ctypes.POINTER(DecodeDesc)
+            for name in ("gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit"):
+                getattr(lib, name).restype = ctypes.c_int
+            lib.gdn_decode_replay.argtypes = [dd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.gdn_decode_verify.argtypes = [dd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+            lib.gdn_decode_commit.argtypes = [dd, vp, vp, vp, vp, vp, vp]
             _lib = lib
     return _lib
 
@@ -218,3 +231,79 @@ def forward_noalloc_raw(desc: Desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc
     return int(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(qn), _ptr(kn), _ptr(vn),
                   _ptr(gn), _ptr(betan), offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(conv_w),
                   _ptr(out), _ptr(out_noisy), _ptr(final_state), ctypes.c_void_p(stream)))
+
+
+# ----------------------------------------------------------------------------- decode side
+def make_decode_desc(num_seqs, num_heads, d_k, d_v, num_tokens, pool_slots, dtype_code) -> DecodeDesc:
+    return DecodeDesc(num_seqs, num_heads, d_k, d_v, num_tokens, pool_slots, dtype_code, 0)
+
+
+def _decode_args(state_pool, slots, q, k, v, g, beta):
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    N, L, H, dk = q.shape
+    dv = v.shape[3]
+    P = state_pool.shape[0]
+    io, f32 = q.dtype, torch.float32
+    for t, name, shape, dt in ((state_pool, "state_pool", (P, H, dk, dv), f32), (slots, "slots", (N,), torch.int32),
+                               (q, "q", (N, L, H, dk), io), (k, "k", (N, L, H, dk), io), (v, "v", (N, L, H, dv), io),
+                               (g, "g", (N, L, H), f32), (beta, "beta", (N, L, H), f32)):
+        _check(t, name, shape, dt, dev)
+    return make_decode_desc(N, H, dk, dv, L, P, _dtype_code(q)), dev, (N, L, H, dk, dv)
+
+
+def _stream(stream):
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream if stream is None else stream)
+
+
+def decode_replay(state_pool, slots, q, k, v, g, beta, *, out=None, device_status=None, stream=None):
+    """Causal replay of a committed block (gdn_decode_replay): runs the L tokens of every sequence
+    from its pooled state, writes the outputs and the final state back into state_pool[slots]."""
+    desc, dev, (N, L, H, dk, dv) = _decode_args(state_pool, slots, q, k, v, g, beta)
+    if out is None:
+        out = torch.empty(N, L, H, dv, dtype=q.dtype, device=dev)
+    _check(out, "out", (N, L, H, dv), q.dtype, dev)
+    st = load_library().gdn_decode_replay(ctypes.byref(desc), _ptr(state_pool), _ptr(slots), _ptr(q), _ptr(k),
+                                          _ptr(v), _ptr(g), _ptr(beta), _ptr(out), _ptr(device_status),
+                                          _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, f"gdn_decode_replay failed: {status_string(st)}")
+    return out
+
+
+def decode_verify(state_pool, slots, q, k, v, g, beta, *, out=None, state_cache=None, device_status=None,
+                  stream=None):
+    """Verify forward with state cache (gdn_decode_verify): outputs of the L candidates and the
+    state after each step in state_cache [N, L, H, d_k, d_v]; the pool is only read."""
+    desc, dev, (N, L, H, dk, dv) = _decode_args(state_pool, slots, q, k, v, g, beta)
+    if out is None:
+        out = torch.empty(N, L, H, dv, dtype=q.dtype, device=dev)
+    if state_cache is None:
+        state_cache = torch.empty(N, L, H, dk, dv, dtype=torch.float32, device=dev)
+    _check(out, "out", (N, L, H, dv), q.dtype, dev)
+    _check(state_cache, "state_cache", (N, L, H, dk, dv), torch.float32, dev)
+    st = load_library().gdn_decode_verify(ctypes.byref(desc), _ptr(state_pool), _ptr(slots), _ptr(q), _ptr(k),
+                                          _ptr(v), _ptr(g), _ptr(beta), _ptr(out), _ptr(state_cache),
+                                          _ptr(device_status), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, f"gdn_decode_verify failed: {status_string(st)}")
+    return out, state_cache
+
+
+def decode_commit(state_pool, slots, state_cache, accepted, *, device_status=None, stream=None):
+    """Commit the accepted prefix (gdn_decode_commit): state_pool[slots[n]] := state_cache[n, r-1]
+    for r = accepted[n] >= 1."""
+    dev = state_pool.device
+    N, L, H, dk, dv = state_cache.shape
+    P = state_pool.shape[0]
+    for t, name, shape, dt in ((state_pool, "state_pool", (P, H, dk, dv), torch.float32),
+                               (slots, "slots", (N,), torch.int32), (accepted, "accepted", (N,), torch.int32),
+                               (state_cache, "state_cache", (N, L, H, dk, dv), torch.float32)):
+        _check(t, name, shape, dt, dev)
+    desc = make_decode_desc(N, H, dk, dv, L, P, GDN_FP32)
+    st = load_library().gdn_decode_commit(ctypes.byref(desc), _ptr(state_pool), _ptr(slots), _ptr(state_cache),
+                                          _ptr(accepted), _ptr(device_status), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, f"gdn_decode_commit failed: {status_string(st)}")
+    return state_pool

@@ -1,0 +1,207 @@
+// gdn_decode.cu -- decode-side state kernels of the Gated DeltaNet layer (include/gdn_decode.h).
+//
+// From the serving paragraph of "FLARE: Diffusion for Hybrid Language Model" (papernotes.org
+// notes): Diffusion-Trust commits a finished block with one causal replay that writes the final
+// state into the state pool; AR-Trust verifies K drafted candidates with one clean forward that
+// also stores the state after every candidate step, and commits the first r accepted ones by a
+// gather-scatter of state r (no recomputation).  The recurrence is that of Method > Key design 2:
+// S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T, o_t = S_t^T q_t / sqrt(d_k).
+//
+// Decode work is small and bound by moving states (d_k x d_v fp32 per sequence and head), so the
+// kernels are CUDA-core kernels sized for bandwidth: one CTA per (sequence, head), the state in
+// registers (thread t owns column t/2 and half of its rows, so k^T S and S^T q need only a pair
+// shuffle), the block's tokens staged once in shared memory, and every state row read or written
+// as whole 32-byte sectors.
+#include <algorithm>
+#include <cmath>
+
+#include "gdn_internal.cuh"
+#include "gdn_decode.h"
+
+namespace gdn {
+namespace {
+
+enum DecodeMode { kReplay = 0, kVerify = 1 };
+
+struct DecodeParams {
+    float *pool;              // [P, H, D, D]
+    const int32_t *slots;     // [N]
+    const void *q, *k, *v;    // [N, L, H, D]
+    const float *g, *beta;    // [N, L, H]
+    void *out;                // [N, L, H, D]
+    float *cache;             // [N, L, H, D, D] (verify)
+    int32_t *status;          // optional
+    int N, H, L, P;
+    float scale;
+};
+
+__device__ __forceinline__ void flag_bad(int32_t *status) {
+    if (status) atomicExch(status, (int32_t)GDN_ERR_INVALID_ARG);
+}
+
+template <typename TIO, int D, int MODE>
+__global__ void __launch_bounds__(2 * D) gdn_decode_kernel(const DecodeParams p) {
+    constexpr int R = D / 2;
+    extern __shared__ float sh[];            // q [L][D], k [L][D], v [L][D], g [L], beta [L]
+    const int n = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int tid = threadIdx.x, j = tid >> 1, half = tid & 1;
+    const int slot = p.slots[n];
+    if (slot < 0 || slot >= p.P) {           // uniform over the CTA
+        if (tid == 0) flag_bad(p.status);
+        return;
+    }
+    const int L = p.L;
+    float *sq = sh, *sk = sh + L * D, *sv = sh + 2 * L * D, *sg = sh + 3 * L * D, *sb = sg + L;
+    const TIO *q = static_cast<const TIO *>(p.q), *k = static_cast<const TIO *>(p.k), *v = static_cast<const TIO *>(p.v);
+    for (int i = tid; i < L * D; i += 2 * D) {
+        const int t = i / D, c = i % D;
+        const int64_t src = ((int64_t)(n * L + t) * p.H + h) * D + c;
+        sq[i] = to_f32(q[src]);
+        sk[i] = to_f32(k[src]);
+        sv[i] = to_f32(v[src]);
+    }
+    for (int t = tid; t < L; t += 2 * D) {
+        const int64_t src = (int64_t)(n * L + t) * p.H + h;
+        sg[t] = p.g[src];
+        sb[t] = p.beta[src];
+    }
+    float S[R];
+    const float *s0 = p.pool + ((int64_t)slot * p.H + h) * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+    for (int r = 0; r < R; ++r) S[r] = s0[(int64_t)r * D];
+    __syncthreads();
+
+    for (int t = 0; t < L; ++t) {
+        const float *kt = sk + t * D + half * R, *qt = sq + t * D + half * R;
+        const float alpha = expf(sg[t]), b = sb[t];
+        // u_j = (k^T S)_j: four partial sums shorten the dependent chain
+        float pu[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < R; ++r) pu[r & 3] = fmaf(kt[r], S[r], pu[r & 3]);
+        float u = (pu[0] + pu[1]) + (pu[2] + pu[3]);
+        u += __shfl_xor_sync(0xffffffffu, u, 1);
+        // S <- alpha S + beta k (v - alpha u)^T   ( = alpha (I - beta k k^T) S + beta k v^T )
+        const float w = b * (sv[t * D + j] - alpha * u);
+#pragma unroll
+        for (int r = 0; r < R; ++r) S[r] = fmaf(alpha, S[r], kt[r] * w);
+        float po[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < R; ++r) po[r & 3] = fmaf(qt[r], S[r], po[r & 3]);
+        float o = (po[0] + po[1]) + (po[2] + po[3]);
+        o += __shfl_xor_sync(0xffffffffu, o, 1);
+        const int64_t row = (int64_t)(n * L + t) * p.H + h;
+        if (half == 0) static_cast<TIO *>(p.out)[row * D + j] = from_f32<TIO>(o * p.scale);
+        if (MODE == kVerify) {
+            float *c = p.cache + row * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+            for (int r = 0; r < R; ++r) c[(int64_t)r * D] = S[r];
+        }
+    }
+    if (MODE == kReplay) {
+        float *s1 = p.pool + ((int64_t)slot * p.H + h) * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+        for (int r = 0; r < R; ++r) s1[(int64_t)r * D] = S[r];
+    }
+}
+
+// Gather-scatter of accepted states: CTA (x, n*H + h) copies its share of state_cache[n, r-1, h]
+// into state_pool[slots[n], h] as 16-byte words.
+__global__ void __launch_bounds__(256) gdn_decode_commit_kernel(float *pool, const int32_t *slots,
+                                                                const float *cache, const int32_t *accepted,
+                                                                int32_t *status, int H, int L, int P, int DD) {
+    const int unit = blockIdx.y, n = unit / H, h = unit % H;
+    const int r = accepted[n], slot = slots[n];
+    if (r < 0 || r > L || slot < 0 || slot >= P) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag_bad(status);
+        return;
+    }
+    if (r == 0) return;
+    const float4 *src = reinterpret_cast<const float4 *>(cache + ((int64_t)(n * L + r - 1) * H + h) * DD);
+    float4 *dst = reinterpret_cast<float4 *>(pool + ((int64_t)slot * H + h) * DD);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < DD / 4; i += gridDim.x * blockDim.x) dst[i] = src[i];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+gdn_status check_desc(const gdn_decode_desc *d) {
+    if (!d || d->num_seqs < 1 || d->num_heads < 1 || d->d_k < 1 || d->d_v < 1 || d->num_tokens < 1 ||
+        d->pool_slots < 1 || d->reserved != 0)
+        return GDN_ERR_INVALID_ARG;
+    if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return GDN_ERR_INVALID_ARG;
+    if (d->d_k != d->d_v || (d->d_k != 32 && d->d_k != 64 && d->d_k != 128)) return GDN_ERR_UNSUPPORTED;
+    if (d->num_tokens > 64) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+template <typename TIO, int D, int MODE>
+gdn_status launch_steps(const DecodeParams &p, size_t smem, cudaStream_t s) {
+    auto fn = gdn_decode_kernel<TIO, D, MODE>;
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    fn<<<p.N * p.H, 2 * D, smem, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+template <int MODE>
+gdn_status run_steps(const gdn_decode_desc *d, float *pool, const int32_t *slots, const void *q, const void *k,
+                     const void *v, const float *g, const float *beta, void *out, float *cache, int32_t *status,
+                     gdn_stream_t stream) {
+    gdn_status st = check_desc(d);
+    if (st != GDN_OK) return st;
+    if (!pool || !slots || !q || !k || !v || !g || !beta || !out || (MODE == kVerify && !cache))
+        return GDN_ERR_INVALID_ARG;
+    for (const void *t : {(const void *)pool, q, k, v, (const void *)g, (const void *)beta, (const void *)out,
+                          (const void *)cache})
+        if (t && !aligned16(t)) return GDN_ERR_ALIGNMENT;
+    if (!aligned4(slots) || (status && !aligned4(status))) return GDN_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (status && cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return GDN_ERR_CUDA;
+    DecodeParams p{pool, slots, q, k, v, g, beta, out, cache, status, d->num_seqs, d->num_heads, d->num_tokens,
+                   d->pool_slots, 1.0f / std::sqrt((float)d->d_k)};
+    const size_t smem = sizeof(float) * ((size_t)3 * d->num_tokens * d->d_k + 2 * (size_t)d->num_tokens);
+    const bool bf = d->dtype == GDN_BF16;
+    switch (d->d_k) {
+    case 32: return bf ? launch_steps<__nv_bfloat16, 32, MODE>(p, smem, s) : launch_steps<float, 32, MODE>(p, smem, s);
+    case 64: return bf ? launch_steps<__nv_bfloat16, 64, MODE>(p, smem, s) : launch_steps<float, 64, MODE>(p, smem, s);
+    default: return bf ? launch_steps<__nv_bfloat16, 128, MODE>(p, smem, s) : launch_steps<float, 128, MODE>(p, smem, s);
+    }
+}
+
+}  // namespace
+}  // namespace gdn
+
+extern "C" gdn_status gdn_decode_replay(const gdn_decode_desc *desc, float *state_pool, const int32_t *slots,
+                                        const void *q, const void *k, const void *v, const float *g,
+                                        const float *beta, void *out, int32_t *device_status, gdn_stream_t stream) {
+    return gdn::run_steps<gdn::kReplay>(desc, state_pool, slots, q, k, v, g, beta, out, nullptr, device_status,
+                                        stream);
+}
+
+extern "C" gdn_status gdn_decode_verify(const gdn_decode_desc *desc, const float *state_pool, const int32_t *slots,
+                                        const void *q, const void *k, const void *v, const float *g,
+                                        const float *beta, void *out, float *state_cache, int32_t *device_status,
+                                        gdn_stream_t stream) {
+    return gdn::run_steps<gdn::kVerify>(desc, const_cast<float *>(state_pool), slots, q, k, v, g, beta, out,
+                                        state_cache, device_status, stream);
+}
+
+extern "C" gdn_status gdn_decode_commit(const gdn_decode_desc *desc, float *state_pool, const int32_t *slots,
+                                        const float *state_cache, const int32_t *accepted, int32_t *device_status,
+                                        gdn_stream_t stream) {
+    gdn_status st = gdn::check_desc(desc);
+    if (st != GDN_OK) return st;
+    if (!state_pool || !slots || !state_cache || !accepted) return GDN_ERR_INVALID_ARG;
+    if (!gdn::aligned16(state_pool) || !gdn::aligned16(state_cache)) return GDN_ERR_ALIGNMENT;
+    if (!gdn::aligned4(slots) || !gdn::aligned4(accepted) || (device_status && !gdn::aligned4(device_status)))
+        return GDN_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (device_status && cudaMemsetAsync(device_status, 0, sizeof(int32_t), s) != cudaSuccess) return GDN_ERR_CUDA;
+    if ((int64_t)desc->num_seqs * desc->num_heads > 65535) return GDN_ERR_UNSUPPORTED;
+    const int DD = desc->d_k * desc->d_v;
+    const int blocks_x = std::max(1, std::min(8, DD / 4 / 256));
+    dim3 grid(blocks_x, desc->num_seqs * desc->num_heads);
+    gdn::gdn_decode_commit_kernel<<<grid, 256, 0, s>>>(state_pool, slots, state_cache, accepted, device_status,
+                                                       desc->num_heads, desc->num_tokens, desc->pool_slots, DD);
+    return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}

@@ -236,3 +236,46 @@ def make_problem(wl: Workload | str, seed: int = 0, device="cpu") -> Problem:
                                     dtype=wl.dtype, g_lo=wl.g_lo, beta_std=wl.beta_std,
                                     conv_width=wl.conv_width, conv_std=wl.conv_std,
                                     seed=seed, device=device)
+
+
+# ----------------------------------------------------------------------------- decode side
+@dataclasses.dataclass
+class DecodeProblem:
+    """One decode call's inputs: a state pool, the pool row of each sequence, and L tokens per
+    sequence (layouts of include/gdn_decode.h)."""
+    state_pool: torch.Tensor   # [P, H, d, d] fp32
+    slots: torch.Tensor        # [N] int32
+    q: torch.Tensor            # [N, L, H, d]
+    k: torch.Tensor
+    v: torch.Tensor
+    g: torch.Tensor            # [N, L, H] fp32
+    beta: torch.Tensor
+
+
+DECODE_WORKLOADS = {
+    # the pages' serving shape: 8 concurrent sequences; one block of B = 4 tokens per replay and
+    # K = 4 drafted candidates per verify
+    "decode_8seq_h32_d128_L4": dict(num_seqs=8, num_heads=32, d=128, num_tokens=4, pool_slots=64),
+    "decode_64seq_h32_d128_L4": dict(num_seqs=64, num_heads=32, d=128, num_tokens=4, pool_slots=128),
+}
+
+
+def make_decode_problem(num_seqs: int, num_heads: int, d: int, num_tokens: int, pool_slots: int,
+                        dtype: str = "bf16", g_lo: float = -0.1, beta_std: float = 1.0,
+                        state_std: float = 0.3, seed: int = 0, device="cpu") -> DecodeProblem:
+    """Seeded decode inputs: pool rows ~ N(0, state_std^2), slots a seeded permutation prefix of
+    the pool rows, tokens drawn like the forward workloads (unit q, k; v ~ N(0,1);
+    g ~ U(g_lo, 0); beta = sigmoid(N(0, beta_std^2)))."""
+    tdt = {"bf16": torch.bfloat16, "fp32": torch.float32}[dtype]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    N, H, L = num_seqs, num_heads, num_tokens
+    normal = lambda *s: torch.randn(*s, generator=gen, device=device, dtype=torch.float32)
+    pool = (normal(pool_slots, H, d, d) * state_std).contiguous()
+    slots = torch.randperm(pool_slots, generator=gen, device=device)[:N].to(torch.int32).contiguous()
+    q = _unit_rows(normal(N, L, H, d)).to(tdt)
+    k = _unit_rows(normal(N, L, H, d)).to(tdt)
+    v = normal(N, L, H, d).to(tdt)
+    g = (torch.rand(N, L, H, generator=gen, device=device) * g_lo).contiguous()
+    beta = torch.sigmoid(normal(N, L, H) * beta_std).contiguous()
+    return DecodeProblem(state_pool=pool, slots=slots, q=q, k=k, v=v, g=g, beta=beta)

@@ -13,13 +13,14 @@ import torch
 from gated_deltanet_dual_b200 import binding as b
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "gdn_dual.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder pointers: host-only check")
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    src = "\n".join(open(h).read() for h in HEADERS)
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(gdn_[a-z_]+)\s*\(",
                                  src, flags=re.M)))
@@ -28,13 +29,14 @@ def declared_functions():
 def test_header_declares_entry_points():
     names = declared_functions()
     assert "gdn_dual_forward" in names and "gdn_dual_workspace_size" in names
+    assert {"gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit"} <= set(names)
     assert set(b.EXPORTED) <= set(names)
 
 
 def test_library_exports_every_declared_symbol():
     lib = b.load_library()
     for name in declared_functions():
-        assert hasattr(lib, name), f"{name} declared in include/gdn_dual.h but not exported"
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
 
 
 def test_version_and_status_strings():
@@ -177,3 +179,61 @@ def test_auto_selects_tensor_core_kernel_where_supported():
     assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 64, b.GDN_BF16)) == b.ALGO_SEQUENTIAL
     assert b.select_algo(b.make_desc(2, 16, 64, 64, 2, 4, b.GDN_BF16)) == b.ALGO_SEQUENTIAL
     assert b.select_algo(b.make_desc(2, 16, 128, 128, 2, 4, b.GDN_FP32)) == b.ALGO_SEQUENTIAL
+
+
+def _decode_call(fn, desc, **over):
+    base = 0x7f0000000000
+    names = ["pool", "slots", "q", "k", "v", "g", "beta", "out", "cache", "accepted", "status"]
+    ptr = {n: base + 0x10000000 * i for i, n in enumerate(names)}
+    ptr["status"] = None
+    ptr.update(over)
+    lib = b.load_library()
+    p = lambda n: None if ptr[n] is None else ctypes.c_void_p(ptr[n])
+    d = ctypes.byref(desc)
+    if fn == "replay":
+        return lib.gdn_decode_replay(d, p("pool"), p("slots"), p("q"), p("k"), p("v"), p("g"), p("beta"),
+                                     p("out"), p("status"), None)
+    if fn == "verify":
+        return lib.gdn_decode_verify(d, p("pool"), p("slots"), p("q"), p("k"), p("v"), p("g"), p("beta"),
+                                     p("out"), p("cache"), p("status"), None)
+    return lib.gdn_decode_commit(d, p("pool"), p("slots"), p("cache"), p("accepted"), p("status"), None)
+
+
+@no_gpu
+@pytest.mark.parametrize("fn", ["replay", "verify", "commit"])
+@pytest.mark.parametrize("case,expect", [
+    ("zero_seqs", b.GDN_ERR_INVALID_ARG), ("zero_tokens", b.GDN_ERR_INVALID_ARG),
+    ("zero_pool", b.GDN_ERR_INVALID_ARG), ("reserved", b.GDN_ERR_INVALID_ARG),
+    ("bad_dtype", b.GDN_ERR_INVALID_ARG), ("d48", b.GDN_ERR_UNSUPPORTED), ("dk_ne_dv", b.GDN_ERR_UNSUPPORTED),
+    ("L65", b.GDN_ERR_UNSUPPORTED), ("null_pool", b.GDN_ERR_INVALID_ARG), ("null_slots", b.GDN_ERR_INVALID_ARG),
+    ("misaligned_pool", b.GDN_ERR_ALIGNMENT), ("misaligned_slots", b.GDN_ERR_ALIGNMENT),
+    ("valid_no_device", b.GDN_ERR_CUDA),
+])
+def test_decode_host_validation(fn, case, expect):
+    d = b.make_decode_desc(2, 4, 64, 64, 4, 8, b.GDN_BF16)
+    over = {}
+    if case == "zero_seqs":
+        d.num_seqs = 0
+    elif case == "zero_tokens":
+        d.num_tokens = 0
+    elif case == "zero_pool":
+        d.pool_slots = 0
+    elif case == "reserved":
+        d.reserved = 3
+    elif case == "bad_dtype":
+        d.dtype = 7
+    elif case == "d48":
+        d.d_k = d.d_v = 48
+    elif case == "dk_ne_dv":
+        d.d_v = 32
+    elif case == "L65":
+        d.num_tokens = 65
+    elif case == "null_pool":
+        over["pool"] = None
+    elif case == "null_slots":
+        over["slots"] = None
+    elif case == "misaligned_pool":
+        over["pool"] = 0x7f0000000008
+    elif case == "misaligned_slots":
+        over["slots"] = 0x7f0000000002
+    assert _decode_call(fn, d, **over) == expect
