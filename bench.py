@@ -291,6 +291,174 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- decode side
+DECODE_METRIC = "decode-side GDN state cycle (verify K + commit + replay) tokens/s on 1 B200 and % of HBM roofline"
+
+
+def decode_bytes(N, H, d, L, n_accepted, io_bytes=2):
+    """Algorithmic HBM bytes of the three decode kernels (fp32 states, bf16 tokens)."""
+    st = d * d * 4
+    tok = 3 * d * io_bytes + 8 + d * io_bytes            # q, k, v, g, beta in; o out
+    return {"verify": N * H * (st + L * st + L * tok), "commit": n_accepted * H * 2 * st,
+            "replay": N * H * (2 * st + L * tok)}
+
+
+def time_decode_oracle(cfg, seed=0, min_seconds=1.0):
+    import oracle  # test infrastructure: the CPU baseline / reference arm only
+    pr = synth.make_decode_problem(**cfg, dtype="bf16", seed=seed, device="cpu")
+    acc = np.random.Generator(np.random.PCG64(seed)).integers(0, cfg["num_tokens"] + 1, cfg["num_seqs"])
+    pool = pr.state_pool.double().numpy()
+    slots = pr.slots.numpy()
+    threads = min(host_cores(), cfg["num_seqs"] * cfg["num_heads"])
+    n, t0 = 0, time.perf_counter()
+    while True:
+        S0 = pool[slots]
+        rec = oracle.decode_steps(S0, pr.q, pr.k, pr.v, pr.g, pr.beta, record_states=True, num_threads=threads)
+        pool = oracle.commit(pool, slots, rec["states"], acc)
+        rep = oracle.decode_steps(pool[slots], pr.q, pr.k, pr.v, pr.g, pr.beta, num_threads=threads)
+        pool[slots] = rep["final_state"]
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    toks = cfg["num_seqs"] * cfg["num_tokens"]
+    return {"value": toks * n / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"the whole workload ({cfg['num_seqs']} sequences x {cfg['num_heads']} heads x "
+                      f"{cfg['num_tokens']} tokens), {n} verify+commit+replay cycles, fp64",
+            "seconds_per_step": el / n}
+
+
+def run_decode(args, name, rank, world, local):
+    cfg = synth.DECODE_WORKLOADS[name]
+    N, H, d, L, P = cfg["num_seqs"], cfg["num_heads"], cfg["d"], cfg["num_tokens"], cfg["pool_slots"]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = time_decode_oracle(cfg, min_seconds=2.0)
+        line = {"metric": DECODE_METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["seconds_per_step"] * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": name, "parallelism": "replicas", "l2": "not applicable (host)"},
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    replicas.init(world, backend="nccl", device=dev)
+    seed = replicas.replica_seed(0, rank)
+    pr = synth.make_decode_problem(**cfg, dtype="bf16", seed=seed, device=dev)
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed + 1)
+    accepted = torch.randint(0, L + 1, (N,), generator=gen, dtype=torch.int32).to(dev)
+    n_acc = int((accepted > 0).sum())
+    out_v = torch.empty(N, L, H, d, dtype=pr.q.dtype, device=dev)
+    out_r = torch.empty_like(out_v)
+    cache = torch.empty(N, L, H, d, d, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)    # > L2, rewritten between steps
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        gb.decode_verify(pr.state_pool, pr.slots, pr.q, pr.k, pr.v, pr.g, pr.beta, out=out_v, state_cache=cache)
+        if ev:
+            ev[1].record(stream)
+        gb.decode_commit(pr.state_pool, pr.slots, cache, accepted)
+        if ev:
+            ev[2].record(stream)
+        gb.decode_replay(pr.state_pool, pr.slots, pr.q, pr.k, pr.v, pr.g, pr.beta, out=out_r)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        replicas.barrier(world)
+        torch.cuda.synchronize()
+        clocks.mark_start()
+        for i in range(args.steps):
+            flush.zero_()                   # L2 flushed before every timed step (outside its events)
+            step(evs[i])
+        clocks.poll_until(evs[-1][3])
+        torch.cuda.synchronize()
+        clocks.mark_stop()
+        replicas.barrier(world)
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]),
+                     e[0].elapsed_time(e[3])] for e in evs])
+    step_ms = replicas.max_over_ranks(float(per[:, 3].mean()), world, device=dev)
+    kms = {k: replicas.max_over_ranks(float(per[:, i].mean()), world, device=dev)
+           for i, k in enumerate(("verify", "commit", "replay"))}
+    by = decode_bytes(N, H, d, L, n_acc)
+    peaks = measured_peaks()
+    kernels = {k: {"ms": kms[k], "algorithmic_bytes": by[k], "GBps": by[k] / (kms[k] / 1e3) / 1e9,
+                   "frac": by[k] / (kms[k] / 1e3) / 1e9 / peaks["hbm_gbs"]} for k in kms}
+    roofline = {"bound": "hbm", "achieved": kernels["verify"]["GBps"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": kernels["verify"]["frac"], "traffic": None, "peak_source": peaks["source"],
+                "kernel": "gdn_decode_kernel (verify)", "kernels": kernels,
+                "step_frac": sum(by.values()) / (step_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+    toks = N * L * world
+    value = toks / (step_ms / 1e3)
+
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k", "v", "g", "beta"]
+        host = {n: getattr(pr, n).cpu().pin_memory() for n in names}
+        h_acc = accepted.cpu().pin_memory()
+        h_ov, h_or = (torch.empty(out_v.shape, dtype=out_v.dtype, pin_memory=True) for _ in range(2))
+        dbuf = {n: torch.empty_like(getattr(pr, n)) for n in names}
+        d_acc = torch.empty_like(accepted)
+
+        def e2e_step():
+            for n in names:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            d_acc.copy_(h_acc, non_blocking=True)
+            gb.decode_verify(pr.state_pool, pr.slots, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
+                             out=out_v, state_cache=cache)
+            gb.decode_commit(pr.state_pool, pr.slots, cache, d_acc)
+            gb.decode_replay(pr.state_pool, pr.slots, dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
+                             out=out_r)
+            h_ov.copy_(out_v, non_blocking=True)
+            h_or.copy_(out_r, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ns = max(3, args.steps)
+        a.record(stream)
+        for _ in range(ns):
+            e2e_step()
+        z.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = replicas.max_over_ranks(a.elapsed_time(z) / ns, world, device=dev)
+        h2d = sum(t.numel() * t.element_size() for t in host.values()) + h_acc.numel() * 4
+        e2e = {"value": toks / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(2 * h_ov.numel() * h_ov.element_size()), "ms_per_step": e2e_ms,
+               "steps": ns}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = time_decode_oracle(cfg, min_seconds=2.0)
+        cpu_baseline = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    replicas.shutdown(world)
+    if rank != 0:
+        return
+    line = {"metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": name, "sequences": N, "heads": H, "d": d, "tokens_per_call": L,
+                       "pool_slots": P, "accepted": accepted.tolist(), "parallelism": f"replicas x{world}",
+                       "l2": "flushed before every timed step (256 MB write, outside the step's events)"},
+            "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+            "gpu_launches": 3 * args.steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -305,6 +473,9 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = replicas.env_rank()
+    if args.workload in synth.DECODE_WORKLOADS:
+        run_decode(args, args.workload, rank, world, local)
+        return
     wl = synth.get_workload(args.workload)
 
     if args.impl == "reference":

@@ -8,10 +8,10 @@
 // S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T, o_t = S_t^T q_t / sqrt(d_k).
 //
 // Decode work is small and bound by moving states (d_k x d_v fp32 per sequence and head), so the
-// kernels are CUDA-core kernels sized for bandwidth: one CTA per (sequence, head), the state in
-// registers (thread t owns column t/2 and half of its rows, so k^T S and S^T q need only a pair
-// shuffle), the block's tokens staged once in shared memory, and every state row read or written
-// as whole 32-byte sectors.
+// kernels are CUDA-core kernels sized for bandwidth: a (sequence, head) is split over CTAs of 32
+// state columns, the columns in registers (thread t owns column t/2 and half of its rows, so
+// k^T S and S^T q need only a pair shuffle), the block's tokens staged once in shared memory, and
+// every state row segment read or written as whole 32-byte sectors.
 #include <algorithm>
 #include <cmath>
 
@@ -39,54 +39,77 @@ __device__ __forceinline__ void flag_bad(int32_t *status) {
     if (status) atomicExch(status, (int32_t)GDN_ERR_INVALID_ARG);
 }
 
+// Columns of S per CTA.  Every column of the state evolves on its own (u_j = k^T S[:, j], and the
+// update and the readout of column j read only column j), so a (sequence, head) is split over
+// D / kCols CTAs for memory-level parallelism.
+constexpr int kCols = 32;
+
 template <typename TIO, int D, int MODE>
-__global__ void __launch_bounds__(2 * D) gdn_decode_kernel(const DecodeParams p) {
-    constexpr int R = D / 2;
-    extern __shared__ float sh[];            // q [L][D], k [L][D], v [L][D], g [L], beta [L]
-    const int n = blockIdx.x / p.H, h = blockIdx.x % p.H;
-    const int tid = threadIdx.x, j = tid >> 1, half = tid & 1;
+__global__ void __launch_bounds__(2 * kCols) gdn_decode_kernel(const DecodeParams p) {
+    constexpr int R = D / 2, NCB = D / kCols;
+    extern __shared__ float4 sh4[];          // q [L][D], k [L][D], v [L][D], g [L], beta [L]
+    float *sh = reinterpret_cast<float *>(sh4);
+    const int unit = blockIdx.x / NCB, cb = blockIdx.x % NCB;
+    const int n = unit / p.H, h = unit % p.H;
+    const int tid = threadIdx.x, j = cb * kCols + (tid >> 1), half = tid & 1;
     const int slot = p.slots[n];
     if (slot < 0 || slot >= p.P) {           // uniform over the CTA
-        if (tid == 0) flag_bad(p.status);
+        if (tid == 0 && cb == 0) flag_bad(p.status);
         return;
     }
     const int L = p.L;
     float *sq = sh, *sk = sh + L * D, *sv = sh + 2 * L * D, *sg = sh + 3 * L * D, *sb = sg + L;
+    // the state column first (its loads are the long pole), then the tokens
+    float S[R];
+    const float *s0 = p.pool + ((int64_t)slot * p.H + h) * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+    for (int r = 0; r < R; ++r) S[r] = s0[(int64_t)r * D];
     const TIO *q = static_cast<const TIO *>(p.q), *k = static_cast<const TIO *>(p.k), *v = static_cast<const TIO *>(p.v);
-    for (int i = tid; i < L * D; i += 2 * D) {
+    for (int i = tid; i < L * D; i += 2 * kCols) {
         const int t = i / D, c = i % D;
         const int64_t src = ((int64_t)(n * L + t) * p.H + h) * D + c;
         sq[i] = to_f32(q[src]);
         sk[i] = to_f32(k[src]);
         sv[i] = to_f32(v[src]);
     }
-    for (int t = tid; t < L; t += 2 * D) {
+    for (int t = tid; t < L; t += 2 * kCols) {
         const int64_t src = (int64_t)(n * L + t) * p.H + h;
         sg[t] = p.g[src];
         sb[t] = p.beta[src];
     }
-    float S[R];
-    const float *s0 = p.pool + ((int64_t)slot * p.H + h) * D * D + (int64_t)(half * R) * D + j;
-#pragma unroll
-    for (int r = 0; r < R; ++r) S[r] = s0[(int64_t)r * D];
     __syncthreads();
 
     for (int t = 0; t < L; ++t) {
-        const float *kt = sk + t * D + half * R, *qt = sq + t * D + half * R;
+        const float4 *kt = reinterpret_cast<const float4 *>(sk + t * D + half * R);
+        const float4 *qt = reinterpret_cast<const float4 *>(sq + t * D + half * R);
         const float alpha = expf(sg[t]), b = sb[t];
         // u_j = (k^T S)_j: four partial sums shorten the dependent chain
         float pu[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int r = 0; r < R; ++r) pu[r & 3] = fmaf(kt[r], S[r], pu[r & 3]);
+        for (int r4 = 0; r4 < R / 4; ++r4) {
+            const float4 kk = kt[r4];
+            pu[0] = fmaf(kk.x, S[4 * r4], pu[0]);
+            pu[1] = fmaf(kk.y, S[4 * r4 + 1], pu[1]);
+            pu[2] = fmaf(kk.z, S[4 * r4 + 2], pu[2]);
+            pu[3] = fmaf(kk.w, S[4 * r4 + 3], pu[3]);
+        }
         float u = (pu[0] + pu[1]) + (pu[2] + pu[3]);
         u += __shfl_xor_sync(0xffffffffu, u, 1);
         // S <- alpha S + beta k (v - alpha u)^T   ( = alpha (I - beta k k^T) S + beta k v^T )
         const float w = b * (sv[t * D + j] - alpha * u);
-#pragma unroll
-        for (int r = 0; r < R; ++r) S[r] = fmaf(alpha, S[r], kt[r] * w);
         float po[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int r = 0; r < R; ++r) po[r & 3] = fmaf(qt[r], S[r], po[r & 3]);
+        for (int r4 = 0; r4 < R / 4; ++r4) {
+            const float4 kk = kt[r4], qq = qt[r4];
+            S[4 * r4] = fmaf(alpha, S[4 * r4], kk.x * w);
+            S[4 * r4 + 1] = fmaf(alpha, S[4 * r4 + 1], kk.y * w);
+            S[4 * r4 + 2] = fmaf(alpha, S[4 * r4 + 2], kk.z * w);
+            S[4 * r4 + 3] = fmaf(alpha, S[4 * r4 + 3], kk.w * w);
+            po[0] = fmaf(qq.x, S[4 * r4], po[0]);
+            po[1] = fmaf(qq.y, S[4 * r4 + 1], po[1]);
+            po[2] = fmaf(qq.z, S[4 * r4 + 2], po[2]);
+            po[3] = fmaf(qq.w, S[4 * r4 + 3], po[3]);
+        }
         float o = (po[0] + po[1]) + (po[2] + po[3]);
         o += __shfl_xor_sync(0xffffffffu, o, 1);
         const int64_t row = (int64_t)(n * L + t) * p.H + h;
@@ -139,7 +162,7 @@ gdn_status launch_steps(const DecodeParams &p, size_t smem, cudaStream_t s) {
     auto fn = gdn_decode_kernel<TIO, D, MODE>;
     if (smem > 48 * 1024 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GDN_ERR_CUDA;
-    fn<<<p.N * p.H, 2 * D, smem, s>>>(p);
+    fn<<<p.N * p.H * (D / kCols), 2 * kCols, smem, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
