@@ -222,8 +222,10 @@ __device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int la
 }
 
 // Noisy rows, step 2: Z_j = Gammatil_B q~_j + (-Y~ K~)_j over the q~ row (d columns [64ch, 64ch+64)).
-__device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int ch, int rho, float gend) {
-    const float Gend = exp2f(gend);
+// zs: a row scale applied on the way out (Gamma_e of the row's block boundary when the chunk's
+// decays factorise, so the later Gamma_e Z pass is not needed; else 1).
+__device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int ch, int rho, float gend, float zs) {
+    const float Gend = exp2f(gend) * zs;
     uint8_t *nq = sm + OFF_NQ + ch * 16384;
     float ykb[2][32];
     tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch), ykb[0]);
@@ -238,7 +240,7 @@ __device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int 
             float z[8];
             unpack8(*reinterpret_cast<const uint4 *>(nq + o), z);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) z[e] = fmaf(Gend, z[e], yk[8 * c4 + e]);
+            for (int e = 0; e < 8; ++e) z[e] = fmaf(Gend, z[e], zs * yk[8 * c4 + e]);
             *reinterpret_cast<uint4 *>(nq + o) = pack8(z);
         }
     }
@@ -1027,7 +1029,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     }
                 }
             }
-            if (noisy) z_epilogue(sm, tb, q, ch, rho, gend);
+            if (noisy) {
+                const int eb = ((rho & 63) / B) * B - 1;     // the row's block boundary (-1: S0)
+                z_epilogue(sm, tb, q, ch, rho, gend, (fact && eb >= 0) ? s_E[eb] : 1.f);
+            }
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
@@ -1065,26 +1070,34 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 tmem_wait_ld();
                 const int jj = rho & 63;
                 const int e = (jj / B) * B - 1;          // chunk-local boundary row (-1: S0)
-                auto body = [&](auto F) {
+                if (fact) {
+                    // the rows already hold Gamma_e Z: M'_Z = (Gamma_e Z K^T) e^{-gamma_i} [i <= e]
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int i = 32 * ch + c;
-                        zk[c] = (i <= e) ? zk[c] * decay(F, e < 0 ? 0 : e, i) : 0.f;
+                        zk[c] = (i <= e) ? zk[c] * s_F[i] : 0.f;
                     }
-                };
-                if (fact) body(std::true_type{}); else body(std::false_type{});
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int i = 32 * ch + c;
+                        zk[c] = (i <= e) ? zk[c] * exp2f(fminf(s_gam[e < 0 ? 0 : e] - s_gam[i], 0.f)) : 0.f;
+                    }
+                }
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
                     *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
-                const float Ge = e >= 0 ? s_E[e] : 1.f;        // Gamma_e (1 for e = -1)
-                uint8_t *zrow = sm + OFF_NQ + ch * 16384;
+                if (!fact) {                      // Z <- Gamma_e Z for the state product
+                    const float Ge = e >= 0 ? s_E[e] : 1.f;    // Gamma_e (1 for e = -1)
+                    uint8_t *zrow = sm + OFF_NQ + ch * 16384;
 #pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    float f[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(zrow + sw128_off(rho, c8)), f);
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        float f[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(zrow + sw128_off(rho, c8)), f);
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) f[x] *= Ge;
-                    *reinterpret_cast<uint4 *>(zrow + sw128_off(rho, c8)) = pack8(f);
+                        for (int x = 0; x < 8; ++x) f[x] *= Ge;
+                        *reinterpret_cast<uint4 *>(zrow + sw128_off(rho, c8)) = pack8(f);
+                    }
                 }
             }
             fence_async_smem();
