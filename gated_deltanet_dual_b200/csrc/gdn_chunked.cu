@@ -260,9 +260,10 @@ __device__ __forceinline__ float4 *wrow4(float *w, int r, int c4) {
 // Lane (g = lane / NC, cl = lane % NC) holds column cb + cl for the rows g + RG*i.  X moves between
 // the lanes by shuffles, so the warp needs no barrier; T11[k][c] = 0 for k < c lets the first
 // product start at k = cb, and the second product of row r stops at k = r (warp-uniform bounds).
-// The result goes to dst[(row, col)] via `store` (block-local row and column).
-template <int S, int NC, typename Store>
-__device__ __forceinline__ void warp_merge(const float *sa, int o, int cb, int lane, Store store) {
+// The result goes out through `store` (block-local row and column) after `before_store()`, which
+// separates this warp's reads from other warps' writes when several warps share one merge.
+template <int S, int NC, typename Store, typename Sync>
+__device__ __forceinline__ void warp_merge(const float *sa, int o, int cb, int lane, Store store, Sync before_store) {
     constexpr int RG = 32 / NC, NR = S / RG;
     const int cl = lane % NC, g = lane / NC, c = cb + cl;
     float x[NR];
@@ -296,73 +297,17 @@ __device__ __forceinline__ void warp_merge(const float *sa, int o, int cb, int l
             }
         }
     }
+    before_store();
 #pragma unroll
     for (int i = 0; i < NR; ++i) store(g + RG * i, c, -y[i]);
 }
 
-// One merge level of the triangular inverse: for every pair of S x S diagonal blocks at offset
-// o (already inverted), X = A[o+S.., o..] T[o.., o..] and T[o+S.., o..] = -T[o+S.., o+S..] X.
-// NT threads (t = 0..NT-1 when `active`): column c, rows g + RG*i.  T[o+S.., o+S..] is unit lower
-// triangular, so the second product of row r stops at k = r.  `side`: barrier of warps 1..7.
-template <int S, int NT>
-__device__ __forceinline__ void tri_merge(float *sa, float *xb, int t, bool active, bool side) {
-    constexpr int RG = NT / 32;                // row groups per merge
-    constexpr int NR = S / RG;                 // rows per thread
-    const int c = t % S, g = (t / S) % RG, m = t / (S * RG), o = m * 2 * S;
-    float *X = xb + m * S * S;
-    float acc[NR], acc2[NR];
-    if (active) {
-#pragma unroll
-        for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
-#pragma unroll
-        for (int k = 0; k < S; k += 8) {
-            float tv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) tv[e] = sa[sidx(o + k + e, o + c)];
-#pragma unroll
-            for (int i = 0; i < NR; ++i) {
-                const float4 a = *srow4(sa, o + S + g + RG * i, o + k);
-                const float4 b = *srow4(sa, o + S + g + RG * i, o + k + 4);
-                acc[i] = fmaf(a.x, tv[0], fmaf(a.y, tv[1], fmaf(a.z, tv[2], fmaf(a.w, tv[3], acc[i]))));
-                acc2[i] = fmaf(b.x, tv[4], fmaf(b.y, tv[5], fmaf(b.z, tv[6], fmaf(b.w, tv[7], acc2[i]))));
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < NR; ++i) X[(g + RG * i) * S + c] = acc[i] + acc2[i];
-    }
-    if (side) bar_side(); else bar_math();
-    if (active) {
-        const int gmax = g | (32 / S - 1);     // largest row group in this warp
-#pragma unroll
-        for (int i = 0; i < NR; ++i) acc[i] = acc2[i] = 0.f;
-#pragma unroll
-        for (int k = 0; k < S; k += 8) {
-            if (k <= gmax + RG * (NR - 1)) {
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = X[(k + e) * S + c];
-#pragma unroll
-                for (int i = 0; i < NR; ++i) {
-                    if (k <= gmax + RG * i) {
-                        const float4 a = *srow4(sa, o + S + g + RG * i, o + S + k);
-                        const float4 b = *srow4(sa, o + S + g + RG * i, o + S + k + 4);
-                        acc[i] = fmaf(a.x, x[0], fmaf(a.y, x[1], fmaf(a.z, x[2], fmaf(a.w, x[3], acc[i]))));
-                        acc2[i] = fmaf(b.x, x[4], fmaf(b.y, x[5], fmaf(b.z, x[6], fmaf(b.w, x[7], acc2[i]))));
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < NR; ++i) sa[sidx(o + S + g + RG * i, o + c)] = -(acc[i] + acc2[i]);
-    }
-    if (side) bar_side(); else bar_math();
-}
-
 // T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch, while warp 0 issues an MMA
-// batch: warps 1-7 invert the eight 8x8 diagonal blocks (one thread per column, right-looking
-// forward substitution) and run the 8- and 16-merges; then all warps run the 32-merge
-// (warp-local, no barrier inside), whose lower-left block goes to the 32 x 32 staging block `wb`
-// (rows 32..63, columns 0..31 of T) so that no warp overwrites A while another still reads it.
+// batch: warps 1-2 invert the eight 8x8 diagonal blocks (one thread per column, right-looking
+// forward substitution), warps 1-4 run the four 8-merges (one warp each, in place) and the two
+// 16-merges (two warps each, in place after a barrier); then all warps run the 32-merge, whose
+// lower-left block goes to the 32 x 32 staging block `wb` (rows 32..63, columns 0..31 of T) so that
+// no warp overwrites A while another still reads it.
 __device__ void solve_T(float *sa, float *wb, int tid, int warp) {
     const int lane = tid & 31;
     if (warp > 0) {
@@ -389,12 +334,24 @@ __device__ void solve_T(float *sa, float *wb, int tid, int warp) {
             for (int jj = 0; jj < 8; ++jj) sa[sidx(o + jj, o + c)] = x[jj];
         }
         bar_side();
-        tri_merge<8, 128>(sa, wb, t, t < 128, true);
-        tri_merge<16, 128>(sa, wb, t, t < 128, true);
+        auto in_place = [sa](int o, int S) {
+            return [sa, o, S](int r, int c, float v) { sa[sidx(o + S + r, o + c)] = v; };
+        };
+        if (warp <= 4) {           // four 8-merges, one warp each (a warp owns its whole merge)
+            const int o = 16 * (warp - 1);
+            warp_merge<8, 8>(sa, o, 0, lane, in_place(o, 8), [] {});
+        }
+        bar_side();
+        if (warp <= 4) {           // two 16-merges, two warps each (8 columns per warp)
+            const int o = 32 * ((warp - 1) >> 1), cb = 8 * ((warp - 1) & 1);
+            warp_merge<16, 8>(sa, o, cb, lane, in_place(o, 16), [] { bar_side(); });
+        } else {
+            bar_side();            // the 16-merges' reads precede their writes
+        }
     }
     bar_math();
     // warp 0 arrives last (it issued the MMA batch): it takes the columns with the least work
-    warp_merge<32, 4>(sa, 0, 4 * (7 - warp), lane, [&](int r, int c, float v) { wb[widx(r, c)] = v; });
+    warp_merge<32, 4>(sa, 0, 4 * (7 - warp), lane, [&](int r, int c, float v) { wb[widx(r, c)] = v; }, [] {});
     bar_math();
 }
 
