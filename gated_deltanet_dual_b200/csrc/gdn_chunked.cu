@@ -133,7 +133,8 @@ __device__ __forceinline__ Unit make_unit(const Params &P, int u) {
 // own I + Atil), then ycoef = y beta~ Gammatil (for Z) and wcoef = y beta~ (for WV).
 template <int B>
 __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float (&wk)[32], int lane, int j,
-                                             const float *ngam, const float *nbeta,
+                                             const float *ngam, const float *nbeta, const float *nE,
+                                             const float *nF, bool nfact,
                                              float (&ycoef)[B], float (&wcoef)[B], float &gend) {
     const int bs = (j / B) * B;
     const int jl = j - bs;
@@ -156,10 +157,20 @@ __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float 
     const float gj = ngam[j], bj = nbeta[j];
     gend = gl[B - 1];
     float arow[B], pt[B], y[B];
+    if (B >= 16 && nfact) {       // e^{gamma~_a - gamma~_b} = E_a F_b, prepared once per row
+        const float Ej = nE[j], Eend = nE[bs + B - 1];
 #pragma unroll
-    for (int l = 0; l < B; ++l) {
-        arow[l] = (l < jl) ? bj * exp2f(fminf(gj - gl[l], 0.f)) * ak[l] : 0.f;
-        pt[l] = aq[l] * exp2f(gend - gl[l]);
+        for (int l = 0; l < B; ++l) {
+            const float Fl = nF[bs + l];
+            arow[l] = (l < jl) ? bj * (Ej * Fl) * ak[l] : 0.f;
+            pt[l] = aq[l] * (Eend * Fl);
+        }
+    } else {
+#pragma unroll
+        for (int l = 0; l < B; ++l) {
+            arow[l] = (l < jl) ? bj * exp2f(fminf(gj - gl[l], 0.f)) * ak[l] : 0.f;
+            pt[l] = aq[l] * exp2f(gend - gl[l]);
+        }
     }
     // Right-looking back substitution: once y_mm is final it is taken out of every earlier
     // position at once, so the dependent chain is B steps of one FMA each.
@@ -173,7 +184,7 @@ __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float 
 #pragma unroll
     for (int l = 0; l < B; ++l) {
         wcoef[l] = y[l] * bl[l];
-        ycoef[l] = wcoef[l] * exp2f(gl[l]);
+        ycoef[l] = wcoef[l] * ((B >= 16 && nfact) ? nE[bs + l] : exp2f(gl[l]));
     }
 }
 
@@ -206,14 +217,16 @@ __device__ __forceinline__ void store_block_row(uint32_t taddr, int ch, int v, i
 // rows of W~ and -Y~ as tensor-memory A operands (columns [0,64) and [64,128) from TM_TK).
 template <int B>
 __device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int lane, int rho,
-                                              const float *s_ngam, const float *s_nbeta) {
+                                              const float *s_ngam, const float *s_nbeta, const float *s_nE,
+                                              const float *s_nF, bool nfact) {
     float wq[32], wk[32];
     tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 32 * q), wq);
     tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 32 * q), wk);
     tmem_wait_ld();
     const int v = rho >> 6, j = rho & 63;
     float ycoef[B], wcoef[B], gend;
-    noisy_coeffs<B>(wq, wk, lane, j, s_ngam + 64 * v, s_nbeta + 64 * v, ycoef, wcoef, gend);
+    noisy_coeffs<B>(wq, wk, lane, j, s_ngam + 64 * v, s_nbeta + 64 * v, s_nE + 64 * v, s_nF + 64 * v, nfact,
+                    ycoef, wcoef, gend);
     bar_math();   // every warp has finished reading TM_TK before it is overwritten
     const int bs = (j / B) * B;
     store_block_row<B>(tmem_addr(tb, q * 32, TM_TK + 32 * ch), ch, v, bs, wcoef, 1.f);
@@ -576,8 +589,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     // Per-chunk scalars, double-buffered so the next chunk's are prepared while this chunk's
     // state phases run: [buffer][gamma | beta | E = 2^gamma | F = 2^-gamma | noisy gamma | noisy beta]
     constexpr int SC_GAM = 0, SC_BETA = CH, SC_E = 2 * CH, SC_F = 3 * CH, SC_NGAM = 4 * CH, SC_NBETA = 6 * CH;
-    __shared__ float s_sc[2][8 * CH];
+    constexpr int SC_NE = 8 * CH, SC_NF = 10 * CH;   // noisy rows: 2^gamma~ and 2^-gamma~ (B >= 16)
+    __shared__ float s_sc[2][(B >= 16 ? 12 : 8) * CH];
     __shared__ int s_okw[2][2];
+    __shared__ int s_okn[2][4];               // every |gamma~| of a 32-row noisy group below 100
     __shared__ float s_g[CH];                 // scan scratch
     __shared__ float s_raw[2][3 * CH];        // [gate, beta][row]: cp.async staging (read before restaged)
     __shared__ uint4 s_halo[3][3][16];        // ShortConv: raw clean rows cstart-3..cstart-1 [q,k,v][row][chunk]
@@ -749,6 +764,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 if (d < B && jl >= d) gv += o2;
             }
             sc[SC_NGAM + idx] = gv;
+            if constexpr (B >= 16) {      // long blocks: the coefficients use precomputed factors
+                sc[SC_NE + idx] = exp2f(gv);
+                sc[SC_NF + idx] = exp2f(-gv);
+                const bool okn = __all_sync(0xffffffffu, fabsf(gv) < 100.f);
+                if (lane == 0) s_okn[buf][idx >> 5] = okn;
+            }
         }
         bar_side();
         if (sr < CH) {
@@ -793,6 +814,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             float *s_gam = s_sc[cb] + SC_GAM, *s_beta = s_sc[cb] + SC_BETA;
             float *s_E = s_sc[cb] + SC_E, *s_F = s_sc[cb] + SC_F;
             float *s_ngam = s_sc[cb] + SC_NGAM, *s_nbeta = s_sc[cb] + SC_NBETA;
+            const float *s_nE = s_sc[cb] + (B >= 16 ? SC_NE : 0), *s_nF = s_sc[cb] + (B >= 16 ? SC_NF : 0);
             if (ci == 0 && warp > 0) {
                 stage_scalars(U, m, rb);
                 prep_scalars(U, m, cb);
@@ -922,7 +944,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             if (noisy) wait_mma2(11);                   // noisy block products of PK1
             // noisy: block coefficients, then W~ and -Y~ rows into TMEM as A operands
             float gend = 0.f;
-            if (noisy) gend = noisy_phase1<B>(tb, q, ch, lane, rho, s_ngam, s_nbeta);
+            if (noisy) {
+                const bool nfact = B >= 16 && s_okn[cb][0] && s_okn[cb][1] && s_okn[cb][2] && s_okn[cb][3];
+                gend = noisy_phase1<B>(tb, q, ch, lane, rho, s_ngam, s_nbeta, s_nE, s_nF, nfact);
+            }
             tmem_wait_st();
             tc_fence_before();
             bar_math();
