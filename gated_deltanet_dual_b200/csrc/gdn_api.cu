@@ -125,6 +125,7 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
     P.N = N; P.H = H; P.dk = desc->d_k; P.dv = desc->d_v; P.V = noisy ? V : 0; P.B = B;
     P.conv_width = desc->conv_width;
     P.num_units = N * H;
+    P.parts = 1;
     P.scale = (float)(1.0 / std::sqrt((double)desc->d_k));
     int64_t roff = 0;
     for (int n = 0; n <= N; ++n) {

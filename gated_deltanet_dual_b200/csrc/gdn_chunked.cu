@@ -650,8 +650,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
 
     // Issue the TMA loads of chunk m of unit U (control lane 0).  group A: [Q;K] and, for a
     // response chunk, [q~;.] and v~;  group B: V and, for a response chunk, [k~;.].
-    auto issue_a = [&](const Unit &U, int m) {
-        const bool nz = (m >= 0) && V > 0;
+    auto issue_a = [&](const Unit &U, int m, bool nz) {
         const int cstart = U.s + U.prompt + CH * m;
         mbar_arrive_expect_tx(&bar_a, 32768u + (nz ? 65536u : 0u));
         for (int hf = 0; hf < 2; ++hf) {
@@ -668,8 +667,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             }
         }
     };
-    auto issue_b = [&](const Unit &U, int m) {
-        const bool nz = (m >= 0) && V > 0;
+    auto issue_b = [&](const Unit &U, int m, bool nz) {
         const int cstart = U.s + U.prompt + CH * m;
         mbar_arrive_expect_tx(&bar_b, 16384u + (nz ? 32768u : 0u));
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_V + hf * 8192, &M.v, &bar_b, hf * 64, U.h, cstart);
@@ -784,8 +782,33 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         }
     };
 
-    for (int u = blockIdx.x; u < P.num_units; u += gridDim.x) {
+    // With few units each one is split over two CTAs: part 0 runs chunks [0, split) in full; part 1
+    // runs [0, split) clean-only (no noisy rows, no outputs: only the state chain, which does not
+    // depend on the noisy stream) and then [split, n) in full.  The split balances the two parts
+    // for a clean-only chunk costing kCleanCost of a full one.
+    constexpr float kCleanCost = 0.45f;
+    const int parts = P.parts;
+    for (int w = blockIdx.x; w < P.num_units * parts; w += gridDim.x) {
+        const int u = w / parts, part = w % parts;
         const Unit U = make_unit(P, u);
+        int ci_full = 0, ci_end = U.nchunks;   // chunks ci < ci_full are clean-only
+        bool final_part = true;
+        if (parts == 2) {
+            if (U.nchunks < 2) {
+                if (part == 0) continue;
+            } else {
+                const int npre = -U.m_first;
+                int split = (int)((U.nchunks + npre * (1.f - kCleanCost)) / (2.f - kCleanCost) + 0.5f);
+                split = max(1, min(U.nchunks - 1, split));
+                if (part == 0) {
+                    ci_end = split;
+                    final_part = false;
+                } else {
+                    ci_full = split;
+                }
+            }
+        }
+        auto chunk_noisy = [&](int ci) { return (U.m_first + ci >= 0) && V > 0 && ci >= ci_full; };
         float S[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) S[c] = 0.f;
@@ -796,20 +819,20 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) *reinterpret_cast<uint4 *>(s0 + sw128_off(rho, c8)) = z;
             fence_async_smem();
-            if (U.nchunks == 0) {
+            if (U.nchunks == 0 && final_part) {
                 float *fs = P.final_state + ((int64_t)U.n * H + U.h) * D * D + (int64_t)rho * D + 64 * ch;
 #pragma unroll
                 for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4 *>(fs + c) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
-        if (tid == 0 && U.nchunks > 0) {
-            issue_a(U, U.m_first);
-            issue_b(U, U.m_first);
+        if (tid == 0 && ci_end > 0) {
+            issue_a(U, U.m_first, chunk_noisy(0));
+            issue_b(U, U.m_first, chunk_noisy(0));
         }
-        for (int ci = 0; ci < U.nchunks; ++ci) {
+        for (int ci = 0; ci < ci_end; ++ci) {
             const int m = U.m_first + ci;
-            const bool noisy = (m >= 0) && V > 0;
-            const bool last = ci == U.nchunks - 1;
+            const bool noisy = chunk_noisy(ci);
+            const bool last = ci == ci_end - 1;
             const int cstart = U.s + U.prompt + CH * m;   // global token of chunk row 0
             float *s_gam = s_sc[cb] + SC_GAM, *s_beta = s_sc[cb] + SC_BETA;
             float *s_E = s_sc[cb] + SC_E, *s_F = s_sc[cb] + SC_F;
@@ -1104,7 +1127,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 // prefetch group A of the next chunk once [Q;K] and Z are consumed
                 if (!last) {
                     if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(40);
-                    else issue_a(U, m + 1);
+                    else issue_a(U, m + 1, chunk_noisy(ci + 1));
                 }
             }
             __syncwarp();
@@ -1113,7 +1136,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             if (rho < 64) {
                 const int t = rho;
                 const int tok = cstart + t;
-                const bool ok = tok >= U.s && tok < U.s + U.len;
+                const bool ok = tok >= U.s && tok < U.s + U.len && ci >= ci_full;
                 const float Gt = s_E[t];
                 __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(P.out) + ((int64_t)tok * H + U.h) * D + 64 * ch;
 #pragma unroll
@@ -1164,7 +1187,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 mma_commit(&bar_mma);
                 if (!last) {
                     if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(50);
-                    else issue_b(U, m + 1);
+                    else issue_b(U, m + 1, chunk_noisy(ci + 1));
                 }
             }
             __syncwarp();
@@ -1185,7 +1208,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8)
                 *reinterpret_cast<uint4 *>(srow + sw128_off(rho, c8)) = pack8(S + 8 * c8);
-            if (last) {
+            if (last && final_part) {
                 float *fs = P.final_state + ((int64_t)U.n * H + U.h) * D * D + (int64_t)rho * D + 64 * ch;
 #pragma unroll
                 for (int c = 0; c < 64; c += 4)
@@ -1291,14 +1314,18 @@ cudaError_t launch_chunked(const Params &p, cudaStream_t stream) {
         attr_err = e;
     });
     if (attr_err != cudaSuccess) return attr_err;
-    const int grid = std::min(p.num_units, num_sms > 0 ? num_sms : 148);
+    // Few units: two CTAs per unit (see the kernel's unit loop).
+    const int sms = num_sms > 0 ? num_sms : 148;
+    Params q = p;
+    q.parts = (noisy && 2 * p.num_units <= sms) ? 2 : 1;
+    const int grid = std::min(p.num_units * q.parts, sms);
     switch (p.B) {
-        case 1: gdn_chunked_kernel<1><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
-        case 2: gdn_chunked_kernel<2><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
-        case 4: gdn_chunked_kernel<4><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
-        case 8: gdn_chunked_kernel<8><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
-        case 16: gdn_chunked_kernel<16><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
-        case 32: gdn_chunked_kernel<32><<<grid, kThreads, SMEM_BYTES, stream>>>(p, maps); break;
+        case 1: gdn_chunked_kernel<1><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
+        case 2: gdn_chunked_kernel<2><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
+        case 4: gdn_chunked_kernel<4><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
+        case 8: gdn_chunked_kernel<8><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
+        case 16: gdn_chunked_kernel<16><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
+        case 32: gdn_chunked_kernel<32><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

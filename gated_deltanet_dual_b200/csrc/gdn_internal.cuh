@@ -34,6 +34,7 @@ struct Params {
     WorkspaceHeader *ws;
     int64_t T, TR;
     int32_t N, H, dk, dv, V, B, conv_width, num_units;
+    int32_t parts;                    // chunked kernel: CTAs per unit (1, or 2 when units are few)
     float scale;                      // 1 / sqrt(d_k)
     int32_t doc_start[kMaxDocs + 1];  // token offset of each document (doc_offsets)
     int32_t doc_prompt[kMaxDocs];     // prompt length of each document
