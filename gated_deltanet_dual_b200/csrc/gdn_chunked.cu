@@ -785,8 +785,9 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     // With few units each one is split over two CTAs: part 0 runs chunks [0, split) in full; part 1
     // runs [0, split) clean-only (no noisy rows, no outputs: only the state chain, which does not
     // depend on the noisy stream) and then [split, n) in full.  The split balances the two parts
-    // for a clean-only chunk costing kCleanCost of a full one.
-    constexpr float kCleanCost = 0.45f;
+    // for a clean-only chunk costing kCleanCost of a full one (lower for long blocks, whose noisy
+    // work weighs more).
+    constexpr float kCleanCost = B >= 32 ? 0.42f : (B >= 16 ? 0.55f : 0.65f);   // measured balance
     const int parts = P.parts;
     for (int w = blockIdx.x; w < P.num_units * parts; w += gridDim.x) {
         const int u = w / parts, part = w % parts;
