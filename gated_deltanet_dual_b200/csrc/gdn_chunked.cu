@@ -578,6 +578,17 @@ __device__ __noinline__ void conv_chunk(uint8_t *sm, uint4 (*halo)[3][16], bool 
     fence_async_smem();                      // the tiles are next read by the tensor cores
 }
 
+// Next work item of the CTA: thread 0 takes one from the workspace counter and broadcasts it (the
+// first gridDim.x items are taken by blockIdx.x at start).  Kept out of line so that the main
+// loop's register allocation does not depend on it.
+__device__ __noinline__ int next_work_item(WorkspaceHeader *ws, int *s_next) {
+    if (threadIdx.x == 0) *s_next = (int)gridDim.x + atomicAdd(&ws->next_unit, 1);
+    __syncthreads();
+    const int nx = *s_next;
+    __syncthreads();                          // read by all before thread 0 writes it again
+    return nx;
+}
+
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps M) {
@@ -788,8 +799,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     // for a clean-only chunk costing kCleanCost of a full one (lower for long blocks, whose noisy
     // work weighs more).
     constexpr float kCleanCost = B >= 32 ? 0.42f : (B >= 16 ? 0.55f : 0.65f);   // measured balance
+    // Work items are (unit, part), longest documents first; each CTA starts with item blockIdx.x and
+    // then takes the next untaken item from a counter in the workspace (greedy list scheduling:
+    // uneven documents no longer pile up on the CTAs that a fixed stride would give them).
     const int parts = P.parts;
-    for (int w = blockIdx.x; w < P.num_units * parts; w += gridDim.x) {
+    __shared__ int s_next;
+    for (int w = blockIdx.x; w < P.num_units * parts; w = next_work_item(P.ws, &s_next)) {
         const int u = w / parts, part = w % parts;
         const Unit U = make_unit(P, u);
         int ci_full = 0, ci_end = U.nchunks;   // chunks ci < ci_full are clean-only
