@@ -8,18 +8,23 @@
 // S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T, o_t = S_t^T q_t / sqrt(d_k).
 //
 // Decode work is small and bound by moving states (d_k x d_v fp32 per sequence and head), so the
-// kernels are CUDA-core kernels sized for bandwidth: a (sequence, head) is split over CTAs of 32
-// state columns, the columns in registers (thread t owns column t/2 and half of its rows, so
-// k^T S and S^T q need only a pair shuffle), the block's tokens staged once in shared memory, and
-// every state row segment read or written as whole 32-byte sectors.
+// kernels are CUDA-core kernels sized for bandwidth: a (sequence, head) is split into items of 32
+// state columns, persistent CTAs prefetch the next item's state slice and tokens with cp.async
+// while they step the current one, the columns live in registers (thread t owns column t/2 and
+// half of its rows, so k^T S and S^T q need only a pair shuffle), and every state row segment is
+// read or written as whole 32-byte sectors.
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 
 #include "gdn_internal.cuh"
 #include "gdn_decode.h"
+#include "sm100.cuh"
 
 namespace gdn {
 namespace {
+
+using namespace sm100;
 
 enum DecodeMode { kReplay = 0, kVerify = 1 };
 
@@ -39,92 +44,154 @@ __device__ __forceinline__ void flag_bad(int32_t *status) {
     if (status) atomicExch(status, (int32_t)GDN_ERR_INVALID_ARG);
 }
 
-// Columns of S per CTA.  Every column of the state evolves on its own (u_j = k^T S[:, j], and the
-// update and the readout of column j read only column j), so a (sequence, head) is split over
-// D / kCols CTAs for memory-level parallelism.
+// Columns of S per work item.  Every column of the state evolves on its own (u_j = k^T S[:, j], and
+// the update and the readout of column j read only column j), so a (sequence, head) is split into
+// D / kCols items of kCols columns.
 constexpr int kCols = 32;
 
+__host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
+
+// Shared-memory bytes of one item buffer: state slice [D][kCols] fp32, q, k, v [L][D] as stored,
+// g and beta [L] fp32.
+template <typename TIO, int D>
+__host__ __device__ constexpr int decode_buf_bytes(int L) {
+    return D * kCols * 4 + 3 * round16(L * D * (int)sizeof(TIO)) + 2 * round16(L * 4);
+}
+
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+
+// Persistent: each CTA walks work items (sequence, head, column slice) with a stride of gridDim.x
+// and prefetches the next item's state slice and tokens into the other shared-memory buffer with
+// cp.async while it runs the current one, so the state reads of one item overlap the steps and
+// the stores of the previous one.
 template <typename TIO, int D, int MODE>
 __global__ void __launch_bounds__(2 * kCols) gdn_decode_kernel(const DecodeParams p) {
     constexpr int R = D / 2, NCB = D / kCols;
-    extern __shared__ float4 sh4[];          // q [L][D], k [L][D], v [L][D], g [L], beta [L]
-    float *sh = reinterpret_cast<float *>(sh4);
-    const int unit = blockIdx.x / NCB, cb = blockIdx.x % NCB;
-    const int n = unit / p.H, h = unit % p.H;
-    const int tid = threadIdx.x, j = cb * kCols + (tid >> 1), half = tid & 1;
-    const int slot = p.slots[n];
-    if (slot < 0 || slot >= p.P) {           // uniform over the CTA
-        if (tid == 0 && cb == 0) flag_bad(p.status);
-        return;
-    }
+    extern __shared__ float4 sh4[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(sh4);
+    const int tid = threadIdx.x, jl = tid >> 1, half = tid & 1;
     const int L = p.L;
-    float *sq = sh, *sk = sh + L * D, *sv = sh + 2 * L * D, *sg = sh + 3 * L * D, *sb = sg + L;
-    // the state column first (its loads are the long pole), then the tokens
-    float S[R];
-    const float *s0 = p.pool + ((int64_t)slot * p.H + h) * D * D + (int64_t)(half * R) * D + j;
-#pragma unroll
-    for (int r = 0; r < R; ++r) S[r] = s0[(int64_t)r * D];
-    const TIO *q = static_cast<const TIO *>(p.q), *k = static_cast<const TIO *>(p.k), *v = static_cast<const TIO *>(p.v);
-    for (int i = tid; i < L * D; i += 2 * kCols) {
-        const int t = i / D, c = i % D;
-        const int64_t src = ((int64_t)(n * L + t) * p.H + h) * D + c;
-        sq[i] = to_f32(q[src]);
-        sk[i] = to_f32(k[src]);
-        sv[i] = to_f32(v[src]);
-    }
-    for (int t = tid; t < L; t += 2 * kCols) {
-        const int64_t src = (int64_t)(n * L + t) * p.H + h;
-        sg[t] = p.g[src];
-        sb[t] = p.beta[src];
-    }
-    __syncthreads();
+    const int tok_bytes = round16(L * D * (int)sizeof(TIO)), sc_bytes = round16(L * 4);
+    const int buf_bytes = decode_buf_bytes<TIO, D>(L);
+    const int total = p.N * p.H * NCB;
 
-    for (int t = 0; t < L; ++t) {
-        const float4 *kt = reinterpret_cast<const float4 *>(sk + t * D + half * R);
-        const float4 *qt = reinterpret_cast<const float4 *>(sq + t * D + half * R);
-        const float alpha = expf(sg[t]), b = sb[t];
-        // u_j = (k^T S)_j: four partial sums shorten the dependent chain
-        float pu[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r4 = 0; r4 < R / 4; ++r4) {
-            const float4 kk = kt[r4];
-            pu[0] = fmaf(kk.x, S[4 * r4], pu[0]);
-            pu[1] = fmaf(kk.y, S[4 * r4 + 1], pu[1]);
-            pu[2] = fmaf(kk.z, S[4 * r4 + 2], pu[2]);
-            pu[3] = fmaf(kk.w, S[4 * r4 + 3], pu[3]);
+    // cp.async the inputs of item w into buffer b; false (and nothing loaded) for a bad slot
+    auto issue_load = [&](int w, int b) -> bool {
+        const int unit = w / NCB, cb = w % NCB;
+        const int n = unit / p.H, h = unit % p.H;
+        const int slot = p.slots[n];
+        if (slot < 0 || slot >= p.P) {
+            if (tid == 0 && cb == 0) flag_bad(p.status);
+            return false;
         }
-        float u = (pu[0] + pu[1]) + (pu[2] + pu[3]);
-        u += __shfl_xor_sync(0xffffffffu, u, 1);
-        // S <- alpha S + beta k (v - alpha u)^T   ( = alpha (I - beta k k^T) S + beta k v^T )
-        const float w = b * (sv[t * D + j] - alpha * u);
-        float po[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r4 = 0; r4 < R / 4; ++r4) {
-            const float4 kk = kt[r4], qq = qt[r4];
-            S[4 * r4] = fmaf(alpha, S[4 * r4], kk.x * w);
-            S[4 * r4 + 1] = fmaf(alpha, S[4 * r4 + 1], kk.y * w);
-            S[4 * r4 + 2] = fmaf(alpha, S[4 * r4 + 2], kk.z * w);
-            S[4 * r4 + 3] = fmaf(alpha, S[4 * r4 + 3], kk.w * w);
-            po[0] = fmaf(qq.x, S[4 * r4], po[0]);
-            po[1] = fmaf(qq.y, S[4 * r4 + 1], po[1]);
-            po[2] = fmaf(qq.z, S[4 * r4 + 2], po[2]);
-            po[3] = fmaf(qq.w, S[4 * r4 + 3], po[3]);
+        uint8_t *buf = smem + b * buf_bytes;
+        const float *st = p.pool + ((int64_t)slot * p.H + h) * D * D + cb * kCols;
+        for (int i = tid; i < D * (kCols / 4); i += 2 * kCols) {
+            const int r = i / (kCols / 4), c4 = i % (kCols / 4);
+            cp_async16(buf + (r * kCols + 4 * c4) * 4, st + (int64_t)r * D + 4 * c4);
         }
-        float o = (po[0] + po[1]) + (po[2] + po[3]);
-        o += __shfl_xor_sync(0xffffffffu, o, 1);
-        const int64_t row = (int64_t)(n * L + t) * p.H + h;
-        if (half == 0) static_cast<TIO *>(p.out)[row * D + j] = from_f32<TIO>(o * p.scale);
-        if (MODE == kVerify) {
-            float *c = p.cache + row * D * D + (int64_t)(half * R) * D + j;
-#pragma unroll
-            for (int r = 0; r < R; ++r) c[(int64_t)r * D] = S[r];
+        constexpr int CPR = D * (int)sizeof(TIO) / 16;   // 16-byte pieces per token row
+        const void *src[3] = {p.q, p.k, p.v};
+        for (int x = 0; x < 3; ++x) {
+            uint8_t *dst = buf + D * kCols * 4 + x * tok_bytes;
+            const uint8_t *s0 = static_cast<const uint8_t *>(src[x]);
+            for (int i = tid; i < L * CPR; i += 2 * kCols) {
+                const int t = i / CPR, c = i % CPR;
+                cp_async16(dst + t * D * (int)sizeof(TIO) + 16 * c,
+                           s0 + (((int64_t)(n * L + t) * p.H + h) * D) * (int64_t)sizeof(TIO) + 16 * c);
+            }
         }
+        float *sg = reinterpret_cast<float *>(buf + D * kCols * 4 + 3 * tok_bytes);
+        float *sb = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(sg) + sc_bytes);
+        for (int t = tid; t < L; t += 2 * kCols) {
+            const int64_t row = (int64_t)(n * L + t) * p.H + h;
+            cp_async4(sg + t, p.g + row, 4);
+            cp_async4(sb + t, p.beta + row, 4);
+        }
+        return true;
+    };
+
+    int w = blockIdx.x, b = 0;
+    bool valid = w < total ? issue_load(w, 0) : false;
+    cp_async_commit();
+    while (w < total) {
+        const int wn = w + gridDim.x;
+        const bool vnext = wn < total ? issue_load(wn, b ^ 1) : false;
+        cp_async_commit();
+        cp_async_wait_group1();               // this item's group has landed (the next may not)
+        __syncthreads();
+        if (valid) {
+            const int unit = w / NCB, cb = w % NCB;
+            const int n = unit / p.H, h = unit % p.H;
+            const int j = cb * kCols + jl;
+            const uint8_t *buf = smem + b * buf_bytes;
+            const float *st = reinterpret_cast<const float *>(buf);
+            const TIO *sq = reinterpret_cast<const TIO *>(buf + D * kCols * 4);
+            const TIO *sk = reinterpret_cast<const TIO *>(buf + D * kCols * 4 + tok_bytes);
+            const TIO *sv = reinterpret_cast<const TIO *>(buf + D * kCols * 4 + 2 * tok_bytes);
+            const float *sg = reinterpret_cast<const float *>(buf + D * kCols * 4 + 3 * tok_bytes);
+            const float *sb = reinterpret_cast<const float *>(buf + D * kCols * 4 + 3 * tok_bytes + sc_bytes);
+            float S[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) S[r] = st[(half * R + r) * kCols + jl];
+            for (int t = 0; t < L; ++t) {
+                const TIO *kt = sk + t * D + half * R, *qt = sq + t * D + half * R;
+                const float alpha = expf(sg[t]), bt = sb[t];
+                // u_j = (k^T S)_j: four partial sums shorten the dependent chain
+                float pu[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int r4 = 0; r4 < R / 4; ++r4) {
+                    const float4 kk = ld4(kt + 4 * r4);
+                    pu[0] = fmaf(kk.x, S[4 * r4], pu[0]);
+                    pu[1] = fmaf(kk.y, S[4 * r4 + 1], pu[1]);
+                    pu[2] = fmaf(kk.z, S[4 * r4 + 2], pu[2]);
+                    pu[3] = fmaf(kk.w, S[4 * r4 + 3], pu[3]);
+                }
+                float u = (pu[0] + pu[1]) + (pu[2] + pu[3]);
+                u += __shfl_xor_sync(0xffffffffu, u, 1);
+                // S <- alpha S + beta k (v - alpha u)^T   ( = alpha (I - beta k k^T) S + beta k v^T )
+                const float wgt = bt * (to_f32(sv[t * D + j]) - alpha * u);
+                float po[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int r4 = 0; r4 < R / 4; ++r4) {
+                    const float4 kk = ld4(kt + 4 * r4), qq = ld4(qt + 4 * r4);
+                    S[4 * r4] = fmaf(alpha, S[4 * r4], kk.x * wgt);
+                    S[4 * r4 + 1] = fmaf(alpha, S[4 * r4 + 1], kk.y * wgt);
+                    S[4 * r4 + 2] = fmaf(alpha, S[4 * r4 + 2], kk.z * wgt);
+                    S[4 * r4 + 3] = fmaf(alpha, S[4 * r4 + 3], kk.w * wgt);
+                    po[0] = fmaf(qq.x, S[4 * r4], po[0]);
+                    po[1] = fmaf(qq.y, S[4 * r4 + 1], po[1]);
+                    po[2] = fmaf(qq.z, S[4 * r4 + 2], po[2]);
+                    po[3] = fmaf(qq.w, S[4 * r4 + 3], po[3]);
+                }
+                float o = (po[0] + po[1]) + (po[2] + po[3]);
+                o += __shfl_xor_sync(0xffffffffu, o, 1);
+                const int64_t row = (int64_t)(n * L + t) * p.H + h;
+                if (half == 0) static_cast<TIO *>(p.out)[row * D + j] = from_f32<TIO>(o * p.scale);
+                if (MODE == kVerify) {
+                    float *c = p.cache + row * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) c[(int64_t)r * D] = S[r];
+                }
+            }
+            if (MODE == kReplay) {
+                const int slot = p.slots[n];
+                float *s1 = p.pool + ((int64_t)slot * p.H + h) * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+                for (int r = 0; r < R; ++r) s1[(int64_t)r * D] = S[r];
+            }
+        }
+        __syncthreads();                      // buffer b is free for the load two items ahead
+        w = wn;
+        b ^= 1;
+        valid = vnext;
     }
-    if (MODE == kReplay) {
-        float *s1 = p.pool + ((int64_t)slot * p.H + h) * D * D + (int64_t)(half * R) * D + j;
-#pragma unroll
-        for (int r = 0; r < R; ++r) s1[(int64_t)r * D] = S[r];
-    }
+    cp_async_wait_all();
 }
 
 // Gather-scatter of accepted states: CTA (x, n*H + h) copies its share of state_cache[n, r-1, h]
@@ -157,12 +224,28 @@ gdn_status check_desc(const gdn_decode_desc *d) {
     return GDN_OK;
 }
 
+int num_sms() {
+    static int n = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    });
+    return n > 0 ? n : 148;
+}
+
 template <typename TIO, int D, int MODE>
-gdn_status launch_steps(const DecodeParams &p, size_t smem, cudaStream_t s) {
+gdn_status launch_steps(const DecodeParams &p, cudaStream_t s) {
     auto fn = gdn_decode_kernel<TIO, D, MODE>;
+    const size_t smem = 2 * (size_t)decode_buf_bytes<TIO, D>(p.L);   // double buffer
     if (smem > 48 * 1024 && cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GDN_ERR_CUDA;
-    fn<<<p.N * p.H * (D / kCols), 2 * kCols, smem, s>>>(p);
+    const int items = p.N * p.H * (D / kCols);
+    const int per_sm = std::max(1, std::min(6, (int)((200 * 1024) / smem)));
+    const int grid = std::min(items, num_sms() * per_sm);
+    fn<<<grid, 2 * kCols, smem, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -182,12 +265,11 @@ gdn_status run_steps(const gdn_decode_desc *d, float *pool, const int32_t *slots
     if (status && cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return GDN_ERR_CUDA;
     DecodeParams p{pool, slots, q, k, v, g, beta, out, cache, status, d->num_seqs, d->num_heads, d->num_tokens,
                    d->pool_slots, 1.0f / std::sqrt((float)d->d_k)};
-    const size_t smem = sizeof(float) * ((size_t)3 * d->num_tokens * d->d_k + 2 * (size_t)d->num_tokens);
     const bool bf = d->dtype == GDN_BF16;
     switch (d->d_k) {
-    case 32: return bf ? launch_steps<__nv_bfloat16, 32, MODE>(p, smem, s) : launch_steps<float, 32, MODE>(p, smem, s);
-    case 64: return bf ? launch_steps<__nv_bfloat16, 64, MODE>(p, smem, s) : launch_steps<float, 64, MODE>(p, smem, s);
-    default: return bf ? launch_steps<__nv_bfloat16, 128, MODE>(p, smem, s) : launch_steps<float, 128, MODE>(p, smem, s);
+    case 32: return bf ? launch_steps<__nv_bfloat16, 32, MODE>(p, s) : launch_steps<float, 32, MODE>(p, s);
+    case 64: return bf ? launch_steps<__nv_bfloat16, 64, MODE>(p, s) : launch_steps<float, 64, MODE>(p, s);
+    default: return bf ? launch_steps<__nv_bfloat16, 128, MODE>(p, s) : launch_steps<float, 128, MODE>(p, s);
     }
 }
 
