@@ -40,8 +40,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = {
     gb.ALGO_SEQUENTIAL: ["gated_deltanet_dual_b200/csrc/gdn_sequential.cu"],
     gb.ALGO_CHUNKED: ["gated_deltanet_dual_b200/csrc/gdn_chunked.cu"],
+    gb.ALGO_ROUTE1: ["gated_deltanet_dual_b200/csrc/gdn_decode.cu"],
 }
-KERNEL_NAMES = {gb.ALGO_SEQUENTIAL: "gdn_sequential_kernel", gb.ALGO_CHUNKED: "gdn_chunked_kernel"}
+KERNEL_NAMES = {gb.ALGO_SEQUENTIAL: "gdn_sequential_kernel", gb.ALGO_CHUNKED: "gdn_chunked_kernel",
+                gb.ALGO_ROUTE1: "gdn_route1_chain_kernel + gdn_decode_kernel (block end)"}
 
 
 # ----------------------------------------------------------------------------- work model
@@ -467,7 +469,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--algo", default="auto", choices=["auto", "sequential", "chunked"])
+    ap.add_argument("--algo", default="auto", choices=["auto", "sequential", "chunked", "route1"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -485,13 +487,15 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     replicas.init(world, backend="nccl", device=dev)
-    algo = {"auto": gb.ALGO_AUTO, "sequential": gb.ALGO_SEQUENTIAL, "chunked": gb.ALGO_CHUNKED}[args.algo]
+    algo = {"auto": gb.ALGO_AUTO, "sequential": gb.ALGO_SEQUENTIAL, "chunked": gb.ALGO_CHUNKED,
+            "route1": gb.ALGO_ROUTE1}[args.algo]
 
     prob = synth.make_problem(wl, seed=replicas.replica_seed(0, rank), device=dev)
     T, TR, V, H, d = prob.T, prob.T_R, prob.num_views, prob.num_heads, prob.d_k
     desc = gb.make_desc(prob.num_docs, H, d, d, V, prob.block_size, gb._dtype_code(prob.q), prob.conv_width, algo)
     used_algo = gb.select_algo(desc)
-    ws = gb.Workspace(gb.workspace_size(desc, prob.doc_offsets), device=dev)
+    ws = gb.Workspace(gb.workspace_size_route1(desc, prob.doc_offsets, prob.prompt_len) if algo == gb.ALGO_ROUTE1
+                      else gb.workspace_size(desc, prob.doc_offsets), device=dev)
     out = torch.empty(T, H, d, dtype=prob.q.dtype, device=dev)
     out_n = torch.empty(V, TR, H, d, dtype=prob.q.dtype, device=dev)
     fs = torch.empty(prob.num_docs, H, d, d, dtype=torch.float32, device=dev)
@@ -597,7 +601,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": wl.name, "docs": prob.num_docs, "tokens_clean": T, "tokens_noisy": V * TR,
                        "heads": H, "d": d, "block_size": prob.block_size, "views": V, "conv_width": prob.conv_width,
-                       "algo": {1: "sequential", 2: "chunked"}.get(used_algo, str(used_algo)),
+                       "algo": {1: "sequential", 2: "chunked", 3: "route1"}.get(used_algo, str(used_algo)),
                        "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush)"},
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks.summary(),

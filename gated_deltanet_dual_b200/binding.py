@@ -19,10 +19,10 @@ LIB_PATH = os.path.join(_PKG, "libgdn_dual.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_ALIGNMENT, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
 GDN_BF16, GDN_FP32 = 0, 1
-ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED = 0, 1, 2
+ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED, ALGO_ROUTE1 = 0, 1, 2, 3
 EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device_status",
             "gdn_status_string", "gdn_dual_version", "gdn_dual_select_algo",
-            "gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit")
+            "gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit", "gdn_dual_workspace_size_route1")
 
 
 class GdnError(RuntimeError):
@@ -60,6 +60,8 @@ def load_library(path: str = LIB_PATH):
                                              ip, ip, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
             lib.gdn_dual_workspace_size.restype = ctypes.c_size_t
             lib.gdn_dual_workspace_size.argtypes = [ctypes.POINTER(Desc), ip]
+            lib.gdn_dual_workspace_size_route1.restype = ctypes.c_size_t
+            lib.gdn_dual_workspace_size_route1.argtypes = [ctypes.POINTER(Desc), ip, ip]
             lib.gdn_dual_read_device_status.restype = ctypes.c_int
             lib.gdn_dual_read_device_status.argtypes = [vp, vp]
             lib.gdn_status_string.restype = ctypes.c_char_p
@@ -105,6 +107,14 @@ def workspace_size(desc: Desc, doc_offsets) -> int:
     offs = _host_i32(doc_offsets)
     return int(load_library().gdn_dual_workspace_size(ctypes.byref(desc),
                                                       offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))))
+
+
+def workspace_size_route1(desc: Desc, doc_offsets, prompt_len) -> int:
+    """Workspace bytes for ALGO_ROUTE1 (header plus the materialised block-boundary states)."""
+    offs, pl = _host_i32(doc_offsets), _host_i32(prompt_len)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    return int(load_library().gdn_dual_workspace_size_route1(ctypes.byref(desc), offs.ctypes.data_as(ip),
+                                                             pl.ctypes.data_as(ip)))
 
 
 def select_algo(desc: Desc) -> int:
@@ -195,7 +205,10 @@ def forward(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, bl
     _check(final_state, "final_state", (N, H, dk, dv), f32, dev)
     desc = make_desc(N, H, dk, dv, V, int(block_size), _dtype_code(q), conv_width, algo)
     if workspace is None:
-        workspace = Workspace(workspace_size(desc, offs), device=dev)
+        nbytes = workspace_size_route1(desc, offs, pl) if algo == ALGO_ROUTE1 else workspace_size(desc, offs)
+        if nbytes == 0:
+            raise ValueError("invalid descriptor or document layout")
+        workspace = Workspace(nbytes, device=dev)
     st = forward_raw(desc, q, k, v, g, beta, qn, kn, vn, gn, betan, offs, pl, conv_w,
                      out, out_noisy, final_state, workspace.tensor, stream=stream)
     if st != GDN_OK:

@@ -25,7 +25,7 @@ bool desc_ok(const gdn_dual_desc *d) {
     if (d->block_size < 1) return false;
     if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return false;
     if (d->conv_width < 0) return false;
-    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_CHUNKED) return false;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_ROUTE1) return false;
     if (d->reserved != 0) return false;
     return true;
 }
@@ -72,7 +72,23 @@ size_t gdn_dual_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_off
     if (doc_offsets_host[0] != 0) return 0;
     for (int n = 0; n < desc->num_docs; ++n)
         if (doc_offsets_host[n + 1] < doc_offsets_host[n]) return 0;
+    if (desc->algo == GDN_ALGO_ROUTE1) return 0;   // needs the prompt lengths: the _route1 variant
     return sizeof(gdn::WorkspaceHeader);
+}
+
+size_t gdn_dual_workspace_size_route1(const gdn_dual_desc *desc, const int32_t *doc_offsets_host,
+                                      const int32_t *prompt_len_host) {
+    if (!desc_ok(desc) || !doc_offsets_host || !prompt_len_host) return 0;
+    if (doc_offsets_host[0] != 0) return 0;
+    int64_t TR = 0;
+    for (int n = 0; n < desc->num_docs; ++n) {
+        const int64_t len = (int64_t)doc_offsets_host[n + 1] - doc_offsets_host[n];
+        if (len < 0 || prompt_len_host[n] < 0 || prompt_len_host[n] > len) return 0;
+        if ((len - prompt_len_host[n]) % desc->block_size != 0) return 0;
+        TR += len - prompt_len_host[n];
+    }
+    const size_t states = (size_t)(TR / desc->block_size) * desc->num_heads * desc->d_k * desc->d_v * sizeof(float);
+    return sizeof(gdn::WorkspaceHeader) + ((states + 255) / 256) * 256;
 }
 
 gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
@@ -106,6 +122,9 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
     const bool noisy = V > 0 && TR > 0;
     if (noisy && (!qn || !kn || !vn || !gn || !betan || !out_noisy)) return GDN_ERR_INVALID_ARG;
     if (!workspace || workspace_bytes < sizeof(gdn::WorkspaceHeader)) return GDN_ERR_INVALID_ARG;
+    const size_t route1_states = (size_t)(TR / B) * H * desc->d_k * desc->d_v * sizeof(float);
+    if (desc->algo == GDN_ALGO_ROUTE1 && workspace_bytes < sizeof(gdn::WorkspaceHeader) + route1_states)
+        return GDN_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, g, beta, qn, kn, vn, gn, betan, conv_w, out, out_noisy, final_state, workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
@@ -113,6 +132,7 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
     const int algo = select_algo(desc);
     if (algo == GDN_ALGO_CHUNKED && !gdn::chunked_supported(desc->dtype, desc->d_k, B, desc->conv_width))
         return GDN_ERR_UNSUPPORTED;
+    if (algo == GDN_ALGO_ROUTE1 && (desc->conv_width != 0 || B > 64)) return GDN_ERR_UNSUPPORTED;
 
     gdn::Params P;
     std::memset(&P, 0, sizeof(P));
@@ -146,8 +166,12 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(gdn::WorkspaceHeader), st) != cudaSuccess) return GDN_ERR_CUDA;
-    cudaError_t err = algo == GDN_ALGO_CHUNKED ? gdn::launch_chunked(P, st)
-                                               : gdn::launch_sequential(P, desc->dtype, st);
+    cudaError_t err;
+    if (algo == GDN_ALGO_CHUNKED) err = gdn::launch_chunked(P, st);
+    else if (algo == GDN_ALGO_ROUTE1)
+        err = gdn::launch_route1(P, desc->dtype,
+                                 reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader)), st);
+    else err = gdn::launch_sequential(P, desc->dtype, st);
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

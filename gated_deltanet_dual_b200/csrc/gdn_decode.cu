@@ -26,7 +26,9 @@ namespace {
 
 using namespace sm100;
 
-enum DecodeMode { kReplay = 0, kVerify = 1 };
+// kReplay / kVerify: the serving kernels.  kBlockEnd: Route I's refinement of one noisy block from
+// its stored boundary state (pool row n % nb), every position reading the block-end state.
+enum DecodeMode { kReplay = 0, kVerify = 1, kBlockEnd = 2 };
 
 struct DecodeParams {
     float *pool;              // [P, H, D, D]
@@ -37,6 +39,7 @@ struct DecodeParams {
     float *cache;             // [N, L, H, D, D] (verify)
     int32_t *status;          // optional
     int N, H, L, P;
+    int nb;                   // kBlockEnd: number of blocks per view (pool row of item n = n % nb)
     float scale;
 };
 
@@ -84,7 +87,7 @@ __global__ void __launch_bounds__(2 * kCols) gdn_decode_kernel(const DecodeParam
     auto issue_load = [&](int w, int b) -> bool {
         const int unit = w / NCB, cb = w % NCB;
         const int n = unit / p.H, h = unit % p.H;
-        const int slot = p.slots[n];
+        const int slot = MODE == kBlockEnd ? n % p.nb : p.slots[n];
         if (slot < 0 || slot >= p.P) {
             if (tid == 0 && cb == 0) flag_bad(p.status);
             return false;
@@ -169,14 +172,34 @@ __global__ void __launch_bounds__(2 * kCols) gdn_decode_kernel(const DecodeParam
                     po[2] = fmaf(qq.z, S[4 * r4 + 2], po[2]);
                     po[3] = fmaf(qq.w, S[4 * r4 + 3], po[3]);
                 }
-                float o = (po[0] + po[1]) + (po[2] + po[3]);
-                o += __shfl_xor_sync(0xffffffffu, o, 1);
                 const int64_t row = (int64_t)(n * L + t) * p.H + h;
-                if (half == 0) static_cast<TIO *>(p.out)[row * D + j] = from_f32<TIO>(o * p.scale);
+                if (MODE != kBlockEnd) {
+                    float o = (po[0] + po[1]) + (po[2] + po[3]);
+                    o += __shfl_xor_sync(0xffffffffu, o, 1);
+                    if (half == 0) static_cast<TIO *>(p.out)[row * D + j] = from_f32<TIO>(o * p.scale);
+                }
                 if (MODE == kVerify) {
                     float *c = p.cache + row * D * D + (int64_t)(half * R) * D + j;
 #pragma unroll
                     for (int r = 0; r < R; ++r) c[(int64_t)r * D] = S[r];
+                }
+            }
+            if (MODE == kBlockEnd) {          // every position of the block reads the block-end state
+                for (int t = 0; t < L; ++t) {
+                    const TIO *qt = sq + t * D + half * R;
+                    float po[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int r4 = 0; r4 < R / 4; ++r4) {
+                        const float4 qq = ld4(qt + 4 * r4);
+                        po[0] = fmaf(qq.x, S[4 * r4], po[0]);
+                        po[1] = fmaf(qq.y, S[4 * r4 + 1], po[1]);
+                        po[2] = fmaf(qq.z, S[4 * r4 + 2], po[2]);
+                        po[3] = fmaf(qq.w, S[4 * r4 + 3], po[3]);
+                    }
+                    float o = (po[0] + po[1]) + (po[2] + po[3]);
+                    o += __shfl_xor_sync(0xffffffffu, o, 1);
+                    const int64_t row = (int64_t)(n * L + t) * p.H + h;
+                    if (half == 0) static_cast<TIO *>(p.out)[row * D + j] = from_f32<TIO>(o * p.scale);
                 }
             }
             if (MODE == kReplay) {
@@ -264,7 +287,7 @@ gdn_status run_steps(const gdn_decode_desc *d, float *pool, const int32_t *slots
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (status && cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return GDN_ERR_CUDA;
     DecodeParams p{pool, slots, q, k, v, g, beta, out, cache, status, d->num_seqs, d->num_heads, d->num_tokens,
-                   d->pool_slots, 1.0f / std::sqrt((float)d->d_k)};
+                   d->pool_slots, 0, 1.0f / std::sqrt((float)d->d_k)};
     const bool bf = d->dtype == GDN_BF16;
     switch (d->d_k) {
     case 32: return bf ? launch_steps<__nv_bfloat16, 32, MODE>(p, s) : launch_steps<float, 32, MODE>(p, s);
@@ -273,7 +296,157 @@ gdn_status run_steps(const gdn_decode_desc *d, float *pool, const int32_t *slots
     }
 }
 
+// ----------------------------------------------------------------------------- Route I
+// Stage 1 of chunk-then-refine (Route I of the notes): the clean chain of every (document, head)
+// token by token, split into items of kCols state columns, writing the clean outputs, the final
+// state and, before every response block, the state S_{e(b-1)} into `states` [T_R / B, H, D, D]
+// (block index = (first response row of the document + position in the response) / B).
+constexpr int kTile = 32;                  // tokens staged per tile
+
+template <typename TIO, int D>
+__host__ __device__ constexpr int chain_buf_bytes() {
+    return 3 * round16(kTile * D * (int)sizeof(TIO)) + 2 * round16(kTile * 4);
+}
+
+template <typename TIO, int D>
+__global__ void __launch_bounds__(2 * kCols) gdn_route1_chain_kernel(const __grid_constant__ Params P, float *states) {
+    constexpr int R = D / 2, NCB = D / kCols;
+    constexpr int tok_bytes = round16(kTile * D * (int)sizeof(TIO)), sc_bytes = round16(kTile * 4);
+    constexpr int buf_bytes = chain_buf_bytes<TIO, D>();
+    constexpr int CPR = D * (int)sizeof(TIO) / 16;
+    extern __shared__ float4 sh4[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(sh4);
+    const int tid = threadIdx.x, jl = tid >> 1, half = tid & 1;
+    const int H = P.H, B = P.B;
+    const int total = P.num_units * NCB;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+        const int unit = w / NCB, cb = w % NCB;
+        const int n = P.unit_doc[unit / H], h = unit % H;
+        const int s0 = P.doc_start[n], len = P.doc_start[n + 1] - s0, prompt = P.doc_prompt[n];
+        const int roff = P.resp_off[n];
+        const int j = cb * kCols + jl;
+        const int ntiles = (len + kTile - 1) / kTile;
+        auto issue = [&](int ti, int b) {
+            uint8_t *buf = smem + b * buf_bytes;
+            const int t0 = ti * kTile, nt = min(kTile, len - t0);
+            const void *src[3] = {P.q, P.k, P.v};
+            for (int x = 0; x < 3; ++x) {
+                const uint8_t *sx = static_cast<const uint8_t *>(src[x]);
+                for (int i = tid; i < nt * CPR; i += 2 * kCols) {
+                    const int t = i / CPR, c = i % CPR;
+                    cp_async16(buf + x * tok_bytes + t * D * (int)sizeof(TIO) + 16 * c,
+                               sx + (((int64_t)(s0 + t0 + t) * H + h) * D) * (int64_t)sizeof(TIO) + 16 * c);
+                }
+            }
+            float *sg = reinterpret_cast<float *>(buf + 3 * tok_bytes), *sb = sg + sc_bytes / 4;
+            for (int t = tid; t < nt; t += 2 * kCols) {
+                const int64_t row = (int64_t)(s0 + t0 + t) * H + h;
+                cp_async4(sg + t, P.g + row, 4);
+                cp_async4(sb + t, P.beta + row, 4);
+            }
+        };
+        float S[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) S[r] = 0.f;
+        if (ntiles > 0) issue(0, 0);
+        cp_async_commit();
+        for (int ti = 0; ti < ntiles; ++ti) {
+            const int b = ti & 1;
+            if (ti + 1 < ntiles) issue(ti + 1, b ^ 1);
+            cp_async_commit();
+            cp_async_wait_group1();
+            __syncthreads();
+            const uint8_t *buf = smem + b * buf_bytes;
+            const TIO *sq = reinterpret_cast<const TIO *>(buf), *sk = reinterpret_cast<const TIO *>(buf + tok_bytes);
+            const TIO *sv = reinterpret_cast<const TIO *>(buf + 2 * tok_bytes);
+            const float *sg = reinterpret_cast<const float *>(buf + 3 * tok_bytes), *sb = sg + sc_bytes / 4;
+            const int t0 = ti * kTile, nt = min(kTile, len - t0);
+            for (int t = 0; t < nt; ++t) {
+                const int pos = t0 + t;
+                if (pos >= prompt && (pos - prompt) % B == 0) {   // state before response block
+                    const int64_t gb = (roff + pos - prompt) / B;
+                    float *dst = states + (gb * H + h) * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) dst[(int64_t)r * D] = S[r];
+                }
+                const TIO *kt = sk + t * D + half * R, *qt = sq + t * D + half * R;
+                const float alpha = expf(sg[t]), bt = sb[t];
+                float pu[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int r4 = 0; r4 < R / 4; ++r4) {
+                    const float4 kk = ld4(kt + 4 * r4);
+                    pu[0] = fmaf(kk.x, S[4 * r4], pu[0]);
+                    pu[1] = fmaf(kk.y, S[4 * r4 + 1], pu[1]);
+                    pu[2] = fmaf(kk.z, S[4 * r4 + 2], pu[2]);
+                    pu[3] = fmaf(kk.w, S[4 * r4 + 3], pu[3]);
+                }
+                float u = (pu[0] + pu[1]) + (pu[2] + pu[3]);
+                u += __shfl_xor_sync(0xffffffffu, u, 1);
+                const float wgt = bt * (to_f32(sv[t * D + j]) - alpha * u);
+                float po[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int r4 = 0; r4 < R / 4; ++r4) {
+                    const float4 kk = ld4(kt + 4 * r4), qq = ld4(qt + 4 * r4);
+                    S[4 * r4] = fmaf(alpha, S[4 * r4], kk.x * wgt);
+                    S[4 * r4 + 1] = fmaf(alpha, S[4 * r4 + 1], kk.y * wgt);
+                    S[4 * r4 + 2] = fmaf(alpha, S[4 * r4 + 2], kk.z * wgt);
+                    S[4 * r4 + 3] = fmaf(alpha, S[4 * r4 + 3], kk.w * wgt);
+                    po[0] = fmaf(qq.x, S[4 * r4], po[0]);
+                    po[1] = fmaf(qq.y, S[4 * r4 + 1], po[1]);
+                    po[2] = fmaf(qq.z, S[4 * r4 + 2], po[2]);
+                    po[3] = fmaf(qq.w, S[4 * r4 + 3], po[3]);
+                }
+                float o = (po[0] + po[1]) + (po[2] + po[3]);
+                o += __shfl_xor_sync(0xffffffffu, o, 1);
+                if (half == 0)
+                    static_cast<TIO *>(P.out)[((int64_t)(s0 + pos) * H + h) * D + j] = from_f32<TIO>(o * P.scale);
+            }
+            __syncthreads();                  // buffer b is free for tile ti + 2
+        }
+        cp_async_wait_all();
+        float *fs = P.final_state + ((int64_t)n * H + h) * D * D + (int64_t)(half * R) * D + j;
+#pragma unroll
+        for (int r = 0; r < R; ++r) fs[(int64_t)r * D] = S[r];
+    }
+}
+
+template <typename TIO, int D>
+cudaError_t route1(const Params &p, float *states, cudaStream_t s) {
+    auto chain = gdn_route1_chain_kernel<TIO, D>;
+    const size_t smem1 = 2 * (size_t)chain_buf_bytes<TIO, D>();
+    cudaError_t e = cudaSuccess;
+    if (smem1 > 48 * 1024) e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    if (e != cudaSuccess) return e;
+    const int items1 = p.num_units * (D / kCols);
+    const int grid1 = std::min(items1, num_sms() * std::max(1, std::min(6, (int)((200 * 1024) / smem1))));
+    if (items1 > 0) chain<<<grid1, 2 * kCols, smem1, s>>>(p, states);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.V == 0 || p.TR == 0) return cudaSuccess;
+    const int nb = (int)(p.TR / p.B);
+    DecodeParams d{states, nullptr, p.qn, p.kn, p.vn, p.gn, p.betan, p.out_noisy, nullptr, nullptr,
+                   p.V * nb, p.H, p.B, nb, nb, p.scale};
+    auto refine = gdn_decode_kernel<TIO, D, kBlockEnd>;
+    const size_t smem2 = 2 * (size_t)decode_buf_bytes<TIO, D>(p.B);
+    if (smem2 > 48 * 1024 && (e = cudaFuncSetAttribute(refine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)) != cudaSuccess)
+        return e;
+    const int items2 = d.N * d.H * (D / kCols);
+    const int grid2 = std::min(items2, num_sms() * std::max(1, std::min(6, (int)((200 * 1024) / smem2))));
+    refine<<<grid2, 2 * kCols, smem2, s>>>(d);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_route1(const Params &p, int dtype, float *states, cudaStream_t stream) {
+    const bool bf = dtype == GDN_BF16;
+    switch (p.dk) {
+    case 32: return bf ? route1<__nv_bfloat16, 32>(p, states, stream) : route1<float, 32>(p, states, stream);
+    case 64: return bf ? route1<__nv_bfloat16, 64>(p, states, stream) : route1<float, 64>(p, states, stream);
+    case 128: return bf ? route1<__nv_bfloat16, 128>(p, states, stream) : route1<float, 128>(p, states, stream);
+    default: return cudaErrorNotSupported;
+    }
+}
+
 }  // namespace gdn
 
 extern "C" gdn_status gdn_decode_replay(const gdn_decode_desc *desc, float *state_pool, const int32_t *slots,

@@ -45,6 +45,8 @@ struct Params {
 // Launchers (one per kernel family).  Return a CUDA error code; the caller maps it.
 cudaError_t launch_sequential(const Params &p, int dtype, cudaStream_t stream);
 cudaError_t launch_chunked(const Params &p, cudaStream_t stream);
+// Route I: clean chain writing block-boundary states into `states`, then block refinement.
+cudaError_t launch_route1(const Params &p, int dtype, float *states, cudaStream_t stream);
 bool chunked_supported(int dtype, int d, int B, int conv_width);
 
 __device__ __forceinline__ float to_f32(float x) { return x; }

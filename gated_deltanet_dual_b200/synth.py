@@ -86,6 +86,8 @@ def get_workload(name: str) -> Workload:
         return WORKLOADS[name]
     if name.startswith("conv_4x8192_h16_d128_B"):
         return WORKLOADS["conv_4x8192_h16_d128_B4"].with_block(int(name.rsplit("B", 1)[1]))
+    if name.startswith("train_8x4096_h16_d128_B"):       # the training shape at other block sizes
+        return WORKLOADS["train_8x4096_h16_d128"].with_block(int(name.rsplit("B", 1)[1]))
     raise KeyError(name)
 
 

@@ -66,7 +66,11 @@ typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 typedef enum {
     GDN_ALGO_AUTO = 0,        /* chunked tensor-core kernel when supported, else sequential */
     GDN_ALGO_SEQUENTIAL = 1,  /* token-sequential CUDA-core kernel, fp32 state (any dtype) */
-    GDN_ALGO_CHUNKED = 2      /* chunked WY/UT tcgen05 kernel (bf16, d_k = d_v = 128) */
+    GDN_ALGO_CHUNKED = 2,     /* chunked WY/UT tcgen05 kernel (bf16, d_k = d_v = 128) */
+    GDN_ALGO_ROUTE1 = 3       /* chunk-then-refine (Route I of the notes, Key design 2), a measured
+                                 comparison: a clean pass writes the state before every response
+                                 block into the workspace, then each (view, block) is refined from
+                                 its stored state; CUDA cores; no ShortConv; never chosen by AUTO */
 } gdn_algo;
 
 /* Problem descriptor.  num_docs N >= 1; num_heads H >= 1; d_k == d_v in {32, 64, 128};
@@ -90,8 +94,16 @@ typedef struct CUstream_st *gdn_stream_t;
 
 /* Bytes of device workspace gdn_dual_forward needs for this problem (>= 256, a multiple of
  * 256).  doc_offsets_host: HOST array [N+1].  Returns 0 if the descriptor or offsets are
- * invalid. */
+ * invalid.  For GDN_ALGO_ROUTE1 it adds the materialised block-boundary states, T_R / B x H x
+ * d_k x d_v fp32 (all documents' responses, T_R from doc_offsets and the prompt lengths); for
+ * that algorithm prompt_len must be known, so use gdn_dual_workspace_size_route1. */
 size_t gdn_dual_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host);
+
+/* Workspace bytes for GDN_ALGO_ROUTE1: 256 + (T_R / B) * H * d_k * d_v * 4, where T_R is the total
+ * response length (doc_offsets_host [N+1] and prompt_len_host [N] are HOST arrays).  Returns 0 if
+ * the descriptor, offsets or prompt lengths are invalid. */
+size_t gdn_dual_workspace_size_route1(const gdn_dual_desc *desc, const int32_t *doc_offsets_host,
+                                      const int32_t *prompt_len_host);
 
 /*
  * Dual-stream GDN forward (Key design 2 and 3 of the FLARE notes; see the file comment).

@@ -22,7 +22,7 @@ no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="placeholder point
 def declared_functions():
     src = "\n".join(open(h).read() for h in HEADERS)
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(gdn_[a-z_]+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(gdn_[a-z0-9_]+)\s*\(",
                                  src, flags=re.M)))
 
 
@@ -237,3 +237,22 @@ def test_decode_host_validation(fn, case, expect):
     elif case == "misaligned_slots":
         over["slots"] = 0x7f0000000002
     assert _decode_call(fn, d, **over) == expect
+
+
+def test_route1_workspace_and_validation():
+    d = b.make_desc(2, 4, 64, 64, 2, 16, b.GDN_BF16, algo=b.ALGO_ROUTE1)
+    offs, pl = [0, 96, 160], [32, 32]                 # responses 64 and 32 tokens: 6 blocks of 16
+    assert b.workspace_size(d, offs) == 0             # needs the prompt lengths
+    assert b.workspace_size_route1(d, offs, pl) == 256 + 6 * 4 * 64 * 64 * 4
+    assert b.workspace_size_route1(d, offs, [30, 32]) == 0          # response not a multiple of B
+    assert b.select_algo(b.make_desc(2, 4, 64, 64, 2, 16, b.GDN_BF16)) != b.ALGO_ROUTE1
+
+
+@no_gpu
+def test_route1_host_validation():
+    d = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32, algo=b.ALGO_ROUTE1)
+    need = b.workspace_size_route1(d, [0, 16, 40], [8, 4])
+    assert _call(d, [0, 16, 40], [8, 4], _ws_bytes=need - 16) == b.GDN_ERR_INVALID_ARG   # states do not fit
+    dc = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32, conv_width=4, algo=b.ALGO_ROUTE1)
+    assert _call(dc, [0, 16, 40], [8, 4], conv_w=_Fake(0x7f0000000000), _ws_bytes=need) == b.GDN_ERR_UNSUPPORTED
+    assert _call(d, [0, 16, 40], [8, 4], _ws_bytes=need) == b.GDN_ERR_CUDA              # valid; no device here
