@@ -204,13 +204,15 @@ def forward(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, bl
     _check(out_noisy, "out_noisy", (V, TR, H, dv), io, dev)
     _check(final_state, "final_state", (N, H, dk, dv), f32, dev)
     desc = make_desc(N, H, dk, dv, V, int(block_size), _dtype_code(q), conv_width, algo)
+    ws_tensor = workspace.tensor if workspace is not None else None
     if workspace is None:
         nbytes = workspace_size_route1(desc, offs, pl) if algo == ALGO_ROUTE1 else workspace_size(desc, offs)
-        if nbytes == 0:
-            raise ValueError("invalid descriptor or document layout")
-        workspace = Workspace(nbytes, device=dev)
+        # size 0: the descriptor or the layout is invalid; the library's own validation below
+        # then returns the status (nothing launches)
+        if nbytes:
+            ws_tensor = Workspace(nbytes, device=dev).tensor
     st = forward_raw(desc, q, k, v, g, beta, qn, kn, vn, gn, betan, offs, pl, conv_w,
-                     out, out_noisy, final_state, workspace.tensor, stream=stream)
+                     out, out_noisy, final_state, ws_tensor, stream=stream)
     if st != GDN_OK:
         raise GdnError(st, f"gdn_dual_forward failed: {status_string(st)}")
     return out, out_noisy, final_state

@@ -75,6 +75,9 @@ __device__ __forceinline__ void bar_all() { asm volatile("bar.sync 1, %0;" ::"n"
 __device__ __forceinline__ void bar_math() { bar_all(); }
 // Warps 1..7 only: work overlapped with an MMA batch that thread 0 (warp 0) is issuing.
 __device__ __forceinline__ void bar_side() { asm volatile("bar.sync 3, %0;" ::"n"(kThreads - 32) : "memory"); }
+// Named barrier 4: warps 1..7 arrive (no wait), warp 0 waits for them.
+__device__ __forceinline__ void bar_arrive_khat() { asm volatile("bar.arrive 4, %0;" ::"n"(kThreads) : "memory"); }
+__device__ __forceinline__ void bar_sync_khat() { asm volatile("bar.sync 4, %0;" ::"n"(kThreads) : "memory"); }
 
 __device__ __forceinline__ uint4 pack8(const float *f) {
     uint4 r;
@@ -131,10 +134,18 @@ __device__ __forceinline__ Unit make_unit(const Params &P, int u) {
 
 // Block coefficients of one noisy row: y = Ptil_j Ttil (back substitution against the block's
 // own I + Atil), then ycoef = y beta~ Gammatil (for Z) and wcoef = y beta~ (for WV).
+// Shared-memory staging of the noisy block coefficients (B >= 16): per TMEM lane quadrant, 32
+// rows of B fp32 values (one 16-byte pad between the two blocks of a quadrant when B = 16, so
+// the two blocks' broadcast reads fall in different bank groups).
+template <int B>
+constexpr int kAtQuadBytes = 32 * B * 4 + (B < 32 ? 16 : 0);
+template <int B>
+__device__ __forceinline__ constexpr int at_swz(int r) { return B >= 32 ? (r & 7) : ((r >> 1) & 3); }
+
 template <int B>
 __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float (&wk)[32], int lane, int j,
                                              const float *ngam, const float *nbeta, const float *nE,
-                                             const float *nF, bool nfact,
+                                             const float *nF, bool nfact, float *s_at,
                                              float (&ycoef)[B], float (&wcoef)[B], float &gend) {
     const int bs = (j / B) * B;
     const int jl = j - bs;
@@ -174,12 +185,39 @@ __device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float 
     }
     // Right-looking back substitution: once y_mm is final it is taken out of every earlier
     // position at once, so the dependent chain is B steps of one FMA each.
-    const int base = lane - jl;
+    if constexpr (B >= 16) {
+        // Row mm of the block's Atil is needed by every lane of the block: the rows go through
+        // shared memory once and are read back as broadcast 16-byte loads (about B^2/8 loads
+        // instead of B^2/2 shuffles).  16-byte column c4 of row r sits at c4 ^ at_swz(r), so the
+        // row stores of 8 consecutive lanes hit 8 distinct bank groups; r & 7 of a block row is
+        // mm & 7, known at compile time.
+        float *myrow = s_at + lane * B + (B < 32 ? (lane / B) * 4 : 0);
 #pragma unroll
-    for (int mm = B - 1; mm >= 0; --mm) {
-        y[mm] = pt[mm];
+        for (int c4 = 0; c4 < B / 4; ++c4)
+            *reinterpret_cast<float4 *>(myrow + 4 * (c4 ^ at_swz<B>(jl))) =
+                make_float4(arow[4 * c4], arow[4 * c4 + 1], arow[4 * c4 + 2], arow[4 * c4 + 3]);
+        __syncwarp();
+        const float *blk = myrow - jl * B;
 #pragma unroll
-        for (int l = 0; l < mm; ++l) pt[l] = fmaf(-y[mm], __shfl_sync(0xffffffffu, arow[l], base + mm), pt[l]);
+        for (int mm = B - 1; mm >= 0; --mm) {
+            y[mm] = pt[mm];
+#pragma unroll
+            for (int c4 = 0; c4 < (mm + 3) / 4; ++c4) {
+                const float4 a = *reinterpret_cast<const float4 *>(blk + mm * B + 4 * (c4 ^ at_swz<B>(mm)));
+                const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (4 * c4 + e < mm) pt[4 * c4 + e] = fmaf(-y[mm], av[e], pt[4 * c4 + e]);
+            }
+        }
+    } else {
+        const int base = lane - jl;
+#pragma unroll
+        for (int mm = B - 1; mm >= 0; --mm) {
+            y[mm] = pt[mm];
+#pragma unroll
+            for (int l = 0; l < mm; ++l) pt[l] = fmaf(-y[mm], __shfl_sync(0xffffffffu, arow[l], base + mm), pt[l]);
+        }
     }
 #pragma unroll
     for (int l = 0; l < B; ++l) {
@@ -218,7 +256,7 @@ __device__ __forceinline__ void store_block_row(uint32_t taddr, int ch, int v, i
 template <int B>
 __device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int lane, int rho,
                                               const float *s_ngam, const float *s_nbeta, const float *s_nE,
-                                              const float *s_nF, bool nfact) {
+                                              const float *s_nF, bool nfact, float *s_at) {
     float wq[32], wk[32];
     tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 32 * q), wq);
     tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 32 * q), wk);
@@ -226,7 +264,7 @@ __device__ __forceinline__ float noisy_phase1(uint32_t tb, int q, int ch, int la
     const int v = rho >> 6, j = rho & 63;
     float ycoef[B], wcoef[B], gend;
     noisy_coeffs<B>(wq, wk, lane, j, s_ngam + 64 * v, s_nbeta + 64 * v, s_nE + 64 * v, s_nF + 64 * v, nfact,
-                    ycoef, wcoef, gend);
+                    s_at, ycoef, wcoef, gend);
     bar_math();   // every warp has finished reading TM_TK before it is overwritten
     const int bs = (j / B) * B;
     store_block_row<B>(tmem_addr(tb, q * 32, TM_TK + 32 * ch), ch, v, bs, wcoef, 1.f);
@@ -799,6 +837,9 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     // for a clean-only chunk costing kCleanCost of a full one (lower for long blocks, whose noisy
     // work weighs more).
     constexpr float kCleanCost = B >= 32 ? 0.42f : (B >= 16 ? 0.55f : 0.65f);   // measured balance
+    // B >= 16: the noisy block coefficients are staged in the Khat buffer, so Khat is built late.
+    constexpr bool kKhatLate = B >= 16;
+    static_assert(4 * kAtQuadBytes<B> <= 16384, "block coefficients must fit the Khat buffer");
     // Work items are (unit, part), longest documents first; each CTA starts with item blockIdx.x and
     // then takes the next untaken item from a counter in the workspace (greedy list scheduling:
     // uneven documents no longer pile up on the CTAs that a fixed stride would give them).
@@ -917,17 +958,22 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 mma_commit(&bar_mma);
             }
             __syncwarp();
-            // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout)
-            const float gC = s_gam[CH - 1];
-            for (int it = tid - 32; it >= 0 && it < 64 * 16; it += kMathThreads - 32) {   // warps 1..7
-                const int t = it >> 4, c16 = it & 15, hf = c16 >> 3, c8 = c16 & 7;
-                float f[8];
-                unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QK + hf * 16384 + sw128_off(64 + t, c8)), f);
-                const float sc = fact ? s_E[CH - 1] * s_F[t] : exp2f(fminf(gC - s_gam[t], 0.f));
+            // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout), on
+            // warps 1..7.  With B >= 16 its buffer first stages the noisy block coefficients and
+            // Khat is built in the S2 phase instead, before the next chunk's tiles replace K.
+            auto build_khat = [&] {
+                const float gC = s_gam[CH - 1];
+                for (int it = tid - 32; it >= 0 && it < 64 * 16; it += kMathThreads - 32) {
+                    const int t = it >> 4, c16 = it & 15, hf = c16 >> 3, c8 = c16 & 7;
+                    float f[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QK + hf * 16384 + sw128_off(64 + t, c8)), f);
+                    const float sc = fact ? s_E[CH - 1] * s_F[t] : exp2f(fminf(gC - s_gam[t], 0.f));
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] *= sc;
-                *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
-            }
+                    for (int e = 0; e < 8; ++e) f[e] *= sc;
+                    *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
+                }
+            };
+            if constexpr (!kKhatLate) build_khat();
             if (!conv) {                                  // V and [k~0;k~1]
                 if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
                 ++ph_b;
@@ -985,7 +1031,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             float gend = 0.f;
             if (noisy) {
                 const bool nfact = B >= 16 && s_okn[cb][0] && s_okn[cb][1] && s_okn[cb][2] && s_okn[cb][3];
-                gend = noisy_phase1<B>(tb, q, ch, lane, rho, s_ngam, s_nbeta, s_nE, s_nF, nfact);
+                gend = noisy_phase1<B>(tb, q, ch, lane, rho, s_ngam, s_nbeta, s_nE, s_nF, nfact,
+                                      reinterpret_cast<float *>(sm + OFF_KH + q * kAtQuadBytes<B>));
             }
             tmem_wait_st();
             tc_fence_before();
@@ -1141,12 +1188,27 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 }
                 mma_commit(&bar_mma);
                 // prefetch group A of the next chunk once [Q;K] and Z are consumed
-                if (!last) {
+                if (!kKhatLate && !last) {
                     if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(40);
                     else issue_a(U, m + 1, chunk_noisy(ci + 1));
                 }
             }
             __syncwarp();
+            if constexpr (kKhatLate) {
+                // Khat reads K from the [Q;K] tile: warps 1..7 build it, then signal warp 0,
+                // whose lane 0 lets the next chunk's group A overwrite the tile.
+                if (warp > 0) {
+                    build_khat();
+                    bar_arrive_khat();
+                } else {
+                    bar_sync_khat();
+                    if (tid == 0 && !last) {
+                        if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(40);
+                        else issue_a(U, m + 1, chunk_noisy(ci + 1));
+                    }
+                    __syncwarp();
+                }
+            }
             if (!last && warp > 0) prep_scalars(U, m + 1, cb ^ 1);   // next chunk's scalars meanwhile
             wait_mma(40);
             if (rho < 64) {
