@@ -297,6 +297,74 @@ __device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int 
     }
 }
 
+// Exact-decay variants of two epilogues, for a chunk whose cumulative decays leave the range in
+// which e^{gamma_t - gamma_i} factorises as E_t F_i.  Such chunks are rare; out of line, they keep
+// the common path's instruction footprint small.
+struct Rows4 {
+    uint4 v[4];
+};
+
+// P rows (rho < 64: returned as bf16) or A rows (rho >= 64: written to the fp32 solve scratch)
+// of [Q;K]K^T (TMEM columns at taddr), with the decays exponentiated one by one.
+__device__ __noinline__ Rows4 pa_rows_exact(uint32_t taddr, int rho, int ch, const float *s_gam,
+                                           const float *s_beta, float *scratch) {
+    float tk[32];
+    tmem_ld32(taddr, tk);
+    tmem_wait_ld();
+    Rows4 r;
+    if (rho < 64) {
+        const int t = rho;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const int i = 32 * ch + c;
+            tk[c] = (i <= t) ? tk[c] * exp2f(fminf(s_gam[t] - s_gam[i], 0.f)) : 0.f;
+        }
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) r.v[c4] = pack8(tk + 8 * c4);
+    } else {
+        const int t = rho - 64;
+        const float bt = s_beta[t];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const int i = 32 * ch + c;
+            tk[c] = (i < t) ? bt * exp2f(fminf(s_gam[t] - s_gam[i], 0.f)) * tk[c] : 0.f;
+        }
+#pragma unroll
+        for (int g4 = 0; g4 < 8; ++g4)
+            *srow4(scratch, t, 32 * ch + 4 * g4) = make_float4(tk[4 * g4], tk[4 * g4 + 1], tk[4 * g4 + 2], tk[4 * g4 + 3]);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) r.v[c4] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    return r;
+}
+
+// M'_Z rows of a noisy row (Z K^T in TMEM at taddr; boundary row e of its block, -1 for S0) with
+// exact decays, then Z <- Gamma_e Z in place for the state product.
+__device__ __noinline__ void mz_rows_exact(uint8_t *sm, uint32_t taddr, int rho, int ch, int e,
+                                          const float *s_gam, const float *s_E) {
+    float zk[32];
+    tmem_ld32(taddr, zk);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const int i = 32 * ch + c;
+        zk[c] = (i <= e) ? zk[c] * exp2f(fminf(s_gam[e < 0 ? 0 : e] - s_gam[i], 0.f)) : 0.f;
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+        *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
+    const float Ge = e >= 0 ? s_E[e] : 1.f;    // Gamma_e (1 for e = -1)
+    uint8_t *zrow = sm + OFF_NQ + ch * 16384;
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4 *>(zrow + sw128_off(rho, c8)), f);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) f[x] *= Ge;
+        *reinterpret_cast<uint4 *>(zrow + sw128_off(rho, c8)) = pack8(f);
+    }
+}
+
 // 32 x 32 fp32 staging block (the 32-merge's result): 128-byte rows, 16-byte chunks swizzled by
 // the row like the solve scratch.
 __device__ __forceinline__ int widx(int r, int c) { return r * 32 + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3); }
@@ -941,11 +1009,6 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             bar_all();
             if (s_abort) break;
             const bool fact = s_okw[cb][0] && s_okw[cb][1];
-            // e^{gamma_t - gamma_i} (i <= t): a product of per-row factors when safe
-            auto decay = [&](auto F, int t, int i) -> float {
-                if constexpr (decltype(F)::value) return s_E[t] * s_F[i];
-                else return exp2f(fminf(s_gam[t] - s_gam[i], 0.f));
-            };
 
             // ================= PK1: [Q;K]K^T now, the noisy products once group B is in ========
             if (tid == 0) {
@@ -994,37 +1057,36 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // clean: P rows (lanes 0-63, bf16 packed in registers until the solve is done) and
             // A rows (lanes 64-127) into the fp32 scratch
             uint4 ppk[4];
-            {
+            if (fact) {
                 float tk[32];
                 tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), tk);
                 tmem_wait_ld();
                 if (rho < 64) {
                     const int t = rho;
-                    auto body = [&](auto F) {
+                    const float Et = s_E[t];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const int i = 32 * ch + c;
-                            tk[c] = (i <= t) ? tk[c] * decay(F, t, i) : 0.f;
-                        }
-                    };
-                    if (fact) body(std::true_type{}); else body(std::false_type{});
+                    for (int c = 0; c < 32; ++c) {
+                        const int i = 32 * ch + c;
+                        tk[c] = (i <= t) ? tk[c] * (Et * s_F[i]) : 0.f;
+                    }
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) ppk[c4] = pack8(tk + 8 * c4);
                 } else {
                     const int t = rho - 64;
-                    const float bt = s_beta[t];
-                    auto body = [&](auto F) {
+                    const float bEt = s_beta[t] * s_E[t];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) {
-                            const int i = 32 * ch + c;
-                            tk[c] = (i < t) ? bt * decay(F, t, i) * tk[c] : 0.f;
-                        }
-                    };
-                    if (fact) body(std::true_type{}); else body(std::false_type{});
+                    for (int c = 0; c < 32; ++c) {
+                        const int i = 32 * ch + c;
+                        tk[c] = (i < t) ? (bEt * s_F[i]) * tk[c] : 0.f;
+                    }
 #pragma unroll
                     for (int g4 = 0; g4 < 8; ++g4)
                         *srow4(scratch, t, 32 * ch + 4 * g4) = make_float4(tk[4 * g4], tk[4 * g4 + 1], tk[4 * g4 + 2], tk[4 * g4 + 3]);
                 }
+            } else {
+                const Rows4 r = pa_rows_exact(tmem_addr(tb, q * 32, TM_TK + 32 * ch), rho, ch, s_gam, s_beta, scratch);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) ppk[c4] = r.v[c4];
             }
             if (noisy) wait_mma2(11);                   // noisy block products of PK1
             // noisy: block coefficients, then W~ and -Y~ rows into TMEM as A operands
@@ -1133,39 +1195,22 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(pt + 8 * c4);
             }
             if (noisy) {
-                float zk[32];
-                tmem_ld32(tmem_addr(tb, q * 32, TM_ZK + 32 * ch), zk);
-                tmem_wait_ld();
-                const int jj = rho & 63;
-                const int e = (jj / B) * B - 1;          // chunk-local boundary row (-1: S0)
+                const int e = ((rho & 63) / B) * B - 1;   // chunk-local boundary row (-1: S0)
                 if (fact) {
+                    float zk[32];
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_ZK + 32 * ch), zk);
+                    tmem_wait_ld();
                     // the rows already hold Gamma_e Z: M'_Z = (Gamma_e Z K^T) e^{-gamma_i} [i <= e]
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int i = 32 * ch + c;
                         zk[c] = (i <= e) ? zk[c] * s_F[i] : 0.f;
                     }
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
+                        *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
                 } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int i = 32 * ch + c;
-                        zk[c] = (i <= e) ? zk[c] * exp2f(fminf(s_gam[e < 0 ? 0 : e] - s_gam[i], 0.f)) : 0.f;
-                    }
-                }
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
-                    *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
-                if (!fact) {                      // Z <- Gamma_e Z for the state product
-                    const float Ge = e >= 0 ? s_E[e] : 1.f;    // Gamma_e (1 for e = -1)
-                    uint8_t *zrow = sm + OFF_NQ + ch * 16384;
-#pragma unroll
-                    for (int c8 = 0; c8 < 8; ++c8) {
-                        float f[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(zrow + sw128_off(rho, c8)), f);
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) f[x] *= Ge;
-                        *reinterpret_cast<uint4 *>(zrow + sw128_off(rho, c8)) = pack8(f);
-                    }
+                    mz_rows_exact(sm, tmem_addr(tb, q * 32, TM_ZK + 32 * ch), rho, ch, e, s_gam, s_E);
                 }
             }
             fence_async_smem();

@@ -106,6 +106,15 @@ def test_strong_gates_and_large_beta():
         check(prob, "bf16", algo)
 
 
+@pytest.mark.parametrize("B", [4, 16, 32])
+def test_extreme_gates_take_the_exact_decay_paths(B):
+    """g ~ U(-8, 0): a chunk's cumulative decay leaves the range in which e^{gamma_t - gamma_i}
+    factorises as E_t F_i (|gamma| >= 100 in log2 units), so the chunked kernel exponentiates every
+    difference (P and A rows, M'_Z and, for B >= 16, the noisy block coefficients)."""
+    prob = small([640, 384], [128, 64], H=2, d=128, B=B, dtype="bf16", seed=41 + B, g_lo=-8.0)
+    check(prob, "bf16", b.ALGO_CHUNKED)
+
+
 def test_chunked_matches_sequential_kernel():
     """The two CUDA kernels agree with each other on a multi-unit problem (both fp32 state)."""
     prob = small([1000, 1536, 520], [232, 512, 8], H=4, d=128, B=4, dtype="bf16", seed=31)
