@@ -634,14 +634,16 @@ struct ConvSeg {
 __device__ __forceinline__ uint32_t conv_weights(uint32_t s, int X, int cc) {
     return s + OFF_CW + (X * 128 + cc) * 16;
 }
-// Noisy item (both views): tensor X, rows r0..r0+LEN-1.  BAR: barrier between loads and stores.
-template <int B, int LEN, bool BAR>
-__device__ __forceinline__ void conv_noisy_item(uint32_t s, uint4 (*halo)[3][16], int X, int cc, int r0, int zr) {
+// Noisy item (both views): tensor X, rows r0..r0+LEN-1.  bar: barrier between loads and stores
+// (uniform over the CTA).  Out of line: both noisy rounds share one copy of the code.
+template <int B, int LEN>
+__device__ __noinline__ void conv_noisy_item(uint32_t s, uint4 (*halo)[3][16], int X, int cc, int r0, int zr,
+                                             bool bar) {
     const int hf = cc >> 3, c8 = cc & 7;
     const uint32_t own = s + noisy_half(X, 0, hf);
     ConvSeg<B, true, LEN> sg;
     sg.load(own, s + clean_half(X, hf), halo[X], cc, r0, c8, zr, (r0 % B) == 0);
-    if (BAR) bar_math();
+    if (bar) bar_math();
     sg.store(own, conv_weights(s, X, cc), r0, c8);
 }
 // Clean item: tensor X, rows r0..r0+LEN-1; the item ending at row 63 carries rows 61..63 (raw)
@@ -674,8 +676,8 @@ __device__ __noinline__ void conv_chunk(uint8_t *sm, uint4 (*halo)[3][16], bool 
     const uint32_t s = smem_u32(sm);
     const int cc = tid & 15;
     if (noisy) {
-        conv_noisy_item<B, 8, (B > 8)>(s, halo, tid >> 7, cc, 8 * ((tid >> 4) & 7), zr);
-        if (tid < 128) conv_noisy_item<B, 8, true>(s, halo, 2, cc, 8 * ((tid >> 4) & 7), zr);
+        conv_noisy_item<B, 8>(s, halo, tid >> 7, cc, 8 * ((tid >> 4) & 7), zr, B > 8);
+        if (tid < 128) conv_noisy_item<B, 8>(s, halo, 2, cc, 8 * ((tid >> 4) & 7), zr, true);
         else conv_clean_item<B, 16>(s, halo, (tid >> 6) & 1, cc, 16 * ((tid >> 4) & 3), zr);
     } else {
         conv_clean_item<B, 8>(s, halo, tid >> 7, cc, 8 * ((tid >> 4) & 7), zr);
