@@ -461,6 +461,155 @@ def run_decode(args, name, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- softmax attention
+ATTN_METRIC = "dual-stream softmax attention fwd tokens/s on 1 B200 and % of tensor roofline"
+
+
+def attn_pairs(offs, pl, B, V):
+    """Visible (query, key) pairs per head under the document-blocked mask."""
+    offs = np.asarray(offs, dtype=np.int64)
+    pairs = 0
+    for n in range(len(pl)):
+        L, P = int(offs[n + 1] - offs[n]), int(pl[n])
+        pairs += L * (L + 1) // 2
+        nb = (L - P) // B
+        pairs += V * B * (nb * (P + B) + B * nb * (nb - 1) // 2)   # sum over blocks of P + b0 + B keys
+    return pairs
+
+
+def time_attn_oracle(name, min_seconds=2.0, seed=0):
+    """The fp64 oracle on a bounded sample: whole documents of one head (host cores, numpy)."""
+    from oracle import attention as oa  # test infrastructure: the CPU baseline / reference arm only
+    pr = synth.make_attn_problem(name, seed=seed, device="cpu")
+    offs, pl, B = pr.doc_offsets.astype(np.int64), pr.prompt_len, pr.block_size
+    V = pr.qn.shape[0]
+    Hkv = pr.k.shape[1]
+    roffs = np.concatenate([[0], np.cumsum(np.diff(offs) - pl)])
+    toks, n, t0 = 0, 0, time.perf_counter()
+    while True:
+        d_ = n % len(pl)
+        s, e, r0, r1 = int(offs[d_]), int(offs[d_ + 1]), int(roffs[d_]), int(roffs[d_ + 1])
+        o1 = np.array([0, e - s], dtype=np.int32)
+        oa.dual_attention(pr.q[s:e, :1], pr.k[s:e, :1], pr.v[s:e, :1], pr.qn[:, r0:r1, :1], pr.kn[:, r0:r1, :1],
+                          pr.vn[:, r0:r1, :1], o1, pl[d_:d_ + 1], B)
+        toks += (e - s) + V * (r1 - r0)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    H = pr.q.shape[1]
+    return {"value": toks / el / H, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"{n} whole documents of one head (of {H}; {Hkv} key/value heads) through the fp64 "
+                      f"numpy oracle; tokens/s scaled to all heads", "seconds": el}
+
+
+def run_attention(args, name, rank, world, local):
+    cfg = synth.ATTN_WORKLOADS[name]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = time_attn_oracle(name)
+        pr = synth.make_attn_problem(name, seed=0, device="cpu")
+        toks = pr.q.shape[0] + pr.qn.shape[0] * pr.qn.shape[1]
+        line = {"metric": ATTN_METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": toks / cb["value"] * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": name, "parallelism": "replicas", "l2": "not applicable (host)"},
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    replicas.init(world, backend="nccl", device=dev)
+    pr = synth.make_attn_problem(name, seed=replicas.replica_seed(0, rank), device=dev)
+    T, H, d = pr.q.shape
+    V, TR = pr.qn.shape[0], pr.qn.shape[1]
+    desc = gb.make_attn_desc(len(pr.prompt_len), H, pr.k.shape[1], d, V, pr.block_size, gb.GDN_BF16)
+    ws = gb.Workspace(gb.attn_workspace_size(desc, pr.doc_offsets, pr.prompt_len), device=dev).tensor
+    out = torch.empty_like(pr.q)
+    out_n = torch.empty_like(pr.qn)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gb.attention_forward(pr.q, pr.k, pr.v, pr.qn, pr.kn, pr.vn, pr.doc_offsets, pr.prompt_len, pr.block_size,
+                             out=out, out_noisy=out_n, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        replicas.barrier(world)
+        torch.cuda.synchronize()
+        clocks.mark_start()
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        clocks.poll_until(evs[-1][1])
+        torch.cuda.synchronize()
+        clocks.mark_stop()
+        replicas.barrier(world)
+    ms = replicas.max_over_ranks(float(np.mean([a.elapsed_time(z) for a, z in evs])), world, device=dev)
+    pairs = attn_pairs(pr.doc_offsets, pr.prompt_len, pr.block_size, V) * H
+    flops = 4 * d * pairs
+    peaks = measured_peaks()
+    achieved = flops / (ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None, "peak_source": peaks["source"] + " (burst)",
+                "kernel": "gdn_attention_kernel", "algorithmic_flops": flops, "visible_pairs": pairs}
+    toks = (T + V * TR) * world
+    value = toks / (ms / 1e3)
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k", "v", "qn", "kn", "vn"]
+        host = {n: getattr(pr, n).cpu().pin_memory() for n in names}
+        dbuf = {n: torch.empty_like(getattr(pr, n)) for n in names}
+        h_o = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h_on = torch.empty(out_n.shape, dtype=out_n.dtype, pin_memory=True)
+
+        def e2e_step():
+            for n in names:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            gb.attention_forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["qn"], dbuf["kn"], dbuf["vn"], pr.doc_offsets,
+                                 pr.prompt_len, pr.block_size, out=out, out_noisy=out_n, workspace=ws)
+            h_o.copy_(out, non_blocking=True)
+            h_on.copy_(out_n, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ns = max(3, args.steps)
+        a.record(stream)
+        for _ in range(ns):
+            e2e_step()
+        z.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = replicas.max_over_ranks(a.elapsed_time(z) / ns, world, device=dev)
+        e2e = {"value": toks / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host.values())),
+               "d2h_bytes_per_step": int(h_o.numel() * 2 + h_on.numel() * 2), "ms_per_step": e2e_ms, "steps": ns}
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = time_attn_oracle(name)
+        cpu_baseline = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    replicas.shutdown(world)
+    if rank != 0:
+        return
+    line = {"metric": ATTN_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": name, "layout": cfg["layout"], "heads": H, "kv_heads": int(pr.k.shape[1]), "d": d,
+                       "block": pr.block_size, "views": V, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 are not guaranteed (K/V reuse through L2 is part of the kernel)"},
+            "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -477,6 +626,9 @@ def main():
     rank, world, local = replicas.env_rank()
     if args.workload in synth.DECODE_WORKLOADS:
         run_decode(args, args.workload, rank, world, local)
+        return
+    if args.workload in synth.ATTN_WORKLOADS:
+        run_attention(args, args.workload, rank, world, local)
         return
     wl = synth.get_workload(args.workload)
 

@@ -22,7 +22,8 @@ GDN_BF16, GDN_FP32 = 0, 1
 ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED, ALGO_ROUTE1 = 0, 1, 2, 3
 EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device_status",
             "gdn_status_string", "gdn_dual_version", "gdn_dual_select_algo",
-            "gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit", "gdn_dual_workspace_size_route1")
+            "gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit", "gdn_dual_workspace_size_route1",
+            "gdn_attn_forward", "gdn_attn_workspace_size")
 
 
 class GdnError(RuntimeError):
@@ -40,6 +41,12 @@ class DecodeDesc(ctypes.Structure):
     """gdn_decode_desc of include/gdn_decode.h."""
     _fields_ = [(n, ctypes.c_int32) for n in ("num_seqs", "num_heads", "d_k", "d_v", "num_tokens",
                                                "pool_slots", "dtype", "reserved")]
+
+
+class AttnDesc(ctypes.Structure):
+    """gdn_attn_desc of include/gdn_attention.h."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("num_docs", "num_heads", "num_kv_heads", "head_dim", "num_views",
+                                               "block_size", "dtype", "reserved")]
 
 
 _lock = threading.Lock()
@@ -75,6 +82,11 @@ def load_library(path: str = LIB_PATH):
             lib.gdn_decode_replay.argtypes = [dd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.gdn_decode_verify.argtypes = [dd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.gdn_decode_commit.argtypes = [dd, vp, vp, vp, vp, vp, vp]
+            ad = ctypes.POINTER(AttnDesc)
+            lib.gdn_attn_workspace_size.restype = ctypes.c_size_t
+            lib.gdn_attn_workspace_size.argtypes = [ad, ip, ip]
+            lib.gdn_attn_forward.restype = ctypes.c_int
+            lib.gdn_attn_forward.argtypes = [ad, vp, vp, vp, vp, vp, vp, ip, ip, vp, vp, vp, ctypes.c_size_t, vp]
             _lib = lib
     return _lib
 
@@ -322,3 +334,66 @@ def decode_commit(state_pool, slots, state_cache, accepted, *, device_status=Non
     if st != GDN_OK:
         raise GdnError(st, f"gdn_decode_commit failed: {status_string(st)}")
     return state_pool
+
+
+# ----------------------------------------------------------------------------- softmax attention
+def make_attn_desc(num_docs, num_heads, num_kv_heads, head_dim, num_views, block_size, dtype_code) -> AttnDesc:
+    return AttnDesc(num_docs, num_heads, num_kv_heads, head_dim, num_views, block_size, dtype_code, 0)
+
+
+def attn_workspace_size(desc: AttnDesc, doc_offsets, prompt_len) -> int:
+    offs = np.ascontiguousarray(doc_offsets, dtype=np.int32)
+    pl = np.ascontiguousarray(prompt_len, dtype=np.int32)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    return int(load_library().gdn_attn_workspace_size(ctypes.byref(desc), offs.ctypes.data_as(ip),
+                                                      pl.ctypes.data_as(ip)))
+
+
+def attention_forward(q, k, v, qn, kn, vn, doc_offsets, prompt_len, block_size, *, out=None, out_noisy=None,
+                      workspace=None, stream=None):
+    """Dual-stream softmax attention with the document-blocked causal / block-bidirectional mask
+    (gdn_attn_forward).  q [T, H, d], k and v [T, H_kv, d]; qn [V, T_R, H, d], kn and vn
+    [V, T_R, H_kv, d]; doc_offsets [N+1] and prompt_len [N] on the host.  Returns (out, out_noisy)."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    T, H, d = q.shape
+    Hkv = k.shape[1]
+    V, TR = qn.shape[0], qn.shape[1]
+    offs = np.ascontiguousarray(doc_offsets, dtype=np.int32)
+    pl = np.ascontiguousarray(prompt_len, dtype=np.int32)
+    N = len(pl)
+    if offs.ndim != 1 or offs.shape[0] != N + 1:
+        raise ValueError("doc_offsets must be [N+1] and prompt_len [N]")
+    if N >= 1 and int(offs[-1]) != T:
+        raise ValueError(f"doc_offsets[-1] = {int(offs[-1])} but q has {T} tokens")
+    if N >= 1 and int((np.diff(offs.astype(np.int64)) - pl).sum()) != TR:
+        raise ValueError(f"noisy tensors have {TR} rows but the documents have "
+                         f"{int((np.diff(offs.astype(np.int64)) - pl).sum())} response tokens")
+    io = q.dtype
+    for t, name, shape in ((q, "q", (T, H, d)), (k, "k", (T, Hkv, d)), (v, "v", (T, Hkv, d)),
+                           (qn, "qn", (V, TR, H, d)), (kn, "kn", (V, TR, Hkv, d)), (vn, "vn", (V, TR, Hkv, d))):
+        _check(t, name, shape, io, dev)
+    if out is None:
+        out = torch.empty(T, H, d, dtype=io, device=dev)
+    if out_noisy is None:
+        out_noisy = torch.empty(V, TR, H, d, dtype=io, device=dev)
+    _check(out, "out", (T, H, d), io, dev)
+    _check(out_noisy, "out_noisy", (V, TR, H, d), io, dev)
+    desc = make_attn_desc(N, H, Hkv, d, V, int(block_size), _dtype_code(q))
+    ws = workspace
+    if ws is None:
+        nbytes = attn_workspace_size(desc, offs, pl)
+        if nbytes:
+            ws = Workspace(nbytes, device=dev).tensor
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    ip = ctypes.POINTER(ctypes.c_int32)
+    noisy = V > 0 and TR > 0
+    st = load_library().gdn_attn_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(qn) if noisy else None, _ptr(kn) if noisy else None,
+                                         _ptr(vn) if noisy else None, offs.ctypes.data_as(ip), pl.ctypes.data_as(ip),
+                                         _ptr(out), _ptr(out_noisy) if noisy else None, _ptr(ws),
+                                         ctypes.c_size_t(ws_bytes), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, f"gdn_attn_forward failed: {status_string(st)}")
+    return out, out_noisy

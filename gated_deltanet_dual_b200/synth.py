@@ -281,3 +281,61 @@ def make_decode_problem(num_seqs: int, num_heads: int, d: int, num_tokens: int, 
     g = (torch.rand(N, L, H, generator=gen, device=device) * g_lo).contiguous()
     beta = torch.sigmoid(normal(N, L, H) * beta_std).contiguous()
     return DecodeProblem(state_pool=pool, slots=slots, q=q, k=k, v=v, g=g, beta=beta)
+
+
+# ----------------------------------------------------------------------------- softmax attention
+@dataclasses.dataclass
+class AttnProblem:
+    """Inputs of one dual-stream attention call (layouts of include/gdn_attention.h)."""
+    q: torch.Tensor            # [T, H, d]
+    k: torch.Tensor            # [T, H_kv, d]
+    v: torch.Tensor
+    qn: torch.Tensor           # [V, T_R, H, d]
+    kn: torch.Tensor           # [V, T_R, H_kv, d]
+    vn: torch.Tensor
+    doc_offsets: np.ndarray    # int32 [N+1]
+    prompt_len: np.ndarray     # int32 [N]
+    block_size: int
+
+
+# The attention layers of the same hybrid model on the same token layouts as the GDN workloads
+# (same document split and blocks); H query heads, H_kv key/value heads.
+ATTN_WORKLOADS = {
+    "attn_train_8x4096_h16_d128": dict(layout="train_8x4096_h16_d128", num_heads=16, num_kv_heads=16),
+    "attn_packed_32768_h16_d128": dict(layout="packed_32768_h16_d128", num_heads=16, num_kv_heads=16),
+    "attn_train_8x4096_h32kv8_d128": dict(layout="train_8x4096_h16_d128", num_heads=32, num_kv_heads=8),
+}
+
+
+def make_attn_problem_from_layout(doc_offsets, prompt_len, *, num_heads: int, num_kv_heads: int, d: int,
+                                  block_size: int, num_views: int = 2, seed: int = 0,
+                                  device="cpu") -> AttnProblem:
+    """q, k, v ~ N(0, 1) in fp32, cast to bf16 (scores q.k / sqrt(d) ~ N(0, 1)).  Draw order:
+    q, k, v, then per view qn, kn, vn."""
+    doc_offsets = np.asarray(doc_offsets, dtype=np.int32)
+    prompt_len = np.asarray(prompt_len, dtype=np.int32)
+    T = int(doc_offsets[-1])
+    T_R = int((np.diff(doc_offsets.astype(np.int64)) - prompt_len).sum())
+    H, Hkv, V = num_heads, num_kv_heads, num_views
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    normal = lambda *s: torch.randn(*s, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    q, k, v = normal(T, H, d), normal(T, Hkv, d), normal(T, Hkv, d)
+    views = [(normal(T_R, H, d), normal(T_R, Hkv, d), normal(T_R, Hkv, d)) for _ in range(V)]
+    if V > 0:
+        qn, kn, vn = (torch.stack([vw[i] for vw in views]).contiguous() for i in range(3))
+    else:
+        qn = torch.empty(0, T_R, H, d, dtype=torch.bfloat16, device=device)
+        kn = torch.empty(0, T_R, Hkv, d, dtype=torch.bfloat16, device=device)
+        vn = torch.empty(0, T_R, Hkv, d, dtype=torch.bfloat16, device=device)
+    return AttnProblem(q=q, k=k, v=v, qn=qn, kn=kn, vn=vn, doc_offsets=doc_offsets, prompt_len=prompt_len,
+                       block_size=block_size)
+
+
+def make_attn_problem(name: str, seed: int = 0, device="cpu") -> AttnProblem:
+    cfg = ATTN_WORKLOADS[name]
+    wl = get_workload(cfg["layout"])
+    offs, prompts = doc_layout(wl, seed)
+    return make_attn_problem_from_layout(offs, prompts, num_heads=cfg["num_heads"], num_kv_heads=cfg["num_kv_heads"],
+                                         d=wl.d, block_size=wl.block_size, num_views=wl.num_views, seed=seed,
+                                         device=device)

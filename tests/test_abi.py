@@ -256,3 +256,78 @@ def test_route1_host_validation():
     dc = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32, conv_width=4, algo=b.ALGO_ROUTE1)
     assert _call(dc, [0, 16, 40], [8, 4], conv_w=_Fake(0x7f0000000000), _ws_bytes=need) == b.GDN_ERR_UNSUPPORTED
     assert _call(d, [0, 16, 40], [8, 4], _ws_bytes=need) == b.GDN_ERR_CUDA              # valid; no device here
+
+
+def _attn_call(desc, offs, pl, ws_bytes=None, **over):
+    base = 0x7f0000000000
+    names = ["q", "k", "v", "qn", "kn", "vn", "out", "out_noisy", "ws"]
+    ptr = {n: base + 0x10000000 * i for i, n in enumerate(names)}
+    ptr.update(over)
+    lib = b.load_library()
+    p = lambda n: None if ptr[n] is None else ctypes.c_void_p(ptr[n])
+    o = np.ascontiguousarray(offs, dtype=np.int32)
+    l = np.ascontiguousarray(pl, dtype=np.int32)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    if ws_bytes is None:
+        ws_bytes = b.attn_workspace_size(desc, o, l)
+    return lib.gdn_attn_forward(ctypes.byref(desc) if desc is not None else None, p("q"), p("k"), p("v"), p("qn"),
+                                p("kn"), p("vn"), o.ctypes.data_as(ip), l.ctypes.data_as(ip), p("out"),
+                                p("out_noisy"), p("ws"), ctypes.c_size_t(ws_bytes), None)
+
+
+def test_attention_workspace_size():
+    d = b.make_attn_desc(2, 4, 2, 128, 2, 4, b.GDN_BF16)
+    # document 0: 3 clean tiles + 2 views x 2 noisy tiles; document 1: 1 + 2 x 1 -> 10 work items
+    assert b.attn_workspace_size(d, [0, 300, 400], [100, 4]) == 256 + 256
+    assert b.attn_workspace_size(d, [0, 300, 400], [101, 4]) == 0       # response 199 % 4
+    assert b.attn_workspace_size(d, [0, 300, 200], [100, 4]) == 0       # offsets decrease
+    assert b.attn_workspace_size(d, [1, 300, 400], [100, 4]) == 0       # must start at 0
+    bad = b.make_attn_desc(2, 4, 2, 128, 2, 4, b.GDN_BF16)
+    bad.reserved = 1
+    assert b.attn_workspace_size(bad, [0, 300, 400], [100, 4]) == 0
+
+
+@no_gpu
+@pytest.mark.parametrize("case,expect", [
+    ("null_desc", b.GDN_ERR_INVALID_ARG), ("reserved", b.GDN_ERR_INVALID_ARG), ("zero_heads", b.GDN_ERR_INVALID_ARG),
+    ("bad_layout", b.GDN_ERR_INVALID_ARG), ("null_q", b.GDN_ERR_INVALID_ARG), ("null_noisy", b.GDN_ERR_INVALID_ARG),
+    ("small_workspace", b.GDN_ERR_INVALID_ARG), ("misaligned_k", b.GDN_ERR_ALIGNMENT),
+    ("d64", b.GDN_ERR_UNSUPPORTED), ("fp32", b.GDN_ERR_UNSUPPORTED), ("kv_heads_3", b.GDN_ERR_UNSUPPORTED),
+    ("views_3", b.GDN_ERR_UNSUPPORTED), ("block_3", b.GDN_ERR_UNSUPPORTED),
+    ("valid_no_device", b.GDN_ERR_CUDA),
+])
+def test_attention_host_validation(case, expect):
+    d = b.make_attn_desc(2, 4, 2, 128, 2, 4, b.GDN_BF16)
+    offs, pl, over, ws = [0, 300, 400], [100, 4], {}, None
+    if case == "null_desc":
+        d = None
+        ws = 4096
+    elif case == "reserved":
+        d.reserved = 2
+        ws = 4096
+    elif case == "zero_heads":
+        d.num_heads = 0
+        ws = 4096
+    elif case == "bad_layout":
+        pl = [101, 4]
+        ws = 4096
+    elif case == "null_q":
+        over["q"] = None
+    elif case == "null_noisy":
+        over["vn"] = None
+    elif case == "small_workspace":
+        ws = 300
+    elif case == "misaligned_k":
+        over["k"] = 0x7f0000000004
+    elif case == "d64":
+        d.head_dim = 64
+    elif case == "fp32":
+        d.dtype = b.GDN_FP32
+    elif case == "kv_heads_3":
+        d.num_kv_heads = 3
+    elif case == "views_3":
+        d.num_views = 3
+    elif case == "block_3":
+        d.block_size = 3
+        pl = [102, 4]     # responses 198 and 96: multiples of 3
+    assert _attn_call(d, offs, pl, ws_bytes=ws, **over) == expect
