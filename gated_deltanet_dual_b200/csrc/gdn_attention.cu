@@ -52,7 +52,7 @@ struct AttnParams {
     int32_t H, Hkv, V, B;
     int64_t TR;
     float scale_log2;                       // log2(e) / sqrt(d)
-    const int32_t *items;                   // work list: tile << 13 | kind << 11 | doc
+    const int32_t *items;                   // work list: (tile << 13 | kind << 11 | doc, head) pairs
     WorkspaceHeader *ws;
     void *out, *out_noisy;
     int32_t doc_start[kMaxDocs + 1];
@@ -63,6 +63,13 @@ struct AttnParams {
 struct AttnMaps {
     CUtensorMap q, k, v, qn, kn, vn;
 };
+
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error ~2^-22, 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
@@ -78,8 +85,8 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int item = P.items[blockIdx.x / P.H];
-    const int h = blockIdx.x % P.H;
+    const int item = P.items[2 * blockIdx.x];
+    const int h = P.items[2 * blockIdx.x + 1];
     const int hk = h / (P.H / P.Hkv);
     const int n = item & 2047, kind = (item >> 11) & 3, tile = item >> 13;
     const int s = P.doc_start[n], len = P.doc_start[n + 1] - s, Pn = P.doc_prompt[n], R = len - Pn;
@@ -177,21 +184,33 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
             lo = b0 - AT * tile;
             hi = min(lo + B, R - AT * tile);
         }
-        // ---- pass 1: masked row max (log2 units)
-        float mt = -INFINITY;
-#pragma unroll 1
-        for (int c0 = 0; c0 < AT; c0 += 32) {
-            float x[32];
-            tmem_ld32(tmem_addr(tb, warp * 32, TA_S + c0), x);
-            tmem_wait_ld();
+        // ---- the row of S (one tensor-memory read), masked row max in log2 units
+        float x[4][32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                if (c0 + e >= lo && c0 + e < hi) mt = fmaxf(mt, x[e] * sl2);
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem_addr(tb, warp * 32, TA_S + 32 * c), x[c]);
+        tmem_wait_ld();
+        const bool full = lo <= 0 && hi >= AT;                  // every key of the tile visible
+        float mt = -INFINITY;
+        if (full) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) mt = fmaxf(mt, x[c][e]);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int col = 32 * c + e;
+                    x[c][e] = (col >= lo && col < hi) ? x[c][e] : -INFINITY;
+                    mt = fmaxf(mt, x[c][e]);
+                }
         }
+        mt *= sl2;                                              // sl2 > 0; -inf stays -inf
         // ---- reference max: move it (and rescale O, l) only past the margin
         float alpha = 1.f;
         if (mt > m_ref + kRescaleLog2) {
-            alpha = m_ref == -INFINITY ? 0.f : exp2f(m_ref - mt);
+            alpha = m_ref == -INFINITY ? 0.f : ex2_approx(m_ref - mt);
             m_ref = mt;
         }
         const float mu = m_ref == -INFINITY ? 0.f : m_ref;
@@ -207,35 +226,21 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
             }
         }
         l *= alpha;
-        // ---- pass 2: P = 2^(s - m) as bf16 pairs over S columns [0, 64); 64 scores at a time, so
-        // each store lands on columns already read
-#pragma unroll 1
-        for (int c0 = 0; c0 < AT; c0 += 64) {
-            float x0[32], x1[32], pk[32];
-            tmem_ld32(tmem_addr(tb, warp * 32, TA_S + c0), x0);
-            tmem_ld32(tmem_addr(tb, warp * 32, TA_S + c0 + 32), x1);
-            tmem_wait_ld();
+        // ---- P = 2^(s - m) (masked scores are -inf: 0) as bf16 pairs over S columns [0, 64)
+        float ls = 0.f;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            float pk[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-                const int c = c0 + e;
-                const float p = (c >= lo && c < hi) ? exp2f(x0[e] * sl2 - mu) : 0.f;
-                x0[e] = p;
-                l += p;
+                const float p0 = ex2_approx(fmaf(x[2 * hf + e / 16][(2 * e) % 32], sl2, -mu));
+                const float p1 = ex2_approx(fmaf(x[2 * hf + e / 16][(2 * e) % 32 + 1], sl2, -mu));
+                ls += p0 + p1;
+                pk[e] = __uint_as_float(pack_bf2(p0, p1));
             }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int c = c0 + 32 + e;
-                const float p = (c >= lo && c < hi) ? exp2f(x1[e] * sl2 - mu) : 0.f;
-                x1[e] = p;
-                l += p;
-            }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                pk[e] = __uint_as_float(pack_bf2(x0[2 * e], x0[2 * e + 1]));
-                pk[16 + e] = __uint_as_float(pack_bf2(x1[2 * e], x1[2 * e + 1]));
-            }
-            tmem_st32(tmem_addr(tb, warp * 32, TA_S + c0 / 2), pk);
+            tmem_st32(tmem_addr(tb, warp * 32, TA_S + 32 * hf), pk);
         }
+        l += ls;
         tmem_wait_st();
         tc_fence_before();
         __syncthreads();
@@ -342,23 +347,35 @@ bool attn_layout(const gdn_attn_desc *d, const int32_t *offs, const int32_t *pl,
     *T = offs[N];
     *TR = tr;
     if (items) {
+        // (document, head) groups, longest documents first; inside a group every query tile of the
+        // document (clean and noisy, heaviest first), so the CTAs that run together read the same
+        // key / value tiles through L2.  Heads that share a key/value head are adjacent.
+        for (int n = 0; n < N; ++n)       // tile index must fit 18 bits
+            if ((int64_t)offs[n + 1] - offs[n] > ((int64_t)1 << 18) * AT) return false;
         const int V = tr > 0 ? d->num_views : 0;
-        std::vector<std::pair<int64_t, int32_t>> list;
-        for (int n = 0; n < N; ++n) {
+        std::vector<int> order(N);
+        std::iota(order.begin(), order.end(), 0);
+        std::stable_sort(order.begin(), order.end(),
+                         [&](int a, int b) { return offs[a + 1] - offs[a] > offs[b + 1] - offs[b]; });
+        items->clear();
+        std::vector<std::pair<int64_t, int32_t>> tiles;
+        for (int n : order) {
             const int64_t len = (int64_t)offs[n + 1] - offs[n], P = pl[n], R = len - P;
-            for (int64_t t = 0; t * AT < len; ++t) list.push_back({t + 1, (int32_t)((t << 13) | n)});
+            tiles.clear();
+            for (int64_t t = 0; t * AT < len; ++t) tiles.push_back({t + 1, (int32_t)((t << 13) | n)});
             for (int v = 0; v < V; ++v)
                 for (int64_t t = 0; t * AT < R; ++t) {
                     const int64_t ilast = std::min<int64_t>(AT * t + AT - 1, R - 1);
                     const int64_t cost = (P + (ilast / B) * B + AT - 1) / AT + 1;
-                    list.push_back({cost, (int32_t)((t << 13) | ((v + 1) << 11) | n)});
+                    tiles.push_back({cost, (int32_t)((t << 13) | ((v + 1) << 11) | n)});
+                }
+            std::stable_sort(tiles.begin(), tiles.end(), [](const auto &a, const auto &b) { return a.first > b.first; });
+            for (int h = 0; h < d->num_heads; ++h)
+                for (const auto &t : tiles) {
+                    items->push_back(t.second);
+                    items->push_back(h);
                 }
         }
-        std::stable_sort(list.begin(), list.end(), [](const auto &a, const auto &b) { return a.first > b.first; });
-        items->resize(list.size());
-        for (size_t i = 0; i < list.size(); ++i) (*items)[i] = list[i].second;
-        for (int n = 0; n < N; ++n)       // tile index must fit 18 bits
-            if ((int64_t)offs[n + 1] - offs[n] > ((int64_t)1 << 18) * AT) return false;
     }
     return true;
 }
@@ -444,7 +461,7 @@ extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q,
     if (cudaMemcpyAsync(static_cast<uint8_t *>(workspace) + attn_items_offset(), items.data(),
                         items.size() * sizeof(int32_t), cudaMemcpyHostToDevice, st) != cudaSuccess)
         return GDN_ERR_CUDA;
-    const int64_t grid = (int64_t)items.size() * H;
+    const int64_t grid = (int64_t)items.size() / 2;
     if (grid > INT32_MAX) return GDN_ERR_UNSUPPORTED;
     gdn_attention_kernel<<<(unsigned)grid, kAThreads, A_SMEM, st>>>(P, maps);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;

@@ -277,8 +277,9 @@ def _attn_call(desc, offs, pl, ws_bytes=None, **over):
 
 def test_attention_workspace_size():
     d = b.make_attn_desc(2, 4, 2, 128, 2, 4, b.GDN_BF16)
-    # document 0: 3 clean tiles + 2 views x 2 noisy tiles; document 1: 1 + 2 x 1 -> 10 work items
-    assert b.attn_workspace_size(d, [0, 300, 400], [100, 4]) == 256 + 256
+    # document 0: 3 clean tiles + 2 views x 2 noisy tiles; document 1: 1 + 2 x 1 -> 10 tiles, each
+    # for 4 heads: 40 (tile, head) work items of 8 bytes
+    assert b.attn_workspace_size(d, [0, 300, 400], [100, 4]) == 256 + 512
     assert b.attn_workspace_size(d, [0, 300, 400], [101, 4]) == 0       # response 199 % 4
     assert b.attn_workspace_size(d, [0, 300, 200], [100, 4]) == 0       # offsets decrease
     assert b.attn_workspace_size(d, [1, 300, 400], [100, 4]) == 0       # must start at 0
