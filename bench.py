@@ -41,9 +41,11 @@ KERNEL_SOURCES = {
     gb.ALGO_SEQUENTIAL: ["gated_deltanet_dual_b200/csrc/gdn_sequential.cu"],
     gb.ALGO_CHUNKED: ["gated_deltanet_dual_b200/csrc/gdn_chunked.cu"],
     gb.ALGO_ROUTE1: ["gated_deltanet_dual_b200/csrc/gdn_decode.cu"],
+    "attention": ["gated_deltanet_dual_b200/csrc/gdn_attention.cu"],
 }
 KERNEL_NAMES = {gb.ALGO_SEQUENTIAL: "gdn_sequential_kernel", gb.ALGO_CHUNKED: "gdn_chunked_kernel",
-                gb.ALGO_ROUTE1: "gdn_route1_chain_kernel + gdn_decode_kernel (block end)"}
+                gb.ALGO_ROUTE1: "gdn_route1_chain_kernel + gdn_decode_kernel (block end)",
+                "attention": "gdn_attention_kernel"}
 
 
 # ----------------------------------------------------------------------------- work model
@@ -77,7 +79,8 @@ def measured_peaks():
 
 def kernel_hash(algo) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES.get(algo, []) + ["gated_deltanet_dual_b200/csrc/gdn_internal.cuh"]:
+    for rel in KERNEL_SOURCES.get(algo, []) + ["gated_deltanet_dual_b200/csrc/gdn_internal.cuh",
+                                               "gated_deltanet_dual_b200/csrc/sm100.cuh"]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -558,7 +561,8 @@ def run_attention(args, name, rank, world, local):
     peaks = measured_peaks()
     achieved = flops / (ms / 1e3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": None, "peak_source": peaks["source"] + " (burst)",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic("attention", name),
+                "peak_source": peaks["source"] + " (burst)",
                 "kernel": "gdn_attention_kernel", "algorithmic_flops": flops, "visible_pairs": pairs}
     toks = (T + V * TR) * world
     value = toks / (ms / 1e3)
