@@ -23,7 +23,8 @@ ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED, ALGO_ROUTE1 = 0, 1, 2, 3
 EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device_status",
             "gdn_status_string", "gdn_dual_version", "gdn_dual_select_algo",
             "gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit", "gdn_dual_workspace_size_route1",
-            "gdn_attn_forward", "gdn_attn_workspace_size")
+            "gdn_attn_forward", "gdn_attn_workspace_size", "gdn_dual_backward",
+            "gdn_dual_backward_workspace_size")
 
 
 class GdnError(RuntimeError):
@@ -82,6 +83,11 @@ def load_library(path: str = LIB_PATH):
             lib.gdn_decode_replay.argtypes = [dd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.gdn_decode_verify.argtypes = [dd, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
             lib.gdn_decode_commit.argtypes = [dd, vp, vp, vp, vp, vp, vp]
+            lib.gdn_dual_backward_workspace_size.restype = ctypes.c_size_t
+            lib.gdn_dual_backward_workspace_size.argtypes = [ctypes.POINTER(Desc), ip]
+            lib.gdn_dual_backward.restype = ctypes.c_int
+            lib.gdn_dual_backward.argtypes = ([ctypes.POINTER(Desc)] + [vp] * 10 + [ip, ip] + [vp] * 3 + [vp] * 10
+                                              + [vp, ctypes.c_size_t, vp])
             ad = ctypes.POINTER(AttnDesc)
             lib.gdn_attn_workspace_size.restype = ctypes.c_size_t
             lib.gdn_attn_workspace_size.argtypes = [ad, ip, ip]
@@ -397,3 +403,61 @@ def attention_forward(q, k, v, qn, kn, vn, doc_offsets, prompt_len, block_size, 
     if st != GDN_OK:
         raise GdnError(st, f"gdn_attn_forward failed: {status_string(st)}")
     return out, out_noisy
+
+
+# ----------------------------------------------------------------------------- backward
+def backward_workspace_size(desc: Desc, doc_offsets) -> int:
+    offs = np.ascontiguousarray(doc_offsets, dtype=np.int32)
+    return int(load_library().gdn_dual_backward_workspace_size(ctypes.byref(desc),
+                                                                offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))))
+
+
+def backward(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, block_size, d_out, d_out_noisy,
+             d_final_state=None, *, workspace=None, stream=None):
+    """Gradients of <d_out, out> + <d_out_noisy, out_noisy> + <d_final_state, final_state> with
+    respect to every input of the dual-stream forward (gdn_dual_backward), fp32.  Returns a dict
+    dq, dk, dv, dg, dbeta, dqn, dkn, dvn, dgn, dbetan."""
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    T, H, dk_ = q.shape
+    dv_ = v.shape[2]
+    V, TR = qn.shape[0], qn.shape[1]
+    offs = np.ascontiguousarray(doc_offsets, dtype=np.int32)
+    pl = np.ascontiguousarray(prompt_len, dtype=np.int32)
+    N = len(pl)
+    if offs.shape != (N + 1,) or (N >= 1 and int(offs[-1]) != T):
+        raise ValueError("doc_offsets must be [N+1] and end at T")
+    if N >= 1 and int((np.diff(offs.astype(np.int64)) - pl).sum()) != TR:
+        raise ValueError("noisy tensors do not match the documents' response tokens")
+    io, f32 = q.dtype, torch.float32
+    for t, name, shape, dt in ((q, "q", (T, H, dk_), io), (k, "k", (T, H, dk_), io), (v, "v", (T, H, dv_), io),
+                               (g, "g", (T, H), f32), (beta, "beta", (T, H), f32),
+                               (qn, "qn", (V, TR, H, dk_), io), (kn, "kn", (V, TR, H, dk_), io),
+                               (vn, "vn", (V, TR, H, dv_), io), (gn, "gn", (V, TR, H), f32),
+                               (betan, "betan", (V, TR, H), f32), (d_out, "d_out", (T, H, dv_), io),
+                               (d_out_noisy, "d_out_noisy", (V, TR, H, dv_), io),
+                               (d_final_state, "d_final_state", (N, H, dk_, dv_), f32)):
+        _check(t, name, shape, dt, dev)
+    out = {n: torch.empty(x.shape, dtype=f32, device=dev) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dg", g),
+                                                                         ("dbeta", beta), ("dqn", qn), ("dkn", kn),
+                                                                         ("dvn", vn), ("dgn", gn), ("dbetan", betan))}
+    desc = make_desc(N, H, dk_, dv_, V, int(block_size), _dtype_code(q))
+    ws = workspace
+    if ws is None:
+        nbytes = backward_workspace_size(desc, offs)
+        if nbytes:
+            ws = Workspace(nbytes, device=dev).tensor
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    noisy = V > 0 and TR > 0
+    nz = lambda t: _ptr(t) if noisy else None
+    ip = ctypes.POINTER(ctypes.c_int32)
+    st = load_library().gdn_dual_backward(
+        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), nz(qn), nz(kn), nz(vn), nz(gn), nz(betan),
+        offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(d_out), nz(d_out_noisy), _ptr(d_final_state),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+        nz(out["dqn"]), nz(out["dkn"]), nz(out["dvn"]), nz(out["dgn"]), nz(out["dbetan"]),
+        _ptr(ws), ctypes.c_size_t(ws_bytes), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, f"gdn_dual_backward failed: {status_string(st)}")
+    return out

@@ -1,0 +1,398 @@
+// gdn_backward.cu -- backward pass of the dual-stream Gated DeltaNet forward on CUDA cores
+// (sm_100a), and its C ABI (gdn_dual_backward in gdn_dual.h).
+//
+// "FLARE: Diffusion for Hybrid Language Model" (papernotes.org notes), Method > Key design 2:
+// the backward injects every noisy block's gradient into the causal chain.  With
+// Lam_t = dL/dS_t (L = <do, out> + <do~, out_noisy> + <dS, final_state>):
+//   Lam_t  = q_t do_t^T / sqrt(d) + A_{t+1}^T Lam_{t+1} + sum_views Lam~_0 of the block starting at t+1,
+//   Lam~_B = sum_l q~_l do~_l^T / sqrt(d),  Lam~_{i-1} = A~_i^T Lam~_i   (A = alpha (I - beta k k^T) = A^T)
+// and per step (state S_prev before it, Lam after it):
+//   dv = beta Lam^T k,  dk = beta Lam v - alpha beta (Lam S_prev^T k + S_prev Lam^T k),
+//   dbeta = k^T Lam v - alpha (k^T S_prev)(Lam^T k),  dg = alpha (<Lam, S_prev> - beta (k^T S_prev)(Lam^T k)),
+//   dq_t = S_t do_t / sqrt(d).
+//
+// Every column of S evolves on its own (the rule only mixes rows), and so does every column of
+// Lam.  One CTA takes one (document, head, slice of 32 columns); two threads per column hold half
+// of its rows of S and of Lam in registers (a pair shuffle completes the k^T S and k^T Lam dot
+// products).  Gradients that sum over columns (dq, dk, dg, dbeta) are reduced over the CTA's 32
+// columns in shared memory and added into the fp32 outputs with atomics (one add per slice).
+//   pass 1: the clean chain, writing the state before every 16th token into the workspace
+//   pass 2: 16-token segments from the last: the segment's states are rebuilt from its
+//           checkpoint, 4 tokens at a time into shared memory, and the adjoint runs backwards
+//           through them; where a response block starts right after a token, each view's block
+//           is rebuilt from that token's state (token by token, from the start for every step)
+//           and run backwards, and its initial-state gradient joins Lam.
+// The work per token is a few dot products of length d per column: CUDA cores, not tensor cores.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int kBwdThreads = 64;       // 32 columns x 2 row halves
+constexpr int kCk = 16;               // checkpoint stride (tokens)
+constexpr int kSeg = 4;               // states rebuilt into shared memory at a time
+
+struct BwdParams {
+    const void *q, *k, *v, *qn, *kn, *vn, *dout, *doutn;
+    const float *g, *beta, *gn, *betan, *dsf;
+    float *dq, *dk, *dv, *dg, *dbeta, *dqn, *dkn, *dvn, *dgn, *dbetan;
+    float *ck;                        // checkpoints [ck index][H][slice][R2][64]
+    int64_t TR;
+    int32_t N, H, V, B;
+    float scale;
+    int32_t doc_start[kMaxDocs + 1];
+    int32_t doc_prompt[kMaxDocs];
+    int32_t resp_off[kMaxDocs + 1];
+    int32_t ck_off[kMaxDocs + 1];     // first checkpoint of each document
+};
+
+template <typename T>
+__device__ __forceinline__ float ld(const void *p, int64_t i) {
+    return to_f32(static_cast<const T *>(p)[i]);
+}
+
+template <int R2>
+__device__ __forceinline__ float pair_sum(float x) {
+    return x + __shfl_xor_sync(0xffffffffu, x, 1);
+}
+
+template <typename TIO, int D>
+__global__ void __launch_bounds__(kBwdThreads)
+gdn_backward_kernel(const __grid_constant__ BwdParams P) {
+    constexpr int R2 = D / 2, NS = D / 32;
+    extern __shared__ float smb[];
+    float *seg = smb;                                 // [kSeg][R2][64]: states before the tokens
+    float *s0b = seg + kSeg * R2 * kBwdThreads;        // [R2][64]: a noisy block's start state
+    float *lmb = s0b + R2 * kBwdThreads;              // [R2][64]: the clean Lam while a block runs
+    float *red = lmb + R2 * kBwdThreads;              // [32][D + 2]: column reduction
+    const int tid = threadIdx.x, c = tid >> 1, hf = tid & 1, rb = hf * R2;
+    const int unit = blockIdx.x / NS, js = blockIdx.x % NS, col = js * 32 + c;
+    const int n = unit / P.H, h = unit % P.H, H = P.H;
+    const int s = P.doc_start[n], len = P.doc_start[n + 1] - s, Pn = P.doc_prompt[n], R = len - Pn;
+    const int roff = P.resp_off[n];
+    const float sc = P.scale;
+    auto at = [&](float *buf, int i) -> float & { return buf[i * kBwdThreads + tid]; };
+
+    // token data of clean row t (or noisy packed row when noisy): k and q rows of this thread
+    auto kq = [&](const void *base, int64_t row, float (&x)[R2]) {
+        const int64_t o = (row * H + h) * D + rb;
+#pragma unroll
+        for (int i = 0; i < R2; ++i) x[i] = ld<TIO>(base, o + i);
+    };
+    // one forward step of this thread's half column
+    auto fwd = [&](float (&st)[R2], const float (&kk)[R2], float vc, float a, float b) {
+        float ks = 0.f;
+#pragma unroll
+        for (int i = 0; i < R2; ++i) ks = fmaf(kk[i], st[i], ks);
+        ks = pair_sum<R2>(ks);
+#pragma unroll
+        for (int i = 0; i < R2; ++i) st[i] = a * fmaf(-b * ks, kk[i], st[i]) + b * kk[i] * vc;
+    };
+    // reduce red[c][0..D+1] over the 32 columns, add into out_vec[0..D) and the two scalars
+    auto reduce_add = [&](float *out_vec, float *sc0, float *sc1) {
+        __syncthreads();
+        for (int r = tid; r < D + 2; r += kBwdThreads) {
+            float acc = 0.f;
+#pragma unroll 8
+            for (int cc = 0; cc < 32; ++cc) acc += red[cc * (D + 2) + r];
+            if (r < D) {
+                if (out_vec) atomicAdd(out_vec + r, acc);
+            } else if (r == D) {
+                if (sc0) atomicAdd(sc0, acc);
+            } else if (sc1) {
+                atomicAdd(sc1, acc);
+            }
+        }
+        __syncthreads();
+    };
+    // backward of one step: Lam (after the step) -> Lam before it; S_prev in sp.
+    // Writes dk rows and the dg, dbeta column terms into red, dv of this column into *dv_out.
+    auto bwd = [&](float (&lam)[R2], const float (&sp)[R2], const float (&kk)[R2], float vc, float a, float b,
+                   float *dv_out) {
+        float kl = 0.f, ks = 0.f, ls = 0.f;
+#pragma unroll
+        for (int i = 0; i < R2; ++i) {
+            kl = fmaf(kk[i], lam[i], kl);
+            ks = fmaf(kk[i], sp[i], ks);
+            ls = fmaf(lam[i], sp[i], ls);
+        }
+        kl = pair_sum<R2>(kl);
+        ks = pair_sum<R2>(ks);
+        float *rr = red + c * (D + 2);
+#pragma unroll
+        for (int i = 0; i < R2; ++i) rr[rb + i] = b * vc * lam[i] - a * b * (ks * lam[i] + kl * sp[i]);
+        // dalpha = <Lam, S_prev> - beta ks kl ; dg = alpha dalpha ; dbeta = kl v - alpha ks kl
+        const float own = a * ls;                             // this half's part of alpha <Lam, S_prev>
+        const float other = __shfl_xor_sync(0xffffffffu, own, 1);
+        if (hf == 0) {
+            rr[D] = own + other - a * b * ks * kl;
+            rr[D + 1] = kl * vc - a * ks * kl;
+            *dv_out = b * kl;
+        }
+#pragma unroll
+        for (int i = 0; i < R2; ++i) lam[i] = a * fmaf(-b * kl, kk[i], lam[i]);
+    };
+    // dq rows = S do / sqrt(d) for one token, reduced over the columns
+    auto dq_rows = [&](const float (&st)[R2], float doc_, float *out_vec) {
+        float *rr = red + c * (D + 2);
+#pragma unroll
+        for (int i = 0; i < R2; ++i) rr[rb + i] = st[i] * doc_ * sc;
+        if (hf == 0) rr[D] = rr[D + 1] = 0.f;
+        reduce_add(out_vec, nullptr, nullptr);
+    };
+
+    // Backward of every view of the noisy block at packed rows [roff + r0, +B), started from the
+    // state in s0b; adds the views' initial-state gradients into lmb.
+    auto noisy_block = [&](int r0, float (&sw)[R2], float (&lt)[R2]) {
+        for (int w = 0; w < P.V; ++w) {
+            const int64_t base = (int64_t)w * P.TR + roff + r0;
+            float kk[R2], qq[R2];
+            // forward to the block end
+#pragma unroll
+            for (int i = 0; i < R2; ++i) sw[i] = at(s0b, i);
+            for (int j = 0; j < P.B; ++j) {
+                const int64_t row = base + j;
+                kq(P.kn, row, kk);
+                fwd(sw, kk, ld<TIO>(P.vn, (row * H + h) * D + col), expf(P.gn[row * H + h]), P.betan[row * H + h]);
+            }
+            // Lam~_B and dq~ of every position
+#pragma unroll
+            for (int i = 0; i < R2; ++i) lt[i] = 0.f;
+            for (int j = 0; j < P.B; ++j) {
+                const int64_t row = base + j;
+                const float dd = ld<TIO>(P.doutn, (row * H + h) * D + col);
+                kq(P.qn, row, qq);
+#pragma unroll
+                for (int i = 0; i < R2; ++i) lt[i] = fmaf(qq[i], dd * sc, lt[i]);
+                dq_rows(sw, dd, P.dqn + (row * H + h) * D);
+            }
+            // steps from the last: rebuild the state before step j from the block start
+            for (int j = P.B - 1; j >= 0; --j) {
+#pragma unroll
+                for (int i = 0; i < R2; ++i) sw[i] = at(s0b, i);
+                for (int jj = 0; jj < j; ++jj) {
+                    const int64_t row = base + jj;
+                    kq(P.kn, row, kk);
+                    fwd(sw, kk, ld<TIO>(P.vn, (row * H + h) * D + col), expf(P.gn[row * H + h]),
+                        P.betan[row * H + h]);
+                }
+                const int64_t row = base + j;
+                kq(P.kn, row, kk);
+                float dvc = 0.f;
+                bwd(lt, sw, kk, ld<TIO>(P.vn, (row * H + h) * D + col), expf(P.gn[row * H + h]),
+                    P.betan[row * H + h], &dvc);
+                if (hf == 0) P.dvn[(row * H + h) * D + col] = dvc;
+                reduce_add(P.dkn + (row * H + h) * D, P.dgn + row * H + h, P.dbetan + row * H + h);
+            }
+#pragma unroll
+            for (int i = 0; i < R2; ++i) at(lmb, i) += lt[i];
+        }
+    };
+
+    float st[R2], lam[R2], kk[R2];
+    // ---------------- pass 1: clean chain with checkpoints every kCk tokens
+#pragma unroll
+    for (int i = 0; i < R2; ++i) st[i] = 0.f;
+    auto ckp = [&](int ci) -> float * {
+        return P.ck + (((int64_t)(P.ck_off[n] + ci) * H + h) * NS + js) * (R2 * kBwdThreads);
+    };
+    for (int t = 0; t < len; ++t) {
+        if (t % kCk == 0) {
+            float *cp = ckp(t / kCk);
+#pragma unroll
+            for (int i = 0; i < R2; ++i) cp[i * kBwdThreads + tid] = st[i];
+        }
+        const int64_t row = s + t;
+        kq(P.k, row, kk);
+        fwd(st, kk, ld<TIO>(P.v, (row * H + h) * D + col), expf(P.g[row * H + h]), P.beta[row * H + h]);
+    }
+    // st = final state; Lam starts at the final-state gradient
+#pragma unroll
+    for (int i = 0; i < R2; ++i)
+        lam[i] = P.dsf ? P.dsf[(((int64_t)n * H + h) * D + rb + i) * D + col] : 0.f;
+
+    // ---------------- pass 2: backwards over the segments
+    float sp[R2];
+    const int nseg = (len + kCk - 1) / kCk;
+    for (int sgi = nseg - 1; sgi >= 0; --sgi) {
+        const int t0 = sgi * kCk, t1 = min(len, t0 + kCk);
+        for (int u0 = t1 - ((t1 - t0 - 1) % kSeg) - 1; u0 >= t0; u0 -= kSeg) {
+            // rebuild the states before tokens u0 .. u1-1 (u0 >= t0 on a kSeg grid from t0)
+            const int u1 = min(t1, u0 + kSeg);
+            const float *cp = ckp(sgi);
+#pragma unroll
+            for (int i = 0; i < R2; ++i) sp[i] = cp[i * kBwdThreads + tid];
+            for (int t = t0; t < u1; ++t) {
+                if (t >= u0) {
+#pragma unroll
+                    for (int i = 0; i < R2; ++i) at(seg, (t - u0) * R2 + i) = sp[i];
+                }
+                const int64_t row = s + t;
+                kq(P.k, row, kk);
+                fwd(sp, kk, ld<TIO>(P.v, (row * H + h) * D + col), expf(P.g[row * H + h]), P.beta[row * H + h]);
+            }
+            // sp = the state after token u1 - 1
+            for (int t = u1 - 1; t >= u0; --t) {
+                const int64_t row = s + t;
+                const float dd = ld<TIO>(P.dout, (row * H + h) * D + col);
+                float qq[R2];
+                kq(P.q, row, qq);
+#pragma unroll
+                for (int i = 0; i < R2; ++i) lam[i] = fmaf(qq[i], dd * sc, lam[i]);
+                // a response block starts right after this token: its views start from S_t
+                const int rel = t + 1 - Pn;
+                if (rel >= 0 && rel < R && rel % P.B == 0 && P.V > 0) {
+#pragma unroll
+                    for (int i = 0; i < R2; ++i) {
+                        at(s0b, i) = sp[i];
+                        at(lmb, i) = lam[i];
+                    }
+                    noisy_block(rel, sp, lam);
+#pragma unroll
+                    for (int i = 0; i < R2; ++i) {
+                        sp[i] = at(s0b, i);
+                        lam[i] = at(lmb, i);
+                    }
+                }
+                dq_rows(sp, dd, P.dq + (row * H + h) * D);
+                // the state before token t
+#pragma unroll
+                for (int i = 0; i < R2; ++i) sp[i] = at(seg, (t - u0) * R2 + i);
+                kq(P.k, row, kk);
+                float dvc = 0.f;
+                bwd(lam, sp, kk, ld<TIO>(P.v, (row * H + h) * D + col), expf(P.g[row * H + h]),
+                    P.beta[row * H + h], &dvc);
+                if (hf == 0) P.dv[(row * H + h) * D + col] = dvc;
+                reduce_add(P.dk + (row * H + h) * D, P.dg + row * H + h, P.dbeta + row * H + h);
+            }
+        }
+    }
+    // first block of a document without prompt: it starts from the hard zero state
+    if (Pn == 0 && R > 0 && P.V > 0) {
+#pragma unroll
+        for (int i = 0; i < R2; ++i) {
+            at(s0b, i) = 0.f;
+            at(lmb, i) = 0.f;
+        }
+        noisy_block(0, sp, lam);
+    }
+}
+
+template <typename TIO, int D>
+cudaError_t launch_bwd(const BwdParams &p, cudaStream_t st) {
+    constexpr int R2 = D / 2;
+    const size_t smem = (size_t)(kSeg + 2) * R2 * kBwdThreads * 4 + 32 * (D + 2) * 4;
+    cudaError_t e = cudaFuncSetAttribute(gdn_backward_kernel<TIO, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (int64_t)p.N * p.H * (D / 32);
+    gdn_backward_kernel<TIO, D><<<(unsigned)grid, kBwdThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t bwd_checkpoints(const gdn_dual_desc *d, const int32_t *offs) {
+    int64_t nck = 0;
+    for (int n = 0; n < d->num_docs; ++n) nck += ((int64_t)offs[n + 1] - offs[n] + kCk - 1) / kCk;
+    return nck;
+}
+
+bool bwd_desc_ok(const gdn_dual_desc *d) {
+    return d && d->num_docs >= 1 && d->num_docs <= kMaxDocs && d->num_heads >= 1 && d->d_k >= 1 && d->d_v >= 1 &&
+           d->num_views >= 0 && d->block_size >= 1 && (d->dtype == GDN_BF16 || d->dtype == GDN_FP32) &&
+           d->conv_width >= 0 && d->reserved == 0;
+}
+
+}  // namespace
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" size_t gdn_dual_backward_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host) {
+    if (!bwd_desc_ok(desc) || !doc_offsets_host || doc_offsets_host[0] != 0) return 0;
+    for (int n = 0; n < desc->num_docs; ++n)
+        if (doc_offsets_host[n + 1] < doc_offsets_host[n]) return 0;
+    const int64_t nck = bwd_checkpoints(desc, doc_offsets_host);
+    return (size_t)nck * desc->num_heads * desc->d_k * desc->d_v * sizeof(float) + 256;
+}
+
+extern "C" gdn_status gdn_dual_backward(const gdn_dual_desc *desc, const void *q, const void *k, const void *v,
+                                        const float *g, const float *beta, const void *qn, const void *kn,
+                                        const void *vn, const float *gn, const float *betan,
+                                        const int32_t *doc_offsets, const int32_t *prompt_len,
+                                        const void *d_out, const void *d_out_noisy, const float *d_final_state,
+                                        float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                                        float *dqn, float *dkn, float *dvn, float *dgn, float *dbetan,
+                                        void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    if (!bwd_desc_ok(desc) || !doc_offsets || !prompt_len || doc_offsets[0] != 0) return GDN_ERR_INVALID_ARG;
+    const int N = desc->num_docs, H = desc->num_heads, B = desc->block_size, D = desc->d_k;
+    int64_t TR = 0;
+    for (int n = 0; n < N; ++n) {
+        const int64_t len = (int64_t)doc_offsets[n + 1] - doc_offsets[n];
+        if (len < 0 || prompt_len[n] < 0 || prompt_len[n] > len || (len - prompt_len[n]) % B != 0)
+            return GDN_ERR_INVALID_ARG;
+        TR += len - prompt_len[n];
+    }
+    const int64_t T = doc_offsets[N];
+    if (TR > INT32_MAX || T > INT32_MAX) return GDN_ERR_INVALID_ARG;
+    const bool noisy = desc->num_views > 0 && TR > 0;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !d_out || !dq || !dk || !dv || !dg || !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    if (noisy && (!qn || !kn || !vn || !gn || !betan || !d_out_noisy || !dqn || !dkn || !dvn || !dgn || !dbetan))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn_dual_backward_workspace_size(desc, doc_offsets);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, qn, kn, vn, gn, betan, d_out, d_out_noisy, d_final_state,
+                          dq, dk, dv, dg, dbeta, dqn, dkn, dvn, dgn, dbetan, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
+    if (desc->d_k != desc->d_v || (D != 32 && D != 64 && D != 128) || desc->conv_width != 0)
+        return GDN_ERR_UNSUPPORTED;
+    if (T == 0) return GDN_OK;
+
+    BwdParams P;
+    std::memset(&P, 0, sizeof(P));
+    P.q = q; P.k = k; P.v = v; P.qn = qn; P.kn = kn; P.vn = vn; P.dout = d_out; P.doutn = d_out_noisy;
+    P.g = g; P.beta = beta; P.gn = gn; P.betan = betan; P.dsf = d_final_state;
+    P.dq = dq; P.dk = dk; P.dv = dv; P.dg = dg; P.dbeta = dbeta;
+    P.dqn = dqn; P.dkn = dkn; P.dvn = dvn; P.dgn = dgn; P.dbetan = dbetan;
+    P.ck = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + 256);
+    P.TR = TR; P.N = N; P.H = H; P.V = noisy ? desc->num_views : 0; P.B = B;
+    P.scale = (float)(1.0 / std::sqrt((double)D));
+    int64_t roff = 0, ck = 0;
+    for (int n = 0; n <= N; ++n) {
+        P.doc_start[n] = doc_offsets[n];
+        P.resp_off[n] = (int32_t)roff;
+        P.ck_off[n] = (int32_t)ck;
+        if (n < N) {
+            P.doc_prompt[n] = prompt_len[n];
+            roff += (int64_t)doc_offsets[n + 1] - doc_offsets[n] - prompt_len[n];
+            ck += ((int64_t)doc_offsets[n + 1] - doc_offsets[n] + kCk - 1) / kCk;
+        }
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the column-summed gradients are accumulated with atomics
+    const size_t tok = (size_t)T * H, ntok = (size_t)(noisy ? desc->num_views : 0) * TR * H;
+    if (cudaMemsetAsync(dq, 0, tok * D * 4, st) != cudaSuccess || cudaMemsetAsync(dk, 0, tok * D * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(dg, 0, tok * 4, st) != cudaSuccess || cudaMemsetAsync(dbeta, 0, tok * 4, st) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (noisy) {
+        if (cudaMemsetAsync(dqn, 0, ntok * D * 4, st) != cudaSuccess || cudaMemsetAsync(dkn, 0, ntok * D * 4, st) != cudaSuccess ||
+            cudaMemsetAsync(dgn, 0, ntok * 4, st) != cudaSuccess || cudaMemsetAsync(dbetan, 0, ntok * 4, st) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    cudaError_t e;
+    const bool bf = desc->dtype == GDN_BF16;
+    switch (D) {
+        case 32: e = bf ? launch_bwd<__nv_bfloat16, 32>(P, st) : launch_bwd<float, 32>(P, st); break;
+        case 64: e = bf ? launch_bwd<__nv_bfloat16, 64>(P, st) : launch_bwd<float, 64>(P, st); break;
+        default: e = bf ? launch_bwd<__nv_bfloat16, 128>(P, st) : launch_bwd<float, 128>(P, st); break;
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}

@@ -133,6 +133,33 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
                             gdn_stream_t stream);
 
 /*
+ * Backward pass of gdn_dual_forward (Method > Key design 2 of the FLARE notes: the noisy
+ * blocks' gradients are injected into the causal chain).  Given the forward's inputs and the
+ * upstream gradients d_out [T, H, d_v] and d_out_noisy [V, T_R, H, d_v] (dtype = desc->dtype)
+ * and d_final_state [N, H, d_k, d_v] fp32 (NULL = zero), writes the gradients of
+ *   L = <d_out, out> + <d_out_noisy, out_noisy> + <d_final_state, final_state>
+ * with respect to every input, all fp32 in the inputs' layouts: dq dk dv [T, H, d], dg dbeta
+ * [T, H], dqn dkn dvn [V, T_R, H, d], dgn dbetan [V, T_R, H] (fully overwritten; the noisy ones
+ * may be NULL when there are no noisy rows).  The workspace holds the clean states at every
+ * 16th token: at least gdn_dual_backward_workspace_size() bytes.  Host validation as for the
+ * forward; GDN_ERR_UNSUPPORTED for ShortConv (conv_width != 0), d_k != d_v or d not in
+ * {32, 64, 128}.  CUDA-core kernel (one CTA per (document, head, 32 state columns)); the
+ * column-summed gradients are accumulated with fp32 atomics, so their last bits may vary from
+ * call to call.
+ */
+size_t gdn_dual_backward_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host);
+gdn_status gdn_dual_backward(const gdn_dual_desc *desc,
+                             const void *q, const void *k, const void *v,
+                             const float *g, const float *beta,
+                             const void *qn, const void *kn, const void *vn,
+                             const float *gn, const float *betan,
+                             const int32_t *doc_offsets, const int32_t *prompt_len,
+                             const void *d_out, const void *d_out_noisy, const float *d_final_state,
+                             float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                             float *dqn, float *dkn, float *dvn, float *dgn, float *dbetan,
+                             void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
  * gdn_dual_forward without a workspace argument, for callers that cannot allocate device
  * memory: e.g. an engine that reserved all device memory for its own pool up front, or a
  * plugin/FFI host with no device allocator reachable through the C ABI.  (The FLARE notes have

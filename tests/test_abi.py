@@ -332,3 +332,32 @@ def test_attention_host_validation(case, expect):
         d.block_size = 3
         pl = [102, 4]     # responses 198 and 96: multiples of 3
     assert _attn_call(d, offs, pl, ws_bytes=ws, **over) == expect
+
+
+@no_gpu
+def test_backward_host_validation():
+    base = 0x7f0000000000
+    lib = b.load_library()
+    offs = np.array([0, 40, 73], np.int32)
+    pl = np.array([8, 1], np.int32)
+    ip = ctypes.POINTER(ctypes.c_int32)
+
+    def call(desc, ws_bytes=None, over=None):
+        ptr = [ctypes.c_void_p(base + 0x10000000 * i) for i in range(24)]   # 10 inputs, 3 upstream, 10 grads, ws
+        for i, v in (over or {}).items():
+            ptr[i] = None if v is None else ctypes.c_void_p(v)
+        nb = b.backward_workspace_size(desc, offs) if ws_bytes is None else ws_bytes
+        return lib.gdn_dual_backward(ctypes.byref(desc), *ptr[:10], offs.ctypes.data_as(ip), pl.ctypes.data_as(ip),
+                                     *ptr[10:23], ptr[23], ctypes.c_size_t(nb), None)
+
+    d = b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32)
+    # 73 tokens in 16-token checkpoints: 3 + 3 per head, 64 x 64 fp32 each, plus 256 bytes
+    assert b.backward_workspace_size(d, offs) == 256 + 6 * 2 * 64 * 64 * 4
+    assert call(d, ws_bytes=1024) == b.GDN_ERR_INVALID_ARG
+    assert call(d, over={0: None}) == b.GDN_ERR_INVALID_ARG                  # q
+    assert call(d, over={3: base + 4}) == b.GDN_ERR_ALIGNMENT                # g
+    dc = b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32, conv_width=4)
+    assert call(dc) == b.GDN_ERR_UNSUPPORTED
+    d48 = b.make_desc(2, 2, 48, 48, 2, 4, b.GDN_FP32)
+    assert call(d48) == b.GDN_ERR_UNSUPPORTED
+    assert call(d) == b.GDN_ERR_CUDA                                         # valid; no device here
