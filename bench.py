@@ -480,6 +480,16 @@ def attn_pairs(offs, pl, B, V):
     return pairs
 
 
+def blas_threads() -> int:
+    """Threads of the BLAS behind numpy (the numpy oracles' matrix products), else 1."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(i.get("num_threads", 1)) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
 def time_attn_oracle(name, min_seconds=2.0, seed=0):
     """The fp64 oracle on a bounded sample: whole documents of one head (host cores, numpy)."""
     from oracle import attention as oa  # test infrastructure: the CPU baseline / reference arm only
@@ -501,7 +511,7 @@ def time_attn_oracle(name, min_seconds=2.0, seed=0):
         if el >= min_seconds:
             break
     H = pr.q.shape[1]
-    return {"value": toks / el / H, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+    return {"value": toks / el / H, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{n} whole documents of one head (of {H}; {Hkv} key/value heads) through the fp64 "
                       f"numpy oracle; tokens/s scaled to all heads", "seconds": el}
 
@@ -614,6 +624,160 @@ def run_attention(args, name, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- backward
+BWD_METRIC = "dual-stream GDN backward tokens/s on 1 B200 and % of HBM roofline"
+BWD_WORKLOADS = {"bwd_train_8x4096_h16_d128": "train_8x4096_h16_d128"}
+
+
+def backward_bytes(prob) -> int:
+    """Algorithmic HBM bytes of one backward call: read q, k, v, g, beta (both streams) and the
+    upstream output gradients (I/O dtype) and final-state gradient (fp32); write the fp32
+    gradients of every input."""
+    s = prob.q.element_size()
+    d = prob.d_k
+    toks = (prob.T + prob.num_views * prob.T_R) * prob.num_heads
+    return int(toks * (4 * d * s + 8 + 3 * d * 4 + 8) + prob.num_docs * prob.num_heads * d * d * 4)
+
+
+def time_backward_oracle(prob, min_seconds=2.0):
+    """The fp64 backward oracle on a bounded sample: whole documents of one head."""
+    from oracle import backward as ob  # test infrastructure: the CPU baseline / reference arm only
+    offs = prob.doc_offsets.astype(np.int64)
+    roffs = prob.response_offsets()
+    toks, n, t0 = 0, 0, time.perf_counter()
+    while True:
+        d_ = n % prob.num_docs
+        s, e, r0, r1 = int(offs[d_]), int(offs[d_ + 1]), int(roffs[d_]), int(roffs[d_ + 1])
+        sl = lambda t: t[s:e, :1]
+        sn = lambda t: t[:, r0:r1, :1]
+        do = np.ones((e - s, 1, prob.d_v))
+        don = np.ones((prob.num_views, r1 - r0, 1, prob.d_v))
+        ob.dual_backward(sl(prob.q), sl(prob.k), sl(prob.v), sl(prob.g), sl(prob.beta), sn(prob.qn), sn(prob.kn),
+                         sn(prob.vn), sn(prob.gn), sn(prob.betan), [0, e - s], prob.prompt_len[d_:d_ + 1],
+                         prob.block_size, do, don, None)
+        toks += (e - s) + prob.num_views * (r1 - r0)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": toks / el / prob.num_heads, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} whole documents of one head (of {prob.num_heads}) through the fp64 numpy backward "
+                      f"oracle; tokens/s scaled to all heads", "seconds": el}
+
+
+def run_backward(args, name, rank, world, local):
+    wl = synth.get_workload(BWD_WORKLOADS[name])
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        prob = synth.make_problem(wl, seed=0, device="cpu")
+        cb = time_backward_oracle(prob)
+        line = {"metric": BWD_METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": prob.tokens() / cb["value"] * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": name, "parallelism": "replicas", "l2": "not applicable (host)"},
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    replicas.init(world, backend="nccl", device=dev)
+    prob = synth.make_problem(wl, seed=replicas.replica_seed(0, rank), device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7 + rank)
+    do = torch.randn(prob.T, prob.num_heads, prob.d_v, generator=gen, device=dev).to(prob.q.dtype)
+    don = torch.randn(prob.num_views, prob.T_R, prob.num_heads, prob.d_v, generator=gen, device=dev).to(prob.q.dtype)
+    desc = gb.make_desc(prob.num_docs, prob.num_heads, prob.d_k, prob.d_v, prob.num_views, prob.block_size,
+                        gb._dtype_code(prob.q))
+    ws = gb.Workspace(gb.backward_workspace_size(desc, prob.doc_offsets), device=dev).tensor
+    names = ("q", "k", "v", "g", "beta", "qn", "kn", "vn", "gn", "betan")
+    ins = [getattr(prob, n) for n in names]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(inputs=None, d_o=None, d_on=None):
+        return gb.backward(*(inputs or ins), prob.doc_offsets, prob.prompt_len, prob.block_size,
+                           do if d_o is None else d_o, don if d_on is None else d_on, None, workspace=ws)
+
+    steps = max(1, args.steps)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with ClockSampler(local) as clocks:
+        replicas.barrier(world)
+        torch.cuda.synchronize()
+        clocks.mark_start()
+        for i in range(steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        clocks.poll_until(evs[-1][1])
+        torch.cuda.synchronize()
+        clocks.mark_stop()
+        replicas.barrier(world)
+    ms = replicas.max_over_ranks(float(np.mean([a.elapsed_time(z) for a, z in evs])), world, device=dev)
+    nbytes = backward_bytes(prob)
+    peaks = measured_peaks()
+    gbps = nbytes / (ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": gbps, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbps / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
+                "kernel": "gdn_backward_kernel", "algorithmic_bytes": nbytes}
+    toks = prob.tokens() * world
+    value = toks / (ms / 1e3)
+    e2e = None
+    if not args.no_e2e:
+        host = {n: getattr(prob, n).cpu().pin_memory() for n in names}
+        h_do, h_don = do.cpu().pin_memory(), don.cpu().pin_memory()
+        dbuf = {n: torch.empty_like(getattr(prob, n)) for n in names}
+        d_do, d_don = torch.empty_like(do), torch.empty_like(don)
+        outs_h = None
+
+        def e2e_step():
+            nonlocal outs_h
+            for n in names:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            d_do.copy_(h_do, non_blocking=True)
+            d_don.copy_(h_don, non_blocking=True)
+            gr = step([dbuf[n] for n in names], d_do, d_don)
+            if outs_h is None:
+                outs_h = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in gr.items()}
+            for k, v in gr.items():
+                outs_h[k].copy_(v, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ns = 3
+        a.record(stream)
+        for _ in range(ns):
+            e2e_step()
+        z.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = replicas.max_over_ranks(a.elapsed_time(z) / ns, world, device=dev)
+        e2e = {"value": toks / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host.values())
+                                         + h_do.numel() * h_do.element_size() + h_don.numel() * h_don.element_size()),
+               "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs_h.values())),
+               "ms_per_step": e2e_ms, "steps": ns}
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = time_backward_oracle(synth.make_problem(wl, seed=0, device="cpu"))
+        cpu_baseline = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    replicas.shutdown(world)
+    if rank != 0:
+        return
+    line = {"metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 I/O, fp32 arithmetic and gradients", "data": "synthetic",
+            "config": {"workload": name, "layout": BWD_WORKLOADS[name], "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2"},
+            "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
+            "gpu_launches": steps, "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- our arm
 def main():
     ap = argparse.ArgumentParser()
@@ -633,6 +797,9 @@ def main():
         return
     if args.workload in synth.ATTN_WORKLOADS:
         run_attention(args, args.workload, rank, world, local)
+        return
+    if args.workload in BWD_WORKLOADS:
+        run_backward(args, args.workload, rank, world, local)
         return
     wl = synth.get_workload(args.workload)
 
