@@ -97,9 +97,10 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
     auto reduce_add = [&](float *out_vec, float *sc0, float *sc1) {
         __syncthreads();
         for (int r = tid; r < D + 2; r += kBwdThreads) {
-            float acc = 0.f;
-#pragma unroll 8
-            for (int cc = 0; cc < 32; ++cc) acc += red[cc * (D + 2) + r];
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};         // four independent chains
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) a4[cc & 3] += red[cc * (D + 2) + r];
+            const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
             if (r < D) {
                 if (out_vec) atomicAdd(out_vec + r, acc);
             } else if (r == D) {
