@@ -78,11 +78,34 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
     const float sc = P.scale;
     auto at = [&](float *buf, int i) -> float & { return buf[i * kBwdThreads + tid]; };
 
-    // token data of clean row t (or noisy packed row when noisy): k and q rows of this thread
+    // this thread's rows of a k or q vector (clean row, or noisy packed row), as 16-byte loads
+    // (the rows start 32-byte aligned: D >= 32 and the tensors are 16-byte aligned)
     auto kq = [&](const void *base, int64_t row, float (&x)[R2]) {
         const int64_t o = (row * H + h) * D + rb;
+        if constexpr (sizeof(TIO) == 4) {
+            const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + o);
 #pragma unroll
-        for (int i = 0; i < R2; ++i) x[i] = ld<TIO>(base, o + i);
+            for (int i = 0; i < R2 / 4; ++i) {
+                const float4 f = __ldg(p + i);
+                x[4 * i] = f.x;
+                x[4 * i + 1] = f.y;
+                x[4 * i + 2] = f.z;
+                x[4 * i + 3] = f.w;
+            }
+        } else {
+            const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(base) + o);
+#pragma unroll
+            for (int i = 0; i < R2 / 8; ++i) {
+                const uint4 u = __ldg(p + i);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
+                    x[8 * i + 2 * j] = f.x;
+                    x[8 * i + 2 * j + 1] = f.y;
+                }
+            }
+        }
     };
     // one forward step of this thread's half column
     auto fwd = [&](float (&st)[R2], const float (&kk)[R2], float vc, float a, float b) {
