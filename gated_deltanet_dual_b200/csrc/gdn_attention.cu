@@ -16,8 +16,10 @@
 //
 // 128 threads, 96 KB of shared memory (Q, K, V tiles) and 256 TMEM columns per CTA, so two CTAs
 // share an SM and one's softmax overlaps the other's MMAs.  K of the next key tile is loaded as
-// soon as S is computed, V as soon as P V is.  Work items are sorted on the host by their number
-// of key tiles, heaviest first.  Every mbarrier wait is bounded; a wait that gives up records
+// soon as S is computed, V as soon as P V is.  Each CTA derives its (document, head, query tile)
+// from its index and per-document prefix tables in the parameter block: documents longest first,
+// then heads, then the document's query tiles, so the CTAs that run together read the same key /
+// value tiles through L2.  Every mbarrier wait is bounded; a wait that gives up records
 // GDN_ERR_TIMEOUT in the workspace and the CTA leaves its loop.
 #include <algorithm>
 #include <cmath>
@@ -52,12 +54,14 @@ struct AttnParams {
     int32_t H, Hkv, V, B;
     int64_t TR;
     float scale_log2;                       // log2(e) / sqrt(d)
-    const int32_t *items;                   // work list: (tile << 13 | kind << 11 | doc, head) pairs
     WorkspaceHeader *ws;
     void *out, *out_noisy;
+    int32_t N;
     int32_t doc_start[kMaxDocs + 1];
     int32_t doc_prompt[kMaxDocs];
     int32_t resp_off[kMaxDocs + 1];
+    int32_t doc_order[kMaxDocs];            // documents, longest first
+    int32_t item_off[kMaxDocs + 1];         // first CTA of each document in that order
 };
 
 struct AttnMaps {
@@ -85,11 +89,30 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int item = P.items[2 * blockIdx.x];
-    const int h = P.items[2 * blockIdx.x + 1];
-    const int hk = h / (P.H / P.Hkv);
-    const int n = item & 2047, kind = (item >> 11) & 3, tile = item >> 13;
+    // Work item of this CTA: documents longest first; per document, every head in turn; per
+    // (document, head) every query tile, clean tiles from the last, then each view's noisy tiles
+    // from the last.  The CTAs that run together thus share the (document, head)'s key/value tiles.
+    int lo_k = 0, hi_k = P.N;                          // largest k with item_off[k] <= blockIdx.x
+    while (hi_k - lo_k > 1) {
+        const int mid = (lo_k + hi_k) >> 1;
+        if (P.item_off[mid] <= (int)blockIdx.x) lo_k = mid;
+        else hi_k = mid;
+    }
+    const int n = P.doc_order[lo_k];
     const int s = P.doc_start[n], len = P.doc_start[n + 1] - s, Pn = P.doc_prompt[n], R = len - Pn;
+    const int nct = (len + AT - 1) / AT, nnt = (R + AT - 1) / AT;
+    const int ntile = nct + P.V * nnt;
+    const int local = (int)blockIdx.x - P.item_off[lo_k];
+    const int h = local / ntile, jt = local % ntile;
+    int kind, tile;
+    if (jt < nct) {
+        kind = 0;
+        tile = nct - 1 - jt;
+    } else {
+        kind = 1 + (jt - nct) / nnt;
+        tile = nnt - 1 - (jt - nct) % nnt;
+    }
+    const int hk = h / (P.H / P.Hkv);
     const int B = P.B;
     const int w = kind - 1;                                   // noisy view (kind > 0)
     const int64_t nrow0 = (int64_t)w * P.TR + P.resp_off[n] + (int64_t)AT * tile;   // noisy tile rows
@@ -331,10 +354,9 @@ bool attn_desc_supported(const gdn_attn_desc *d) {
            d->num_heads % d->num_kv_heads == 0 && d->num_docs <= kMaxDocs;
 }
 
-// Layout check; fills the work list (heaviest first) when `items` is given.  Returns false on an
-// invalid layout.
-bool attn_layout(const gdn_attn_desc *d, const int32_t *offs, const int32_t *pl, int64_t *T, int64_t *TR,
-                 std::vector<int32_t> *items) {
+// Layout check: documents from offset 0, non-decreasing, prompts inside them, responses in
+// whole blocks.
+bool attn_layout(const gdn_attn_desc *d, const int32_t *offs, const int32_t *pl, int64_t *T, int64_t *TR) {
     if (!offs || !pl || offs[0] != 0) return false;
     const int N = d->num_docs, B = d->block_size;
     int64_t tr = 0;
@@ -346,41 +368,9 @@ bool attn_layout(const gdn_attn_desc *d, const int32_t *offs, const int32_t *pl,
     if (tr > INT32_MAX || offs[N] > INT32_MAX) return false;
     *T = offs[N];
     *TR = tr;
-    if (items) {
-        // (document, head) groups, longest documents first; inside a group every query tile of the
-        // document (clean and noisy, heaviest first), so the CTAs that run together read the same
-        // key / value tiles through L2.  Heads that share a key/value head are adjacent.
-        for (int n = 0; n < N; ++n)       // tile index must fit 18 bits
-            if ((int64_t)offs[n + 1] - offs[n] > ((int64_t)1 << 18) * AT) return false;
-        const int V = tr > 0 ? d->num_views : 0;
-        std::vector<int> order(N);
-        std::iota(order.begin(), order.end(), 0);
-        std::stable_sort(order.begin(), order.end(),
-                         [&](int a, int b) { return offs[a + 1] - offs[a] > offs[b + 1] - offs[b]; });
-        items->clear();
-        std::vector<std::pair<int64_t, int32_t>> tiles;
-        for (int n : order) {
-            const int64_t len = (int64_t)offs[n + 1] - offs[n], P = pl[n], R = len - P;
-            tiles.clear();
-            for (int64_t t = 0; t * AT < len; ++t) tiles.push_back({t + 1, (int32_t)((t << 13) | n)});
-            for (int v = 0; v < V; ++v)
-                for (int64_t t = 0; t * AT < R; ++t) {
-                    const int64_t ilast = std::min<int64_t>(AT * t + AT - 1, R - 1);
-                    const int64_t cost = (P + (ilast / B) * B + AT - 1) / AT + 1;
-                    tiles.push_back({cost, (int32_t)((t << 13) | ((v + 1) << 11) | n)});
-                }
-            std::stable_sort(tiles.begin(), tiles.end(), [](const auto &a, const auto &b) { return a.first > b.first; });
-            for (int h = 0; h < d->num_heads; ++h)
-                for (const auto &t : tiles) {
-                    items->push_back(t.second);
-                    items->push_back(h);
-                }
-        }
-    }
     return true;
 }
 
-size_t attn_items_offset() { return sizeof(WorkspaceHeader); }
 
 }  // namespace
 }  // namespace gdn
@@ -391,9 +381,8 @@ extern "C" size_t gdn_attn_workspace_size(const gdn_attn_desc *desc, const int32
                                           const int32_t *prompt_len_host) {
     if (!attn_desc_ok(desc)) return 0;
     int64_t T = 0, TR = 0;
-    std::vector<int32_t> items;
-    if (!attn_layout(desc, doc_offsets_host, prompt_len_host, &T, &TR, &items)) return 0;
-    return attn_items_offset() + ((items.size() * sizeof(int32_t) + 255) / 256) * 256;
+    if (!attn_layout(desc, doc_offsets_host, prompt_len_host, &T, &TR)) return 0;
+    return sizeof(WorkspaceHeader);
 }
 
 extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q, const void *k, const void *v,
@@ -403,18 +392,15 @@ extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q,
                                        gdn_stream_t stream) {
     if (!attn_desc_ok(desc)) return GDN_ERR_INVALID_ARG;
     int64_t T = 0, TR = 0;
-    std::vector<int32_t> items;
-    if (!attn_layout(desc, doc_offsets, prompt_len, &T, &TR, &items)) return GDN_ERR_INVALID_ARG;
+    if (!attn_layout(desc, doc_offsets, prompt_len, &T, &TR)) return GDN_ERR_INVALID_ARG;
     const int V = TR > 0 ? desc->num_views : 0;
     if (T > 0 && (!q || !k || !v || !out)) return GDN_ERR_INVALID_ARG;
     if (V > 0 && (!qn || !kn || !vn || !out_noisy)) return GDN_ERR_INVALID_ARG;
-    const size_t need = attn_items_offset() + ((items.size() * sizeof(int32_t) + 255) / 256) * 256;
-    if (!workspace || workspace_bytes < need) return GDN_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < sizeof(WorkspaceHeader)) return GDN_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, qn, kn, vn, out, out_noisy, workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
     if (!attn_desc_supported(desc)) return GDN_ERR_UNSUPPORTED;
-    if (items.empty()) return GDN_OK;
 
     AttnParams P;
     std::memset(&P, 0, sizeof(P));
@@ -425,18 +411,36 @@ extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q,
     P.TR = TR;
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)desc->head_dim));
     P.ws = static_cast<WorkspaceHeader *>(workspace);
-    P.items = reinterpret_cast<const int32_t *>(static_cast<uint8_t *>(workspace) + attn_items_offset());
     P.out = out;
     P.out_noisy = out_noisy;
+    const int N = desc->num_docs;
+    P.N = N;
     int64_t roff = 0;
-    for (int n = 0; n <= desc->num_docs; ++n) {
+    for (int n = 0; n <= N; ++n) {
         P.doc_start[n] = doc_offsets[n];
         P.resp_off[n] = (int32_t)roff;
-        if (n < desc->num_docs) {
+        if (n < N) {
             P.doc_prompt[n] = prompt_len[n];
             roff += (int64_t)doc_offsets[n + 1] - doc_offsets[n] - prompt_len[n];
         }
     }
+    // documents longest first; each takes H x (its query tiles) CTAs
+    std::vector<int> order(N);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+        return doc_offsets[a + 1] - doc_offsets[a] > doc_offsets[b + 1] - doc_offsets[b];
+    });
+    int64_t items = 0;
+    for (int k = 0; k < N; ++k) {
+        const int n = order[k];
+        const int64_t len = (int64_t)doc_offsets[n + 1] - doc_offsets[n], R = len - prompt_len[n];
+        P.doc_order[k] = n;
+        P.item_off[k] = (int32_t)std::min<int64_t>(items, INT32_MAX);
+        items += (int64_t)desc->num_heads * ((len + AT - 1) / AT + (int64_t)V * ((R + AT - 1) / AT));
+    }
+    P.item_off[N] = (int32_t)std::min<int64_t>(items, INT32_MAX);
+    if (items > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+    if (items == 0) return GDN_OK;
     AttnMaps maps;
     const int H = desc->num_heads, Hkv = desc->num_kv_heads;
     if (!attn_map(&maps.q, q, H, T) || !attn_map(&maps.k, k, Hkv, T) || !attn_map(&maps.v, v, Hkv, T))
@@ -458,11 +462,6 @@ extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q,
     if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), st) != cudaSuccess) return GDN_ERR_CUDA;
-    if (cudaMemcpyAsync(static_cast<uint8_t *>(workspace) + attn_items_offset(), items.data(),
-                        items.size() * sizeof(int32_t), cudaMemcpyHostToDevice, st) != cudaSuccess)
-        return GDN_ERR_CUDA;
-    const int64_t grid = (int64_t)items.size() / 2;
-    if (grid > INT32_MAX) return GDN_ERR_UNSUPPORTED;
-    gdn_attention_kernel<<<(unsigned)grid, kAThreads, A_SMEM, st>>>(P, maps);
+    gdn_attention_kernel<<<(unsigned)items, kAThreads, A_SMEM, st>>>(P, maps);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -22,8 +22,9 @@
  *   kn, vn        [V, T_R, H_kv, d]   order), the layout of gdn_dual_forward's noisy twins
  *   doc_offsets   [N+1] int32, HOST   doc_offsets[0] = 0, non-decreasing, T = doc_offsets[N]
  *   prompt_len    [N] int32, HOST     0 <= P_n <= len_n, (len_n - P_n) % B == 0
- *   workspace     device, >= gdn_attn_workspace_size(...) bytes, 16-byte aligned; holds the
- *                 call's work list (written on `stream`), so calls sharing it race.
+ *   workspace     device, >= gdn_attn_workspace_size(...) bytes (256), 16-byte aligned: the
+ *                 device status word (GDN_ERR_TIMEOUT if a bounded wait gave up; read it with
+ *                 gdn_dual_read_device_status), cleared on `stream` by each call.
  *
  * gdn_attn_forward validates on the host (no partial launch on error), enqueues on `stream`
  * and returns; nothing is allocated and nothing synchronises.  Errors: GDN_ERR_INVALID_ARG
