@@ -23,10 +23,8 @@
 //           is rebuilt from that token's state (token by token, from the start for every step)
 //           and run backwards, and its initial-state gradient joins Lam.
 // The work per token is a few dot products of length d per column: CUDA cores, not tensor cores.
-#include <algorithm>
 #include <cmath>
 #include <cstring>
-#include <vector>
 
 #include "gdn_internal.cuh"
 
@@ -56,7 +54,7 @@ __device__ __forceinline__ float ld(const void *p, int64_t i) {
     return to_f32(static_cast<const T *>(p)[i]);
 }
 
-template <int R2>
+// the two threads of a column (adjacent lanes) hold its two row halves
 __device__ __forceinline__ float pair_sum(float x) {
     return x + __shfl_xor_sync(0xffffffffu, x, 1);
 }
@@ -112,7 +110,7 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
         float ks = 0.f;
 #pragma unroll
         for (int i = 0; i < R2; ++i) ks = fmaf(kk[i], st[i], ks);
-        ks = pair_sum<R2>(ks);
+        ks = pair_sum(ks);
 #pragma unroll
         for (int i = 0; i < R2; ++i) st[i] = a * fmaf(-b * ks, kk[i], st[i]) + b * kk[i] * vc;
     };
@@ -145,8 +143,8 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
             ks = fmaf(kk[i], sp[i], ks);
             ls = fmaf(lam[i], sp[i], ls);
         }
-        kl = pair_sum<R2>(kl);
-        ks = pair_sum<R2>(ks);
+        kl = pair_sum(kl);
+        ks = pair_sum(ks);
         float *rr = red + c * (D + 2);
 #pragma unroll
         for (int i = 0; i < R2; ++i) rr[rb + i] = b * vc * lam[i] - a * b * (ks * lam[i] + kl * sp[i]);
