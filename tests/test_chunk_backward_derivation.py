@@ -1,0 +1,56 @@
+"""The chunked (WY / UT) backward of the clean stream (tests/chunk_backward_reference.py, the
+derivation a tensor-core backward would use) against the token-by-token fp64 backward oracle."""
+import numpy as np
+import pytest
+
+from oracle import backward as ob
+import chunk_backward_reference as cbr
+
+
+@pytest.mark.parametrize("C", [16, 64])
+@pytest.mark.parametrize("lens", [[150, 70], [64, 1, 129]])
+def test_chunked_clean_backward_matches_the_oracle(C, lens):
+    rng = np.random.default_rng(C + len(lens))
+    H, d = 2, 8
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(offs[-1])
+    unit = lambda a: a / np.linalg.norm(a, axis=-1, keepdims=True)
+    q, k = unit(rng.standard_normal((T, H, d))), unit(rng.standard_normal((T, H, d)))
+    v = rng.standard_normal((T, H, d))
+    g = -0.5 * rng.random((T, H))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((T, H))))
+    do = rng.standard_normal((T, H, d))
+    dsf = rng.standard_normal((len(lens), H, d, d))
+    prompts = np.asarray(lens, np.int32)                     # no response: clean stream only
+    e = np.zeros((0, 0, H, d))
+    e1 = np.zeros((0, 0, H))
+    ref = ob.dual_backward(q, k, v, g, beta, e, e, e, e1, e1, offs, prompts, 1, do, e, dsf)
+    got = cbr.clean_backward_chunked(q, k, v, g, beta, offs, do, dsf, C=C)
+    for name in ("dq", "dk", "dv", "dg", "dbeta"):
+        r = ref[name]
+        assert np.abs(got[name] - r).max() <= 1e-10 * max(np.abs(r).max(), 1.0), name
+
+
+@pytest.mark.parametrize("C,B", [(16, 4), (64, 4), (64, 16), (16, 1)])
+def test_chunked_dual_backward_matches_the_oracle(C, B):
+    """Both streams: the noisy blocks' initial-state gradients enter the chunk backward at their
+    boundary states (prompts not on the chunk grid, an empty prompt, two views)."""
+    rng = np.random.default_rng(C + B)
+    H, d, V = 2, 6, 2
+    R = lambda x: (x // B) * B
+    lens = [21 + R(80), R(48), 13 + R(16)]
+    prompts = [21, 0, 13]
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, TR = int(offs[-1]), int(sum(lens) - sum(prompts))
+    unit = lambda a: a / np.linalg.norm(a, axis=-1, keepdims=True)
+    x = lambda *sh: rng.standard_normal(sh)
+    ins = dict(q=unit(x(T, H, d)), k=unit(x(T, H, d)), v=x(T, H, d), g=-0.4 * rng.random((T, H)),
+               beta=1 / (1 + np.exp(-x(T, H))), qn=unit(x(V, TR, H, d)), kn=unit(x(V, TR, H, d)),
+               vn=x(V, TR, H, d), gn=-0.4 * rng.random((V, TR, H)), betan=1 / (1 + np.exp(-x(V, TR, H))))
+    order = ("q", "k", "v", "g", "beta", "qn", "kn", "vn", "gn", "betan")
+    do, don, dsf = x(T, H, d), x(V, TR, H, d), x(len(lens), H, d, d)
+    ref = ob.dual_backward(*(ins[n] for n in order), offs, prompts, B, do, don, dsf)
+    got = cbr.dual_backward_chunked(*(ins[n] for n in order), offs, prompts, B, do, don, dsf, C=C)
+    for name in ref:
+        r = ref[name]
+        assert np.abs(got[name] - r).max() <= 1e-10 * max(np.abs(r).max(), 1.0), name
