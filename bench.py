@@ -618,7 +618,7 @@ def run_attention(args, name, rank, world, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": name, "layout": cfg["layout"], "heads": H, "kv_heads": int(pr.k.shape[1]), "d": d,
                        "block": pr.block_size, "views": V, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 are not guaranteed (K/V reuse through L2 is part of the kernel)"},
+                       "l2": f"inputs larger than L2 ({sum(t.numel() * t.element_size() for t in (pr.q, pr.k, pr.v, pr.qn, pr.kn, pr.vn)) / 1e9:.2f} GB; K/V reuse inside a call goes through L2)"},
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
