@@ -29,6 +29,21 @@ from __future__ import annotations
 
 import numpy as np
 
+# Operand rounding of the matrix products (identity: exact fp64).  The precision study sets it
+# to bf16 rounding to emulate tensor-core products with bf16 operands and wide accumulation.
+_ROUND = None
+
+
+def set_operand_rounding(fn):
+    global _ROUND
+    _ROUND = fn
+
+
+def mm(a, b):
+    if _ROUND is not None:
+        a, b = _ROUND(a), _ROUND(b)
+    return a @ b
+
 
 def clean_backward_chunked(q, k, v, g, beta, doc_offsets, d_out, d_final_state, C=64):
     """Clean-stream gradients (dq, dk, dv, dg, dbeta) by chunks of C tokens from each document
@@ -69,17 +84,17 @@ def _chunk_forward(Q, K, V, g, beta, S0, s):
     lower = np.tril(np.ones((L, L))) > 0
     strict = np.tril(np.ones((L, L)), -1) > 0
     D = np.where(lower, np.exp(np.where(lower, gam[:, None] - gam[None, :], 0.0)), 0.0)
-    KK = K @ K.T
+    KK = mm(K, K.T)
     A = np.where(strict, beta[:, None] * D * KK, 0.0)
     Tm = np.linalg.inv(np.eye(L) + A)
-    KS0 = K @ S0
+    KS0 = mm(K, S0)
     R = beta[:, None] * V - (beta * Gam)[:, None] * KS0
-    U = Tm @ R
-    M = (Q @ K.T) * D
+    U = mm(Tm, R)
+    M = mm(Q, K.T) * D
     ec = np.exp(gam[-1] - gam)                    # e^{gamma_C - gamma_i}
     Khat = ec[:, None] * K
-    O = s * (Gam[:, None] * (Q @ S0) + M @ U)
-    SC = Gam[-1] * S0 + Khat.T @ U
+    O = s * (Gam[:, None] * mm(Q, S0) + mm(M, U))
+    SC = Gam[-1] * S0 + mm(Khat.T, U)
     return dict(Q=Q, K=K, V=V, beta=beta, S0=S0, gam=gam, Gam=Gam, lower=lower, strict=strict, D=D, KK=KK,
                 A=A, Tm=Tm, KS0=KS0, R=R, U=U, M=M, ec=ec, Khat=Khat, O=O, SC=SC)
 
@@ -89,7 +104,7 @@ def chunk_state(f, e):
     if e < 0:
         return f["S0"].copy()
     w = np.exp(f["gam"][e] - f["gam"][:e + 1])
-    return f["Gam"][e] * f["S0"] + (w[:, None] * f["K"][:e + 1]).T @ f["U"][:e + 1]
+    return f["Gam"][e] * f["S0"] + mm((w[:, None] * f["K"][:e + 1]).T, f["U"][:e + 1])
 
 
 def _chunk_backward(f, dO, dSC, s, inject=()):
@@ -99,7 +114,7 @@ def _chunk_backward(f, dO, dSC, s, inject=()):
     Gam, D, KK, Tm, U, R, M, ec, Khat = f["Gam"], f["D"], f["KK"], f["Tm"], f["U"], f["R"], f["M"], f["ec"], f["Khat"]
     strict, lower, KS0, gam = f["strict"], f["lower"], f["KS0"], f["gam"]
     L = Q.shape[0]
-    dU = s * M.T @ dO + Khat @ dSC
+    dU = s * mm(M.T, dO) + mm(Khat, dSC)
     dS0_inj = np.zeros_like(S0)
     dK_inj = np.zeros_like(K)
     dgam_inj = np.zeros(L)
@@ -109,20 +124,20 @@ def _chunk_backward(f, dO, dSC, s, inject=()):
             continue
         w = np.exp(gam[e] - gam[:e + 1])                       # e^{gamma_e - gamma_i}, i <= e
         dS0_inj += Gam[e] * lam_e
-        dU[:e + 1] += w[:, None] * (K[:e + 1] @ lam_e)
-        dK_inj[:e + 1] += w[:, None] * (U[:e + 1] @ lam_e.T)
+        dU[:e + 1] += w[:, None] * mm(K[:e + 1], lam_e)
+        dK_inj[:e + 1] += w[:, None] * mm(U[:e + 1], lam_e.T)
         t = w * np.sum((K[:e + 1] @ lam_e) * U[:e + 1], axis=1)
         dgam_inj[e] += Gam[e] * np.sum(lam_e * S0) + t.sum()
         dgam_inj[:e + 1] -= t
-    dR = Tm.T @ dU
-    dA = np.where(strict, -(dR @ U.T), 0.0)
-    dS0 = Gam[-1] * dSC + s * Q.T @ (Gam[:, None] * dO) - K.T @ ((beta * Gam)[:, None] * dR) + dS0_inj
+    dR = mm(Tm.T, dU)
+    dA = np.where(strict, -mm(dR, U.T), 0.0)
+    dS0 = Gam[-1] * dSC + s * mm(Q.T, Gam[:, None] * dO) - mm(K.T, (beta * Gam)[:, None] * dR) + dS0_inj
     dV = beta[:, None] * dR
-    dM = s * dO @ U.T
+    dM = s * mm(dO, U.T)
     dMD = np.where(lower, dM * D, 0.0)
-    dQ = s * Gam[:, None] * (dO @ S0.T) + dMD @ K
+    dQ = s * Gam[:, None] * mm(dO, S0.T) + mm(dMD, K)
     G = np.where(strict, dA * beta[:, None] * D, 0.0)
-    dK = dMD.T @ Q + ec[:, None] * (U @ dSC.T) - (beta * Gam)[:, None] * (dR @ S0.T) + G @ K + G.T @ K + dK_inj
+    dK = mm(dMD.T, Q) + ec[:, None] * mm(U, dSC.T) - (beta * Gam)[:, None] * mm(dR, S0.T) + mm(G, K) + mm(G.T, K) + dK_inj
     dbeta = np.sum(dR * V, axis=1) - Gam * np.sum(dR * KS0, axis=1) + np.sum(np.where(strict, dA * D * KK, 0.0), axis=1)
     # d gamma: through Gamma_t (O and R), Gamma_C (S_C), and the pairwise decays e^{gamma_t-gamma_i}
     dgam = Gam * (s * np.sum(dO * (Q @ S0), axis=1) - beta * np.sum(dR * KS0, axis=1))
