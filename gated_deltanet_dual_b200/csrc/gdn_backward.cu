@@ -326,7 +326,7 @@ int64_t bwd_checkpoints(const gdn_dual_desc *d, const int32_t *offs) {
 }
 
 bool bwd_desc_ok(const gdn_dual_desc *d) {
-    return d && d->num_docs >= 1 && d->num_docs <= kMaxDocs && d->num_heads >= 1 && d->d_k >= 1 && d->d_v >= 1 &&
+    return d && d->num_docs >= 1 && d->num_heads >= 1 && d->d_k >= 1 && d->d_v >= 1 &&
            d->num_views >= 0 && d->block_size >= 1 && (d->dtype == GDN_BF16 || d->dtype == GDN_FP32) &&
            d->conv_width >= 0 && d->reserved == 0;
 }
@@ -374,7 +374,7 @@ extern "C" gdn_status gdn_dual_backward(const gdn_dual_desc *desc, const void *q
                           dq, dk, dv, dg, dbeta, dqn, dkn, dvn, dgn, dbetan, workspace};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
-    if (desc->d_k != desc->d_v || (D != 32 && D != 64 && D != 128) || desc->conv_width != 0)
+    if (desc->d_k != desc->d_v || (D != 32 && D != 64 && D != 128) || desc->conv_width != 0 || N > kMaxDocs)
         return GDN_ERR_UNSUPPORTED;
     if (T == 0) return GDN_OK;
 

@@ -359,3 +359,19 @@ def test_backward_host_validation():
     d48 = b.make_desc(2, 2, 48, 48, 2, 4, b.GDN_FP32)
     assert call(d48) == b.GDN_ERR_UNSUPPORTED
     assert call(d) == b.GDN_ERR_CUDA                                         # valid; no device here
+
+
+@no_gpu
+def test_backward_more_documents_than_supported():
+    lib = b.load_library()
+    N = 1025
+    offs = np.arange(N + 1, dtype=np.int32) * 4
+    pl = np.zeros(N, np.int32)
+    d = b.make_desc(N, 1, 32, 32, 1, 4, b.GDN_FP32)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    ptr = [ctypes.c_void_p(0x7f0000000000 + 0x10000000 * i) for i in range(24)]
+    nb = b.backward_workspace_size(d, offs)
+    assert nb > 0
+    st = lib.gdn_dual_backward(ctypes.byref(d), *ptr[:10], offs.ctypes.data_as(ip), pl.ctypes.data_as(ip),
+                               *ptr[10:23], ptr[23], ctypes.c_size_t(nb), None)
+    assert st == b.GDN_ERR_UNSUPPORTED
