@@ -54,3 +54,33 @@ def test_chunked_dual_backward_matches_the_oracle(C, B):
     for name in ref:
         r = ref[name]
         assert np.abs(got[name] - r).max() <= 1e-10 * max(np.abs(r).max(), 1.0), name
+
+
+def test_noisy_injection_is_rank_B_in_carried_back_queries():
+    """A block's initial-state gradient sum_l (A~_1^T ... A~_B^T q~_l) do~_l^T / sqrt(d): the
+    block's queries carried back through its steps (B rows per view) times their upstream
+    gradients, so a kernel can inject it as extra read-out rows instead of a d x d matrix."""
+    rng = np.random.default_rng(3)
+    d, B = 6, 4
+    unit = lambda a: a / np.linalg.norm(a)
+    kn = [unit(rng.standard_normal(d)) for _ in range(B)]
+    qn = [unit(rng.standard_normal(d)) for _ in range(B)]
+    gn = -0.3 * rng.random(B)
+    bn = 1 / (1 + np.exp(-rng.standard_normal(B)))
+    don = [rng.standard_normal(d) for _ in range(B)]
+    s = 1 / np.sqrt(d)
+    A = [np.exp(gn[i]) * (np.eye(d) - bn[i] * np.outer(kn[i], kn[i])) for i in range(B)]
+    # the adjoint written out: Lam_B = sum_l q_l do_l^T s, Lam_{i-1} = A_i^T Lam_i
+    lam = sum(np.outer(qn[l], don[l]) for l in range(B)) * s
+    for i in range(B - 1, -1, -1):
+        lam = A[i].T @ lam
+    # rank-B form: x_l = A_1^T ... A_B^T q_l s
+    xs = []
+    for l in range(B):
+        x = qn[l] * s
+        for i in range(B - 1, -1, -1):
+            x = A[i].T @ x
+        xs.append(x)
+    lam_rank = sum(np.outer(xs[l], don[l]) for l in range(B))
+    np.testing.assert_allclose(lam_rank, lam, rtol=1e-12, atol=1e-14)
+    assert np.linalg.matrix_rank(lam) <= B
