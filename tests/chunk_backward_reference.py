@@ -107,9 +107,12 @@ def chunk_state(f, e):
     return f["Gam"][e] * f["S0"] + mm((w[:, None] * f["K"][:e + 1]).T, f["U"][:e + 1])
 
 
-def _chunk_backward(f, dO, dSC, s, inject=()):
+def _chunk_backward(f, dO, dSC, s, inject=(), rows=None):
     """inject: (e, Lam_e) pairs, gradients dL/dS_e of block-boundary states inside the chunk
-    (the views' initial-state gradients of the noisy block starting after token e)."""
+    (the views' initial-state gradients of the noisy block starting after token e).
+    rows: the same injections in rank-B form, (X, dOx, e) with X [n, d_k] the carried-back
+    queries, dOx [n, d_v] their upstream gradients and e [n] their boundary rows: each row reads
+    S_e^T x like an output row with its decay boundary at e, as the forward's Z rows do."""
     Q, K, V, beta, S0 = f["Q"], f["K"], f["V"], f["beta"], f["S0"]
     Gam, D, KK, Tm, U, R, M, ec, Khat = f["Gam"], f["D"], f["KK"], f["Tm"], f["U"], f["R"], f["M"], f["ec"], f["Khat"]
     strict, lower, KS0, gam = f["strict"], f["lower"], f["KS0"], f["gam"]
@@ -118,6 +121,23 @@ def _chunk_backward(f, dO, dSC, s, inject=()):
     dS0_inj = np.zeros_like(S0)
     dK_inj = np.zeros_like(K)
     dgam_inj = np.zeros(L)
+    if rows is not None and len(rows[0]):
+        X, dOx, e = rows
+        e = np.asarray(e)
+        ge = np.where(e >= 0, gam[np.maximum(e, 0)], 0.0)          # gamma at the boundary (0 for S0)
+        Ge = np.where(e >= 0, Gam[np.maximum(e, 0)], 1.0)
+        vis = np.arange(L)[None, :] <= e[:, None]                    # key i visible from boundary e
+        DX = np.where(vis, np.exp(np.where(vis, ge[:, None] - gam[None, :], 0.0)), 0.0)
+        XK = mm(X, K.T)
+        MX = XK * DX                                                 # the rows' masked X K^T (like M'_Z)
+        dS0_inj += mm(X.T, Ge[:, None] * dOx)
+        dU += mm(MX.T, dOx)
+        dMX = mm(dOx, U.T)
+        dK_inj += mm((dMX * DX).T, X)
+        W = dMX * XK * DX                                            # d(decay) terms
+        dgam_inj -= W.sum(axis=0)
+        tot = W.sum(axis=1) + Ge * np.sum(mm(X, S0) * dOx, axis=1)   # towards gamma at each boundary
+        np.add.at(dgam_inj, np.maximum(e, 0), np.where(e >= 0, tot, 0.0))
     for e, lam_e in inject:
         if e < 0:
             dS0_inj += lam_e
@@ -153,7 +173,7 @@ def _chunk_backward(f, dO, dSC, s, inject=()):
 
 
 def dual_backward_chunked(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, block_size,
-                          d_out, d_out_noisy, d_final_state, C=64):
+                          d_out, d_out_noisy, d_final_state, C=64, rank_rows=False):
     """All gradients of the dual-stream forward by chunks of C tokens anchored at each document's
     response start (C a multiple of B, so no block straddles a chunk).  Per chunk: the clean
     forward quantities, the boundary state S_e of every block starting in the chunk, each view's
@@ -196,6 +216,7 @@ def dual_backward_chunked(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, 
             for (a, b), S0 in reversed(list(zip(chunks, starts))):
                 f = _chunk_forward(q[a:b, h], k[a:b, h], v[a:b, h], g[a:b, h], beta[a:b, h], S0, s)
                 inject = []
+                rx, rdo, re_ = [], [], []                       # rank-B rows (rank_rows=True)
                 for p in range(max(a, r), b, B):                # blocks starting in this chunk
                     e = p - 1 - a
                     Se = chunk_state(f, e) if (p > s0) else np.zeros_like(S0)
@@ -217,9 +238,20 @@ def dual_backward_chunked(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, 
                             res["dgn"][w, rr + i, h] = dgg
                             res["dbetan"][w, rr + i, h] = dbb
                         total += Lt
-                    if p > s0:                                  # a document's first block starts from zero
+                        if p > s0 and rank_rows:
+                            for i in range(B):                  # x = A~_1^T ... A~_B^T q~ s
+                                xv = qn[w, rr + i, h] * s
+                                for j in range(B - 1, -1, -1):
+                                    kj = kn[w, rr + j, h]
+                                    xv = np.exp(gn[w, rr + j, h]) * (xv - betan[w, rr + j, h] * kj * (kj @ xv))
+                                rx.append(xv)
+                                rdo.append(don[w, rr + i, h])
+                                re_.append(e)
+                    if p > s0 and not rank_rows:                # a document's first block starts from zero
                         inject.append((e, total))
-                gr = _chunk_backward(f, do[a:b, h], lam, s, inject)
+                rows = (np.array(rx).reshape(-1, dk), np.array(rdo).reshape(-1, v.shape[2]),
+                        np.array(re_, dtype=np.int64)) if rank_rows else None
+                gr = _chunk_backward(f, do[a:b, h], lam, s, inject, rows)
                 for name in ("dq", "dk", "dv", "dg", "dbeta"):
                     res[name][a:b, h] = gr[name]
                 lam = gr["dS0"]

@@ -84,3 +84,26 @@ def test_noisy_injection_is_rank_B_in_carried_back_queries():
     lam_rank = sum(np.outer(xs[l], don[l]) for l in range(B))
     np.testing.assert_allclose(lam_rank, lam, rtol=1e-12, atol=1e-14)
     assert np.linalg.matrix_rank(lam) <= B
+
+
+@pytest.mark.parametrize("C,B", [(16, 4), (64, 16)])
+def test_injection_as_rank_B_rows_matches_the_matrix_form(C, B):
+    """The kernel's form of the injection: B carried-back query rows per view and block, read out
+    against the chunk like the forward's Z rows, give the same gradients as the d x d matrices."""
+    rng = np.random.default_rng(10 + B)
+    H, d, V = 1, 6, 2
+    R = lambda x: (x // B) * B
+    lens = [21 + R(80), R(48)]
+    prompts = [21, 0]
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, TR = int(offs[-1]), int(sum(lens) - sum(prompts))
+    unit = lambda a: a / np.linalg.norm(a, axis=-1, keepdims=True)
+    x = lambda *sh: rng.standard_normal(sh)
+    ins = (unit(x(T, H, d)), unit(x(T, H, d)), x(T, H, d), -0.4 * rng.random((T, H)), 1 / (1 + np.exp(-x(T, H))),
+           unit(x(V, TR, H, d)), unit(x(V, TR, H, d)), x(V, TR, H, d), -0.4 * rng.random((V, TR, H)),
+           1 / (1 + np.exp(-x(V, TR, H))))
+    do, don, dsf = x(T, H, d), x(V, TR, H, d), x(len(lens), H, d, d)
+    a = cbr.dual_backward_chunked(*ins, offs, prompts, B, do, don, dsf, C=C)
+    r = cbr.dual_backward_chunked(*ins, offs, prompts, B, do, don, dsf, C=C, rank_rows=True)
+    for name in a:
+        assert np.abs(a[name] - r[name]).max() <= 1e-11 * max(np.abs(a[name]).max(), 1.0), name
