@@ -132,3 +132,89 @@ def _noisy_block(res, S0, qn, kn, vn, gn, betan, don, r0, B, h, sc, step, step_g
             res["dbetan"][w, r, h] += dbb
         total += Lam
     return total
+
+
+def _conv_taps(L, P, B, W):
+    """Source of every tap of the width-W ShortConv (Key design 3 of the FLARE notes) for one
+    document of L tokens with prompt P: tap j of output position i reads position i - j.
+    Clean position i: the clean input at i - j, or 0 before the document.  Noisy response
+    position r (block start b0 = B floor(r / B)): the noisy input at r - j inside the block,
+    else the clean raw input at P + r - j, else 0.  Returns two lists of (out, j, kind, src)
+    with kind 'c' (clean source) or 'n' (noisy source)."""
+    clean = [(i, j, "c", i - j) for i in range(L) for j in range(W) if i - j >= 0]
+    noisy = []
+    for r in range(L - P):
+        b0 = (r // B) * B
+        for j in range(W):
+            src = r - j
+            if src >= b0:
+                noisy.append((r, j, "n", src))
+            elif P + src >= 0:
+                noisy.append((r, j, "c", P + src))
+    return clean, noisy
+
+
+def dual_backward_conv(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, block_size, conv_w,
+                       d_out, d_out_noisy, d_final_state=None):
+    """Gradients with the ShortConv prologue on q, k, v (both streams, the same weights
+    conv_w [3, H d, W], tap W-1 = the current token: x'_p = sum_j w[W-1-j] x_{p-j}).  The conv is
+    linear: apply it, differentiate the rule with respect to the convolved inputs
+    (dual_backward), then send every tap's gradient back to its source (the transposed taps; a
+    noisy output's taps before its block start feed the CLEAN raw input) and to its weight.
+    Returns dual_backward's dict plus dconv_w."""
+    q, k, v, g, beta = (_as64(x) for x in (q, k, v, g, beta))
+    qn, kn, vn, gn, betan = (_as64(x) for x in (qn, kn, vn, gn, betan))
+    w = _as64(conv_w)
+    offs = np.asarray(doc_offsets, dtype=np.int64)
+    pl = np.asarray(prompt_len, dtype=np.int64)
+    B = int(block_size)
+    T, H, d = q.shape
+    W = w.shape[-1]
+    wr = w.reshape(3, H, d, W)
+    ins = {"q": q, "k": k, "v": v}
+    noisy_in = {"q": qn, "k": kn, "v": vn}
+    conv = {n: np.zeros_like(x) for n, x in ins.items()}
+    convn = {n: np.zeros_like(x) for n, x in noisy_in.items()}
+    taps = []
+    roff = 0
+    for n in range(len(pl)):
+        s0, L, P = int(offs[n]), int(offs[n + 1] - offs[n]), int(pl[n])
+        clean, noisy = _conv_taps(L, P, B, W)
+        taps.append((s0, roff, clean, noisy))
+        for X, name in enumerate(("q", "k", "v")):
+            wx = wr[X]                                           # [H, d, W]
+            for (i, j, _, src) in clean:
+                conv[name][s0 + i] += wx[..., W - 1 - j] * ins[name][s0 + src]
+            for view in range(qn.shape[0]):
+                for (r, j, kind, src) in noisy:
+                    x_src = noisy_in[name][view, roff + src] if kind == "n" else ins[name][s0 + src]
+                    convn[name][view, roff + r] += wx[..., W - 1 - j] * x_src
+        roff += L - P
+    res = dual_backward(conv["q"], conv["k"], conv["v"], g, beta, convn["q"], convn["k"], convn["v"], gn, betan,
+                        doc_offsets, prompt_len, B, d_out, d_out_noisy, d_final_state)
+    dw = np.zeros_like(wr)
+    grads = {"q": np.zeros_like(q), "k": np.zeros_like(k), "v": np.zeros_like(v)}
+    gradsn = {"q": np.zeros_like(qn), "k": np.zeros_like(kn), "v": np.zeros_like(vn)}
+    for (s0, roff, clean, noisy) in taps:
+        for X, name in enumerate(("q", "k", "v")):
+            wx = wr[X]
+            dc = res["d" + name]                                 # gradient w.r.t. the convolved clean input
+            dn = res["d" + name + "n"]
+            for (i, j, _, src) in clean:
+                grads[name][s0 + src] += wx[..., W - 1 - j] * dc[s0 + i]
+                dw[X, ..., W - 1 - j] += ins[name][s0 + src] * dc[s0 + i]
+            for view in range(qn.shape[0]):
+                for (r, j, kind, src) in noisy:
+                    gout = dn[view, roff + r]
+                    if kind == "n":
+                        gradsn[name][view, roff + src] += wx[..., W - 1 - j] * gout
+                        dw[X, ..., W - 1 - j] += noisy_in[name][view, roff + src] * gout
+                    else:
+                        grads[name][s0 + src] += wx[..., W - 1 - j] * gout
+                        dw[X, ..., W - 1 - j] += ins[name][s0 + src] * gout
+    out = dict(res)
+    for name in ("q", "k", "v"):
+        out["d" + name] = grads[name]
+        out["d" + name + "n"] = gradsn[name]
+    out["dconv_w"] = dw.reshape(w.shape)
+    return out

@@ -86,3 +86,49 @@ def test_finite_differences_catch_planted_mistakes(name):
     mod = _mutant(*MUTANTS[name])
     with pytest.raises(AssertionError):
         fd_check(mod, [10, 8], [2, 0], 2, seed=4)
+
+
+def _conv_fd_check(mod):
+    lens, prompts, B = [10, 8], [2, 0], 2
+    inp, up, offs, pl = draw(lens, prompts, B, seed=11)
+    H, d = inp["q"].shape[1], inp["q"].shape[2]
+    w = 0.5 * np.random.default_rng(12).standard_normal((3, H * d, 4))
+
+    def loss_w(inp_, w_):
+        r = oracle.forward(*(inp_[n] for n in NAMES), offs, pl, B, conv_w=w_)
+        return (np.sum(r["out"] * up["d_out"]) + np.sum(r["out_noisy"] * up["d_out_noisy"])
+                + np.sum(r["final_state"] * up["d_final_state"]))
+
+    grads = mod.dual_backward_conv(*(inp[n] for n in NAMES), offs, pl, B, w, up["d_out"], up["d_out_noisy"],
+                                   up["d_final_state"])
+    eps = 1e-6
+    for n, x in [(n, inp[n]) for n in NAMES] + [("conv_w", w)]:
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            keep = x[i]
+            x[i] = keep + eps
+            lp = loss_w(inp, w)
+            x[i] = keep - eps
+            lm = loss_w(inp, w)
+            x[i] = keep
+            fd[i] = (lp - lm) / (2 * eps)
+        scale = max(np.abs(fd).max(), 1e-12)
+        assert np.abs(grads["d" + n] - fd).max() <= 1e-6 * scale, f"d{n}"
+
+
+def test_shortconv_mistake_is_caught():
+    """Noisy taps that cross the block start into the noisy stream (the leak the anti-leak rule
+    forbids) disagree with the finite differences."""
+    mod = _mutant("            if src >= b0:", "            if src >= 0:")
+    with pytest.raises(AssertionError):
+        _conv_fd_check(mod)
+
+
+def test_shortconv_gradients_match_finite_differences():
+    """With the width-4 ShortConv prologue: every input gradient and the weight gradient against
+    central differences of the C forward oracle (which convolves internally); with B = 2 every
+    noisy position has taps before its block start, which read (and send gradient to) the clean
+    raw input."""
+    _conv_fd_check(ob)
