@@ -173,7 +173,7 @@ def _chunk_backward(f, dO, dSC, s, inject=(), rows=None):
 
 
 def dual_backward_chunked(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, block_size,
-                          d_out, d_out_noisy, d_final_state, C=64, rank_rows=False):
+                          d_out, d_out_noisy, d_final_state, C=64, rank_rows=False, checkpoint_round=None):
     """All gradients of the dual-stream forward by chunks of C tokens anchored at each document's
     response start (C a multiple of B, so no block straddles a chunk).  Per chunk: the clean
     forward quantities, the boundary state S_e of every block starting in the chunk, each view's
@@ -210,7 +210,8 @@ def dual_backward_chunked(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, 
         for h in range(H):
             starts, S = [], np.zeros((dk, dk))
             for a, b in chunks:
-                starts.append(S.copy())
+                # the chunk-start state as the backward reads it back (checkpoint precision)
+                starts.append(S.copy() if checkpoint_round is None else checkpoint_round(S))
                 S = _chunk_forward(q[a:b, h], k[a:b, h], v[a:b, h], g[a:b, h], beta[a:b, h], S, s)["SC"]
             lam = dsf[n, h].copy()
             for (a, b), S0 in reversed(list(zip(chunks, starts))):
