@@ -1,5 +1,8 @@
 """Build the in-tree CUDA library libgdn_dual.so for sm_100a with nvcc.
 
+Every .cu file is compiled to an object of its own (in parallel, under _build/ next to the
+package), then the objects are linked into one shared library.
+
 Usage: python -m gated_deltanet_dual_b200.build [--force] [--verbose-ptxas]
 """
 from __future__ import annotations
@@ -9,20 +12,28 @@ import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
+OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdn_dual.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
+         "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def headers():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+
+
 def deps():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+    return sources() + headers()
 
 
 def needs_build() -> bool:
@@ -32,16 +43,31 @@ def needs_build() -> bool:
     return any(os.path.getmtime(f) > t for f in deps())
 
 
+def _object(src: str) -> str:
+    return os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+
+
+def _compile(src: str, force: bool, verbose_ptxas: bool) -> str:
+    obj = _object(src)
+    newest_dep = max(os.path.getmtime(f) for f in [src] + headers())
+    if not force and os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep:
+        return obj
+    tmp = obj + f".tmp{os.getpid()}"
+    cmd = [NVCC] + (["-Xptxas=-v"] if verbose_ptxas else []) + FLAGS + ["-c", "-o", tmp, src]
+    subprocess.check_call(cmd)
+    os.replace(tmp, obj)
+    return obj
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if not force and not needs_build():
         return LIB
+    os.makedirs(OBJ, exist_ok=True)
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        objs = list(ex.map(lambda s: _compile(s, force, verbose_ptxas), srcs))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-           "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
-           "-I", os.path.join(ROOT, "include"), "-o", tmp] + sources()
-    if verbose_ptxas:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.check_call(cmd)
+    subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp] + objs)
     os.replace(tmp, LIB)
     return LIB
 
