@@ -21,6 +21,24 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void *g_scratch_addr[kMaxDevices] = {};   // device address of the array, per device ordinal
 
+// Device address of the scratch array on the current device.  The first call on a device looks
+// it up (host code cannot use the symbol itself, which is only a host-side stand-in for the
+// device array) and keeps it for the life of the process: the address belongs to the device's
+// primary context, the one the CUDA runtime uses.
+gdn_status scratch_address(void **addr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" gdn_status gdn_dual_forward_noalloc(const gdn_dual_desc *desc,
@@ -33,26 +51,23 @@ extern "C" gdn_status gdn_dual_forward_noalloc(const gdn_dual_desc *desc,
                                                void *out, void *out_noisy, float *final_state,
                                                gdn_stream_t stream) {
     if (!desc || !doc_offsets) return GDN_ERR_INVALID_ARG;
+    // Route I keeps every block-boundary state in its workspace: far more than the array holds.
+    if (desc->algo == GDN_ALGO_ROUTE1) return GDN_ERR_UNSUPPORTED;
     const size_t need = gdn_dual_workspace_size(desc, doc_offsets);
     if (need == 0) return GDN_ERR_INVALID_ARG;
     if (need > kNoAllocScratchBytes) return GDN_ERR_UNSUPPORTED;   // problem needs more scratch than the array holds
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
     void *scratch = nullptr;
-    {
-        // First call on this device: look up the array's device address (host code cannot use
-        // the symbol itself, which is only a host-side stand-in for the device array).
-        std::lock_guard<std::mutex> lock(g_setup_mutex);
-        if (!g_scratch_addr[dev]) {
-            void *p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
-            g_scratch_addr[dev] = p;
-        }
-        scratch = g_scratch_addr[dev];
-    }
+    const gdn_status st = scratch_address(&scratch);
+    if (st != GDN_OK) return st;
     // gdn_dual_forward clears the status words at the start of the scratch on `stream` before
     // the launch; the rest of the array is never read before it is written.
     return gdn_dual_forward(desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, conv_w,
                             out, out_noisy, final_state, scratch, kNoAllocScratchBytes, stream);
+}
+
+extern "C" gdn_status gdn_dual_noalloc_read_device_status(gdn_stream_t stream) {
+    void *scratch = nullptr;
+    const gdn_status st = scratch_address(&scratch);
+    if (st != GDN_OK) return st;
+    return gdn_dual_read_device_status(scratch, stream);
 }
