@@ -19,12 +19,14 @@ LIB_PATH = os.path.join(_PKG, "libgdn_dual.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_ALIGNMENT, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
 GDN_BF16, GDN_FP32 = 0, 1
-ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED, ALGO_ROUTE1 = 0, 1, 2, 3
+ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED, ALGO_ROUTE1, ALGO_PIPELINED = 0, 1, 2, 3, 4
 EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device_status",
             "gdn_status_string", "gdn_dual_version", "gdn_dual_select_algo",
             "gdn_decode_replay", "gdn_decode_verify", "gdn_decode_commit", "gdn_dual_workspace_size_route1",
             "gdn_attn_forward", "gdn_attn_workspace_size", "gdn_dual_backward",
-            "gdn_dual_backward_workspace_size")
+            "gdn_dual_backward_workspace_size", "gdn_dual_forward_noalloc",
+            "gdn_dual_noalloc_read_device_status", "gdn_dual_forward_test_wait_limit",
+            "gdn_dual_read_device_status_where", "gdn_attn_forward_test_wait_limit")
 
 
 class GdnError(RuntimeError):
@@ -156,6 +158,40 @@ def forward_raw(desc: Desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets
                                     _ptr(workspace), ctypes.c_size_t(ws_bytes), ctypes.c_void_p(stream)))
 
 
+def forward_test_wait_limit_raw(desc: Desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len,
+                                conv_w, out, out_noisy, final_state, workspace, wait_iters: int, stream=None) -> int:
+    """C-ABI call of gdn_dual_forward_test_wait_limit (tests of the bounded-wait error path only:
+    every device-side wait is bounded by `wait_iters` try-waits).  Returns the status code."""
+    lib = load_library()
+    fn = lib.gdn_dual_forward_test_wait_limit
+    vp, ip = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(Desc)] + [vp] * 10 + [ip, ip] + [vp] * 5 + [ctypes.c_size_t, ctypes.c_uint32, vp]
+    offs = _host_i32(doc_offsets)
+    pl = _host_i32(prompt_len)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    ws_bytes = workspace.numel() * workspace.element_size()
+    return int(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(qn), _ptr(kn), _ptr(vn),
+                  _ptr(gn), _ptr(betan), offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(conv_w),
+                  _ptr(out), _ptr(out_noisy), _ptr(final_state), _ptr(workspace), ctypes.c_size_t(ws_bytes),
+                  ctypes.c_uint32(wait_iters), ctypes.c_void_p(stream)))
+
+
+def read_device_status_where(workspace_tensor, stream=None):
+    """(status, where): the device-side status word of a workspace and the diagnostic code of the
+    wait that gave up (0 when none did).  Synchronises the stream."""
+    lib = load_library()
+    fn = lib.gdn_dual_read_device_status_where
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]
+    where = ctypes.c_int32(0)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    st = int(fn(_ptr(workspace_tensor), ctypes.byref(where), ctypes.c_void_p(stream)))
+    return st, int(where.value)
+
+
 class Workspace:
     """Caller-owned device scratch for gdn_dual_forward (allocated by torch, reused)."""
 
@@ -264,6 +300,18 @@ def forward_noalloc_raw(desc: Desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc
     return int(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(qn), _ptr(kn), _ptr(vn),
                   _ptr(gn), _ptr(betan), offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(conv_w),
                   _ptr(out), _ptr(out_noisy), _ptr(final_state), ctypes.c_void_p(stream)))
+
+
+def noalloc_read_device_status(stream=None) -> int:
+    """C-ABI call of gdn_dual_noalloc_read_device_status: the device-side status of the last
+    gdn_dual_forward_noalloc on the current device (synchronises the stream)."""
+    lib = load_library()
+    fn = lib.gdn_dual_noalloc_read_device_status
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p]
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return int(fn(ctypes.c_void_p(stream)))
 
 
 # ----------------------------------------------------------------------------- decode side
@@ -403,6 +451,23 @@ def attention_forward(q, k, v, qn, kn, vn, doc_offsets, prompt_len, block_size, 
     if st != GDN_OK:
         raise GdnError(st, f"gdn_attn_forward failed: {status_string(st)}")
     return out, out_noisy
+
+
+def attention_forward_test_wait_limit_raw(desc, q, k, v, qn, kn, vn, doc_offsets, prompt_len, out, out_noisy,
+                                          workspace, wait_iters: int, stream=None) -> int:
+    """C-ABI call of gdn_attn_forward_test_wait_limit (tests of the bounded-wait error path only).
+    Returns the status code."""
+    lib = load_library()
+    fn = lib.gdn_attn_forward_test_wait_limit
+    vp, ip = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32)
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(AttnDesc)] + [vp] * 6 + [ip, ip] + [vp] * 3 + [ctypes.c_size_t, ctypes.c_uint32, vp]
+    offs = np.ascontiguousarray(doc_offsets, dtype=np.int32)
+    pl = np.ascontiguousarray(prompt_len, dtype=np.int32)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    return int(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(qn), _ptr(kn), _ptr(vn),
+                  offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(out), _ptr(out_noisy), _ptr(workspace),
+                  ctypes.c_size_t(ws_bytes), ctypes.c_uint32(wait_iters), _stream(stream)))
 
 
 # ----------------------------------------------------------------------------- backward

@@ -25,7 +25,7 @@ bool desc_ok(const gdn_dual_desc *d) {
     if (d->block_size < 1) return false;
     if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return false;
     if (d->conv_width < 0) return false;
-    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_ROUTE1) return false;
+    if (d->algo < GDN_ALGO_AUTO || d->algo > GDN_ALGO_PIPELINED) return false;
     if (d->reserved != 0) return false;
     return true;
 }
@@ -91,16 +91,20 @@ size_t gdn_dual_workspace_size_route1(const gdn_dual_desc *desc, const int32_t *
     return sizeof(gdn::WorkspaceHeader) + ((states + 255) / 256) * 256;
 }
 
-gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
-                            const void *q, const void *k, const void *v,
-                            const float *g, const float *beta,
-                            const void *qn, const void *kn, const void *vn,
-                            const float *gn, const float *betan,
-                            const int32_t *doc_offsets, const int32_t *prompt_len,
-                            const float *conv_w,
-                            void *out, void *out_noisy, float *final_state,
-                            void *workspace, size_t workspace_bytes,
-                            gdn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+gdn_status forward_impl(const gdn_dual_desc *desc,
+                        const void *q, const void *k, const void *v,
+                        const float *g, const float *beta,
+                        const void *qn, const void *kn, const void *vn,
+                        const float *gn, const float *betan,
+                        const int32_t *doc_offsets, const int32_t *prompt_len,
+                        const float *conv_w,
+                        void *out, void *out_noisy, float *final_state,
+                        void *workspace, size_t workspace_bytes,
+                        uint32_t wait_iters, gdn_stream_t stream) {
     if (!desc_ok(desc) || !doc_offsets || !prompt_len) return GDN_ERR_INVALID_ARG;
     const int N = desc->num_docs, H = desc->num_heads, B = desc->block_size, V = desc->num_views;
     // documents: offsets monotone from 0, prompt within the document, response aligned to B
@@ -130,8 +134,10 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
         if (p && !aligned16(p)) return GDN_ERR_ALIGNMENT;
     if (!desc_supported(desc)) return GDN_ERR_UNSUPPORTED;
     const int algo = select_algo(desc);
-    if (algo == GDN_ALGO_CHUNKED && !gdn::chunked_supported(desc->dtype, desc->d_k, B, desc->conv_width))
+    if ((algo == GDN_ALGO_CHUNKED || algo == GDN_ALGO_PIPELINED) &&
+        !gdn::chunked_supported(desc->dtype, desc->d_k, B, desc->conv_width))
         return GDN_ERR_UNSUPPORTED;
+    if (algo == GDN_ALGO_PIPELINED && desc->conv_width != 0) return GDN_ERR_UNSUPPORTED;
     if (algo == GDN_ALGO_ROUTE1 && (desc->conv_width != 0 || B > 64)) return GDN_ERR_UNSUPPORTED;
 
     gdn::Params P;
@@ -147,6 +153,8 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
     P.num_units = N * H;
     P.parts = 1;
     P.scale = (float)(1.0 / std::sqrt((double)desc->d_k));
+    P.wait_iters = wait_iters;
+    P.wait_test = wait_iters < gdn::kWaitIters ? 1u : 0u;
     int64_t roff = 0;
     for (int n = 0; n <= N; ++n) {
         P.doc_start[n] = doc_offsets[n];
@@ -167,22 +175,62 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(gdn::WorkspaceHeader), st) != cudaSuccess) return GDN_ERR_CUDA;
     cudaError_t err;
-    if (algo == GDN_ALGO_CHUNKED) err = gdn::launch_chunked(P, st);
+    if (algo == GDN_ALGO_CHUNKED || algo == GDN_ALGO_PIPELINED)
+        err = gdn::launch_chunked(P, algo == GDN_ALGO_PIPELINED, st);
     else if (algo == GDN_ALGO_ROUTE1)
         err = gdn::launch_route1(P, desc->dtype,
                                  reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader)), st);
     else err = gdn::launch_sequential(P, desc->dtype, st);
+    if (err == cudaErrorNotSupported) return GDN_ERR_UNSUPPORTED;
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
+                            const void *q, const void *k, const void *v,
+                            const float *g, const float *beta,
+                            const void *qn, const void *kn, const void *vn,
+                            const float *gn, const float *betan,
+                            const int32_t *doc_offsets, const int32_t *prompt_len,
+                            const float *conv_w,
+                            void *out, void *out_noisy, float *final_state,
+                            void *workspace, size_t workspace_bytes,
+                            gdn_stream_t stream) {
+    return forward_impl(desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, conv_w, out,
+                        out_noisy, final_state, workspace, workspace_bytes, gdn::kWaitIters, stream);
+}
+
+gdn_status gdn_dual_forward_test_wait_limit(const gdn_dual_desc *desc,
+                                            const void *q, const void *k, const void *v,
+                                            const float *g, const float *beta,
+                                            const void *qn, const void *kn, const void *vn,
+                                            const float *gn, const float *betan,
+                                            const int32_t *doc_offsets, const int32_t *prompt_len,
+                                            const float *conv_w,
+                                            void *out, void *out_noisy, float *final_state,
+                                            void *workspace, size_t workspace_bytes,
+                                            uint32_t wait_iters, gdn_stream_t stream) {
+    if (wait_iters < 1) return GDN_ERR_INVALID_ARG;
+    return forward_impl(desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, conv_w, out,
+                        out_noisy, final_state, workspace, workspace_bytes, wait_iters, stream);
+}
+
 gdn_status gdn_dual_read_device_status(const void *workspace, gdn_stream_t stream) {
+    return gdn_dual_read_device_status_where(workspace, nullptr, stream);
+}
+
+gdn_status gdn_dual_read_device_status_where(const void *workspace, int32_t *where, gdn_stream_t stream) {
     if (!workspace) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    int32_t status = 0;
-    if (cudaMemcpyAsync(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    gdn::WorkspaceHeader h;
+    if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return GDN_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return GDN_ERR_CUDA;
-    return status == 0 ? GDN_OK : static_cast<gdn_status>(status);
+    if (where) *where = h.timeout_where;
+    return h.status == 0 ? GDN_OK : static_cast<gdn_status>(h.status);
 }
 
 }  // extern "C"

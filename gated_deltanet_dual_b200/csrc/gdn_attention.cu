@@ -43,7 +43,7 @@ using namespace sm100;
 constexpr int AD = 128;                     // head dim
 constexpr int AT = 128;                     // query rows / keys per tile
 constexpr int kAThreads = 128;              // thread t owns query row t
-constexpr uint32_t kAWaitIters = 1u << 24;
+constexpr uint32_t kAWaitIters = 1u << 24;   // bound of an ordinary wait (the test entry point lowers it)
 constexpr int A_OFF_Q = 0, A_OFF_K = 32768, A_OFF_V = 65536;   // [2 d-halves][128 rows][128 B] each
 constexpr int A_SMEM = 3 * 32768 + 1024;
 constexpr uint32_t TA_S = 0;                // S (fp32, 128 columns); P (bf16 pairs) over its first 64
@@ -54,6 +54,7 @@ struct AttnParams {
     int32_t H, Hkv, V, B;
     int64_t TR;
     float scale_log2;                       // log2(e) / sqrt(d)
+    uint32_t wait_iters;                    // test instantiation: bound of the mbarrier waits, in polls
     WorkspaceHeader *ws;
     void *out, *out_noisy;
     int32_t N;
@@ -80,6 +81,8 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&p);
 }
 
+// TW: the test instantiation, whose waits poll with the caller's bound (gdn_attn_forward_test_wait_limit).
+template <bool TW>
 __global__ void __launch_bounds__(kAThreads, 2)
 gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant__ AttnMaps M) {
     extern __shared__ uint8_t smraw[];
@@ -152,16 +155,34 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
             atomicExch(&P.ws->timeout_where, where);
         }
     };
+    // Error path (as in the chunked kernel): after one of its waits gave up, a thread waits on
+    // nothing more; thread 0, which issues every TMA load and MMA commit, counts per mbarrier the
+    // phases it issued and those it saw complete, and drains the rest before the CTA frees its
+    // tensor memory.
+    bool dead = false;
+    uint32_t iss_q = 0, iss_k = 0, iss_v = 0, iss_s = 0, iss_o = 0;
+    uint32_t ok_q = 0, ok_k = 0, ok_v = 0, ok_s = 0, ok_o = 0;
+    auto wait_bar = [&](uint64_t *bar, uint32_t parity, uint32_t &ok, int where) {
+        if (!dead && *reinterpret_cast<volatile int *>(&s_abort)) dead = true;
+        if (dead) return;
+        if (kwait<TW>(bar, parity, kAWaitIters, P.wait_iters)) ++ok;
+        else {
+            dead = true;
+            fail(where);
+        }
+    };
     // key tile j: clean keys [s + 128 j, +128) or (j == nkc) the tile's own noisy rows
     auto issue_tile = [&](uint8_t *dst, const CUtensorMap *clean, const CUtensorMap *noisy, uint64_t *bar, int j) {
         const CUtensorMap *map = j < nkc ? clean : noisy;
         const int row0 = j < nkc ? s + AT * j : (int)nrow0;
+        ++(bar == &bar_k ? iss_k : iss_v);
         mbar_arrive_expect_tx(bar, 32768u);
         for (int hf = 0; hf < 2; ++hf)
             for (int rh = 0; rh < 2; ++rh)
                 tma_load_3d(dst + hf * 16384 + rh * 8192, map, bar, hf * 64, hk, row0 + 64 * rh);
     };
     if (tid == 0) {
+        ++iss_q;
         mbar_arrive_expect_tx(&bar_q, 32768u);
         const CUtensorMap *qm = kind == 0 ? &M.q : &M.qn;
         for (int hf = 0; hf < 2; ++hf)
@@ -182,24 +203,29 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
     const int b0 = kind ? (i_resp / B) * B : 0;
     float m_ref = -INFINITY, l = 0.f;
     const float sl2 = P.scale_log2;
+    bool stop = false;        // uniform over the CTA: leave the key loop (a wait gave up)
 
     for (int j = 0; j < nk; ++j) {
         // ---- S = Q K_j^T
         if (tid == 0) {
-            if (j == 0 && !mbar_wait(&bar_q, 0, kAWaitIters)) fail(1);
-            if (!mbar_wait(&bar_k, j & 1, kAWaitIters)) fail(2);
+            if (j == 0) wait_bar(&bar_q, 0, ok_q, 1);
+            wait_bar(&bar_k, j & 1, ok_k, 2);
             tc_fence_after();
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                 mma_bf16(tb + TA_S, dQ + (off >> 4), dK + (off >> 4), idesc, kk > 0);
             }
             mma_commit(&bar_s);
+            ++iss_s;
         }
         __syncwarp();
-        if (!mbar_wait(&bar_s, j & 1, kAWaitIters)) fail(3);
+        {
+            uint32_t okv = 0;
+            wait_bar(&bar_s, j & 1, tid == 0 ? ok_s : okv, 3);
+        }
         __syncwarp();
         tc_fence_after();
-        if (tid == 0 && j + 1 < nk) issue_tile(sm + A_OFF_K, &M.k, &M.kn, &bar_k, j + 1);
+        if (tid == 0 && j + 1 < nk && !dead) issue_tile(sm + A_OFF_K, &M.k, &M.kn, &bar_k, j + 1);
         // visible columns of this row in tile j: [lo, hi)
         int lo = 0, hi;
         if (j < nkc) hi = kind == 0 ? AT * (tile - j) + r + 1 : Pn + b0 - AT * j;
@@ -266,27 +292,29 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
         l += ls;
         tmem_wait_st();
         tc_fence_before();
-        __syncthreads();
-        if (s_abort) break;
+        if ((stop = __syncthreads_or(*reinterpret_cast<volatile int *>(&s_abort) != 0))) break;
         // ---- O += P V_j
         if (tid == 0) {
             tc_fence_after();
-            if (!mbar_wait(&bar_v, j & 1, kAWaitIters)) fail(4);
+            wait_bar(&bar_v, j & 1, ok_v, 4);
             for (int kk = 0; kk < 8; ++kk)
                 mma_bf16_ts(tb + TA_O, tb + TA_S + kk * 8, dV + ((kk * 2048) >> 4), idesc_pv, (j > 0 || kk > 0));
             mma_commit(&bar_o);
+            ++iss_o;
         }
         __syncwarp();
-        if (!mbar_wait(&bar_o, j & 1, kAWaitIters)) fail(5);
+        {
+            uint32_t okv = 0;
+            wait_bar(&bar_o, j & 1, tid == 0 ? ok_o : okv, 5);
+        }
         __syncwarp();
         tc_fence_after();
-        if (tid == 0 && j + 1 < nk) issue_tile(sm + A_OFF_V, &M.v, &M.vn, &bar_v, j + 1);
-        __syncthreads();
-        if (s_abort) break;
+        if (tid == 0 && j + 1 < nk && !dead) issue_tile(sm + A_OFF_V, &M.v, &M.vn, &bar_v, j + 1);
+        if ((stop = __syncthreads_or(*reinterpret_cast<volatile int *>(&s_abort) != 0))) break;
     }
 
     // ---- out = O / l
-    if (!s_abort) {
+    if (!stop) {
         const bool valid = kind == 0 ? (AT * tile + r < len) : (i_resp < R);
         __nv_bfloat16 *orow = kind == 0
             ? static_cast<__nv_bfloat16 *>(P.out) + ((int64_t)(qrow0 + r) * P.H + h) * AD
@@ -309,6 +337,16 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
                 }
             }
         }
+    }
+    // Drain (a no-op unless a wait gave up): every phase thread 0 issued but did not see
+    // complete, in order, with the normal limit.
+    if (tid == 0) {
+        const uint32_t lim = kDrainWaitIters;
+        for (uint32_t p = ok_q; p < iss_q; ++p) mbar_wait(&bar_q, p & 1, lim);
+        for (uint32_t p = ok_k; p < iss_k; ++p) mbar_wait(&bar_k, p & 1, lim);
+        for (uint32_t p = ok_v; p < iss_v; ++p) mbar_wait(&bar_v, p & 1, lim);
+        for (uint32_t p = ok_s; p < iss_s; ++p) mbar_wait(&bar_s, p & 1, lim);
+        for (uint32_t p = ok_o; p < iss_o; ++p) mbar_wait(&bar_o, p & 1, lim);
     }
     tc_fence_before();
     __syncthreads();
@@ -385,11 +423,11 @@ extern "C" size_t gdn_attn_workspace_size(const gdn_attn_desc *desc, const int32
     return sizeof(WorkspaceHeader);
 }
 
-extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q, const void *k, const void *v,
-                                       const void *qn, const void *kn, const void *vn,
-                                       const int32_t *doc_offsets, const int32_t *prompt_len,
-                                       void *out, void *out_noisy, void *workspace, size_t workspace_bytes,
-                                       gdn_stream_t stream) {
+static gdn_status attn_forward_impl(const gdn_attn_desc *desc, const void *q, const void *k, const void *v,
+                                    const void *qn, const void *kn, const void *vn,
+                                    const int32_t *doc_offsets, const int32_t *prompt_len,
+                                    void *out, void *out_noisy, void *workspace, size_t workspace_bytes,
+                                    uint32_t wait_iters, gdn_stream_t stream) {
     if (!attn_desc_ok(desc)) return GDN_ERR_INVALID_ARG;
     int64_t T = 0, TR = 0;
     if (!attn_layout(desc, doc_offsets, prompt_len, &T, &TR)) return GDN_ERR_INVALID_ARG;
@@ -411,6 +449,7 @@ extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q,
     P.TR = TR;
     P.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)desc->head_dim));
     P.ws = static_cast<WorkspaceHeader *>(workspace);
+    P.wait_iters = wait_iters;
     P.out = out;
     P.out_noisy = out_noisy;
     const int N = desc->num_docs;
@@ -457,11 +496,34 @@ extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q,
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(gdn_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, A_SMEM);
+        attr_err = cudaFuncSetAttribute(gdn_attention_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, A_SMEM);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(gdn_attention_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, A_SMEM);
     });
     if (attr_err != cudaSuccess) return GDN_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(WorkspaceHeader), st) != cudaSuccess) return GDN_ERR_CUDA;
-    gdn_attention_kernel<<<(unsigned)items, kAThreads, A_SMEM, st>>>(P, maps);
+    if (wait_iters < kAWaitIters) gdn_attention_kernel<true><<<(unsigned)items, kAThreads, A_SMEM, st>>>(P, maps);
+    else gdn_attention_kernel<false><<<(unsigned)items, kAThreads, A_SMEM, st>>>(P, maps);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+extern "C" gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q, const void *k, const void *v,
+                                       const void *qn, const void *kn, const void *vn,
+                                       const int32_t *doc_offsets, const int32_t *prompt_len,
+                                       void *out, void *out_noisy, void *workspace, size_t workspace_bytes,
+                                       gdn_stream_t stream) {
+    return attn_forward_impl(desc, q, k, v, qn, kn, vn, doc_offsets, prompt_len, out, out_noisy, workspace,
+                             workspace_bytes, kAWaitIters, stream);
+}
+
+extern "C" gdn_status gdn_attn_forward_test_wait_limit(const gdn_attn_desc *desc, const void *q, const void *k,
+                                                       const void *v, const void *qn, const void *kn,
+                                                       const void *vn, const int32_t *doc_offsets,
+                                                       const int32_t *prompt_len, void *out, void *out_noisy,
+                                                       void *workspace, size_t workspace_bytes,
+                                                       uint32_t wait_iters, gdn_stream_t stream) {
+    if (wait_iters < 1) return GDN_ERR_INVALID_ARG;
+    return attn_forward_impl(desc, q, k, v, qn, kn, vn, doc_offsets, prompt_len, out, out_noisy, workspace,
+                             workspace_bytes, wait_iters, stream);
 }

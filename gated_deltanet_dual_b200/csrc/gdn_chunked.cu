@@ -18,34 +18,36 @@
 //   Z_j  = Gammatil_B q~_j - sum_l y_l beta~_l Gammatil_l k~_l,   WV_j = sum_l y_l beta~_l v~_l,
 //   o~_j = Gamma_e Z_j S0 + (Z_j K^T o M_j) U + WV_j,   M_ji = e^{gamma_e-gamma_i} [i <= e].
 //
-// One CTA per (document, head) unit (static schedule over the longest-first unit order), one
-// CTA per SM: 8 math warps + 1 control warp (TMA producer and single-thread MMA issuer).  Each
-// chunk runs five tensor-core phases, each followed by a math phase:
+// Persistent CTAs, one per SM, take (document, head) work items longest first by greedy list
+// scheduling (a counter in the workspace); with fewer units than half the SMs each unit is split
+// over two CTAs (the second rebuilds its split-point state with the clean-only chain).  256
+// threads = 8 warps, all of them math warps; thread 0 also issues the TMA loads and the MMAs.
+// Each chunk runs five tensor-core phases, each followed by a math phase:
 //   PK1  [Q;K]K^T, [q~0;q~1][k~0;k~1]^T, [k~0;k~1][k~0;k~1]^T     (S-independent)
 //   PK2  [P;T] T -> P T,  [Z0;Z1] K^T                              (S-independent)
 //   S1   [Q;K] S0,  [Gamma_e Z] S0 (+= WV)                         (needs S0)
 //   S2   [P T; T] R                                                (needs R)
 //   S3   Khat^T U,  M'_Z U (+=)                                    (needs U)
 // Inputs of the next chunk are prefetched by TMA while the current chunk's S-dependent phases
-// run.  All waits are bounded; on timeout the kernel records GDN_ERR_TIMEOUT and exits.
+// run.  All waits are bounded; on timeout the kernel records GDN_ERR_TIMEOUT, waits for the
+// copies and MMAs it has issued, and exits.
+#include <algorithm>
 #include <cudaTypedefs.h>
 #include <mutex>
 #include <type_traits>
 
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
+#include "gdn_chunk_common.cuh"
 
 namespace gdn {
 namespace {
 
 using namespace sm100;
 
-constexpr int D = 128;                 // d_k = d_v
-constexpr int CH = 64;                 // chunk length
 constexpr int kMathWarps = 8;
 constexpr int kMathThreads = kMathWarps * 32;
 constexpr int kThreads = kMathThreads;   // thread 0 also issues TMA and MMA
-constexpr uint32_t kWaitIters = 1u << 22;
 
 // Dynamic shared memory layout (offsets from a 1024-byte aligned base).
 constexpr int OFF_S0 = 0;          // 32 KB  S0 bf16, MN-major B: 2 v-halves x [128 k-rows x 128 B]
@@ -67,10 +69,6 @@ constexpr uint32_t TM_N = 256;     // noisy accumulator (WV + Gamma_e Z S0 + M'_
 constexpr uint32_t TM_TK = 384;    // [Q;K]K^T | P T
 constexpr uint32_t TM_ZK = 448;    // Z K^T
 
-struct Maps {
-    CUtensorMap q, k, v, qn, kn, vn;
-};
-
 __device__ __forceinline__ void bar_all() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
 __device__ __forceinline__ void bar_math() { bar_all(); }
 // Warps 1..7 only: work overlapped with an MMA batch that thread 0 (warp 0) is issuing.
@@ -78,178 +76,6 @@ __device__ __forceinline__ void bar_side() { asm volatile("bar.sync 3, %0;" ::"n
 // Named barrier 4: warps 1..7 arrive (no wait), warp 0 waits for them.
 __device__ __forceinline__ void bar_arrive_khat() { asm volatile("bar.arrive 4, %0;" ::"n"(kThreads) : "memory"); }
 __device__ __forceinline__ void bar_sync_khat() { asm volatile("bar.sync 4, %0;" ::"n"(kThreads) : "memory"); }
-
-__device__ __forceinline__ uint4 pack8(const float *f) {
-    uint4 r;
-    __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
-    __nv_bfloat162 b = __floats2bfloat162_rn(f[2], f[3]);
-    __nv_bfloat162 c = __floats2bfloat162_rn(f[4], f[5]);
-    __nv_bfloat162 d = __floats2bfloat162_rn(f[6], f[7]);
-    r.x = *reinterpret_cast<uint32_t *>(&a);
-    r.y = *reinterpret_cast<uint32_t *>(&b);
-    r.z = *reinterpret_cast<uint32_t *>(&c);
-    r.w = *reinterpret_cast<uint32_t *>(&d);
-    return r;
-}
-
-__device__ __forceinline__ void unpack8(uint4 u, float *f) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
-        float2 p = __bfloat1622float2(h);
-        f[2 * i] = p.x;
-        f[2 * i + 1] = p.y;
-    }
-}
-
-// fp32 64x64 solve scratch: 16-byte chunk c>>2 of row r sits at chunk (c>>2) ^ (r & 7), so both
-// row-segment accesses by one thread (float4) and column accesses across a warp avoid conflicts.
-__device__ __forceinline__ int sidx(int r, int c) { return r * 64 + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3); }
-__device__ __forceinline__ float4 *srow4(float *sa, int r, int c4) {
-    return reinterpret_cast<float4 *>(sa + r * 64 + ((((c4 >> 2) ^ (r & 7))) << 2));
-}
-
-struct Unit {
-    int n, h;
-    int s, len, prompt, R, roff;
-    int nchunks, m_first;
-};
-
-__device__ __forceinline__ Unit make_unit(const Params &P, int u) {
-    Unit U;
-    U.n = P.unit_doc[u / P.H];
-    U.h = u % P.H;
-    U.s = P.doc_start[U.n];
-    U.len = P.doc_start[U.n + 1] - U.s;
-    U.prompt = P.doc_prompt[U.n];
-    U.R = U.len - U.prompt;
-    U.roff = P.resp_off[U.n];
-    const int npre = (U.prompt + CH - 1) / CH;
-    const int nres = (U.R + CH - 1) / CH;
-    U.m_first = -npre;
-    U.nchunks = npre + nres;
-    return U;
-}
-
-// Block coefficients of one noisy row: y = Ptil_j Ttil (back substitution against the block's
-// own I + Atil), then ycoef = y beta~ Gammatil (for Z) and wcoef = y beta~ (for WV).
-// Shared-memory staging of the noisy block coefficients (B >= 16): per TMEM lane quadrant, 32
-// rows of B fp32 values (one 16-byte pad between the two blocks of a quadrant when B = 16, so
-// the two blocks' broadcast reads fall in different bank groups).
-template <int B>
-constexpr int kAtQuadBytes = 32 * B * 4 + (B < 32 ? 16 : 0);
-template <int B>
-__device__ __forceinline__ constexpr int at_swz(int r) { return B >= 32 ? (r & 7) : ((r >> 1) & 3); }
-
-template <int B>
-__device__ __forceinline__ void noisy_coeffs(const float (&wq)[32], const float (&wk)[32], int lane, int j,
-                                             const float *ngam, const float *nbeta, const float *nE,
-                                             const float *nF, bool nfact, float *s_at,
-                                             float (&ycoef)[B], float (&wcoef)[B], float &gend) {
-    const int bs = (j / B) * B;
-    const int jl = j - bs;
-    const int wofs = bs & 31;
-    float aq[B], ak[B], gl[B], bl[B];
-#pragma unroll
-    for (int l = 0; l < B; ++l) {
-        aq[l] = 0.f;
-        ak[l] = 0.f;
-        gl[l] = ngam[bs + l];
-        bl[l] = nbeta[bs + l];
-    }
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-        if ((c / B) * B == wofs) {
-            aq[c % B] = wq[c];
-            ak[c % B] = wk[c];
-        }
-    }
-    const float gj = ngam[j], bj = nbeta[j];
-    gend = gl[B - 1];
-    float arow[B], pt[B], y[B];
-    if (B >= 16 && nfact) {       // e^{gamma~_a - gamma~_b} = E_a F_b, prepared once per row
-        const float Ej = nE[j], Eend = nE[bs + B - 1];
-#pragma unroll
-        for (int l = 0; l < B; ++l) {
-            const float Fl = nF[bs + l];
-            arow[l] = (l < jl) ? bj * (Ej * Fl) * ak[l] : 0.f;
-            pt[l] = aq[l] * (Eend * Fl);
-        }
-    } else {
-#pragma unroll
-        for (int l = 0; l < B; ++l) {
-            arow[l] = (l < jl) ? bj * exp2f(fminf(gj - gl[l], 0.f)) * ak[l] : 0.f;
-            pt[l] = aq[l] * exp2f(gend - gl[l]);
-        }
-    }
-    // Right-looking back substitution: once y_mm is final it is taken out of every earlier
-    // position at once, so the dependent chain is B steps of one FMA each.
-    if constexpr (B >= 16) {
-        // Row mm of the block's Atil is needed by every lane of the block: the rows go through
-        // shared memory once and are read back as broadcast 16-byte loads (about B^2/8 loads
-        // instead of B^2/2 shuffles).  16-byte column c4 of row r sits at c4 ^ at_swz(r), so the
-        // row stores of 8 consecutive lanes hit 8 distinct bank groups; r & 7 of a block row is
-        // mm & 7, known at compile time.
-        float *myrow = s_at + lane * B + (B < 32 ? (lane / B) * 4 : 0);
-#pragma unroll
-        for (int c4 = 0; c4 < B / 4; ++c4)
-            *reinterpret_cast<float4 *>(myrow + 4 * (c4 ^ at_swz<B>(jl))) =
-                make_float4(arow[4 * c4], arow[4 * c4 + 1], arow[4 * c4 + 2], arow[4 * c4 + 3]);
-        __syncwarp();
-        const float *blk = myrow - jl * B;
-#pragma unroll
-        for (int mm = B - 1; mm >= 0; --mm) {
-            y[mm] = pt[mm];
-#pragma unroll
-            for (int c4 = 0; c4 < (mm + 3) / 4; ++c4) {
-                const float4 a = *reinterpret_cast<const float4 *>(blk + mm * B + 4 * (c4 ^ at_swz<B>(mm)));
-                const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (4 * c4 + e < mm) pt[4 * c4 + e] = fmaf(-y[mm], av[e], pt[4 * c4 + e]);
-            }
-        }
-    } else {
-        const int base = lane - jl;
-#pragma unroll
-        for (int mm = B - 1; mm >= 0; --mm) {
-            y[mm] = pt[mm];
-#pragma unroll
-            for (int l = 0; l < mm; ++l) pt[l] = fmaf(-y[mm], __shfl_sync(0xffffffffu, arow[l], base + mm), pt[l]);
-        }
-    }
-#pragma unroll
-    for (int l = 0; l < B; ++l) {
-        wcoef[l] = y[l] * bl[l];
-        ycoef[l] = wcoef[l] * ((B >= 16 && nfact) ? nE[bs + l] : exp2f(gl[l]));
-    }
-}
-
-// This thread's half (K columns [64ch, 64ch+64), i.e. the noisy rows of view ch) of the
-// block-diagonal row `sign * coef` of noisy row (view v, block start bs), stored into tensor
-// memory as bf16 pairs (low half = even k): an A operand for a tensor-memory MMA.
-template <int B>
-__device__ __forceinline__ void store_block_row(uint32_t taddr, int ch, int v, int bs, const float (&coef)[B],
-                                                float sign) {
-    float w[32];
-    if constexpr (B == 1) {
-        __nv_bfloat162 pr = (bs & 1) ? __floats2bfloat162_rn(0.f, sign * coef[0]) : __floats2bfloat162_rn(sign * coef[0], 0.f);
-        const float pf = __uint_as_float(*reinterpret_cast<uint32_t *>(&pr));
-#pragma unroll
-        for (int x = 0; x < 32; ++x) w[x] = (ch == v && x == (bs >> 1)) ? pf : 0.f;
-    } else {
-        constexpr int HB = B / 2;
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-            const int l0 = 2 * (x % HB);
-            __nv_bfloat162 pr = __floats2bfloat162_rn(sign * coef[l0], sign * coef[l0 + 1]);
-            const float pf = __uint_as_float(*reinterpret_cast<uint32_t *>(&pr));
-            w[x] = (ch == v && (x / HB) == (bs / B)) ? pf : 0.f;
-        }
-    }
-    tmem_st32(taddr, w);
-}
 
 // Noisy rows, step 1: block coefficients of this thread's row from [q~;k~]k~^T (TMEM), then the
 // rows of W~ and -Y~ as tensor-memory A operands (columns [0,64) and [64,128) from TM_TK).
@@ -295,130 +121,6 @@ __device__ __forceinline__ void z_epilogue(uint8_t *sm, uint32_t tb, int q, int 
             *reinterpret_cast<uint4 *>(nq + o) = pack8(z);
         }
     }
-}
-
-// Exact-decay variants of two epilogues, for a chunk whose cumulative decays leave the range in
-// which e^{gamma_t - gamma_i} factorises as E_t F_i.  Such chunks are rare; out of line, they keep
-// the common path's instruction footprint small.
-struct Rows4 {
-    uint4 v[4];
-};
-
-// P rows (rho < 64: returned as bf16) or A rows (rho >= 64: written to the fp32 solve scratch)
-// of [Q;K]K^T (TMEM columns at taddr), with the decays exponentiated one by one.
-__device__ __noinline__ Rows4 pa_rows_exact(uint32_t taddr, int rho, int ch, const float *s_gam,
-                                           const float *s_beta, float *scratch) {
-    float tk[32];
-    tmem_ld32(taddr, tk);
-    tmem_wait_ld();
-    Rows4 r;
-    if (rho < 64) {
-        const int t = rho;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-            const int i = 32 * ch + c;
-            tk[c] = (i <= t) ? tk[c] * exp2f(fminf(s_gam[t] - s_gam[i], 0.f)) : 0.f;
-        }
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) r.v[c4] = pack8(tk + 8 * c4);
-    } else {
-        const int t = rho - 64;
-        const float bt = s_beta[t];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-            const int i = 32 * ch + c;
-            tk[c] = (i < t) ? bt * exp2f(fminf(s_gam[t] - s_gam[i], 0.f)) * tk[c] : 0.f;
-        }
-#pragma unroll
-        for (int g4 = 0; g4 < 8; ++g4)
-            *srow4(scratch, t, 32 * ch + 4 * g4) = make_float4(tk[4 * g4], tk[4 * g4 + 1], tk[4 * g4 + 2], tk[4 * g4 + 3]);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) r.v[c4] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    return r;
-}
-
-// M'_Z rows of a noisy row (Z K^T in TMEM at taddr; boundary row e of its block, -1 for S0) with
-// exact decays, then Z <- Gamma_e Z in place for the state product.
-__device__ __noinline__ void mz_rows_exact(uint8_t *sm, uint32_t taddr, int rho, int ch, int e,
-                                          const float *s_gam, const float *s_E) {
-    float zk[32];
-    tmem_ld32(taddr, zk);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-        const int i = 32 * ch + c;
-        zk[c] = (i <= e) ? zk[c] * exp2f(fminf(s_gam[e < 0 ? 0 : e] - s_gam[i], 0.f)) : 0.f;
-    }
-#pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4)
-        *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
-    const float Ge = e >= 0 ? s_E[e] : 1.f;    // Gamma_e (1 for e = -1)
-    uint8_t *zrow = sm + OFF_NQ + ch * 16384;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4 *>(zrow + sw128_off(rho, c8)), f);
-#pragma unroll
-        for (int x = 0; x < 8; ++x) f[x] *= Ge;
-        *reinterpret_cast<uint4 *>(zrow + sw128_off(rho, c8)) = pack8(f);
-    }
-}
-
-// 32 x 32 fp32 staging block (the 32-merge's result): 128-byte rows, 16-byte chunks swizzled by
-// the row like the solve scratch.
-__device__ __forceinline__ int widx(int r, int c) { return r * 32 + ((((c >> 2) ^ (r & 7))) << 2) + (c & 3); }
-__device__ __forceinline__ float4 *wrow4(float *w, int r, int c4) {
-    return reinterpret_cast<float4 *>(w + r * 32 + ((((c4 >> 2) ^ (r & 7))) << 2));
-}
-
-// One merge of the triangular inverse by one warp that owns NC consecutive output columns
-// [cb, cb + NC) of the S x S block below the diagonal at offset o.  With T11 = T[o.., o..] and
-// T22 = T[o+S.., o+S..] already inverted (unit lower, zeros above the diagonal):
-//   X = A[o+S.., o..] T11,   T[o+S.., o..] = -T22 X.
-// Lane (g = lane / NC, cl = lane % NC) holds column cb + cl for the rows g + RG*i.  X moves between
-// the lanes by shuffles, so the warp needs no barrier; T11[k][c] = 0 for k < c lets the first
-// product start at k = cb, and the second product of row r stops at k = r (warp-uniform bounds).
-// The result goes out through `store` (block-local row and column) after `before_store()`, which
-// separates this warp's reads from other warps' writes when several warps share one merge.
-template <int S, int NC, typename Store, typename Sync>
-__device__ __forceinline__ void warp_merge(const float *sa, int o, int cb, int lane, Store store, Sync before_store) {
-    constexpr int RG = 32 / NC, NR = S / RG;
-    const int cl = lane % NC, g = lane / NC, c = cb + cl;
-    float x[NR];
-#pragma unroll
-    for (int i = 0; i < NR; ++i) x[i] = 0.f;
-#pragma unroll
-    for (int k4 = 0; k4 < S; k4 += 4) {
-        if (k4 < (cb & ~3)) continue;
-        float tv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) tv[e] = sa[sidx(o + k4 + e, o + c)];
-#pragma unroll
-        for (int i = 0; i < NR; ++i) {
-            const float4 a = *srow4(const_cast<float *>(sa), o + S + g + RG * i, o + k4);
-            x[i] = fmaf(a.w, tv[3], fmaf(a.z, tv[2], fmaf(a.y, tv[1], fmaf(a.x, tv[0], x[i]))));
-        }
-    }
-    float y[NR];
-#pragma unroll
-    for (int i = 0; i < NR; ++i) y[i] = 0.f;
-#pragma unroll
-    for (int k4 = 0; k4 < S; k4 += 4) {
-        float xk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) xk[e] = __shfl_sync(0xffffffffu, x[(k4 + e) / RG], ((k4 + e) % RG) * NC + cl);
-#pragma unroll
-        for (int i = 0; i < NR; ++i) {
-            if (k4 <= RG * i + RG - 1) {
-                const float4 a = *srow4(const_cast<float *>(sa), o + S + g + RG * i, o + S + k4);
-                y[i] = fmaf(a.w, xk[3], fmaf(a.z, xk[2], fmaf(a.y, xk[1], fmaf(a.x, xk[0], y[i]))));
-            }
-        }
-    }
-    before_store();
-#pragma unroll
-    for (int i = 0; i < NR; ++i) store(g + RG * i, c, -y[i]);
 }
 
 // T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 scratch, while warp 0 issues an MMA
@@ -697,12 +399,14 @@ __device__ __noinline__ int next_work_item(WorkspaceHeader *ws, int *s_next) {
     return nx;
 }
 
-template <int B>
+// TW: the test instantiation, whose waits poll with the caller's bound (gdn_dual_forward_test_wait_limit).
+template <int B, bool TW = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps M) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bar_a, bar_b, bar_mma, bar_mma2;   // bar_mma2: the noisy half of PK1 only
+    __shared__ uint64_t bar_drain;                         // error path: all MMAs of thread 0 done
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     // Per-chunk scalars, double-buffered so the next chunk's are prepared while this chunk's
@@ -729,6 +433,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         mbar_init(&bar_b, 1);
         mbar_init(&bar_mma, 1);
         mbar_init(&bar_mma2, 1);
+        mbar_init(&bar_drain, 1);
         fence_mbar_init();
         s_abort = 0;
     }
@@ -754,23 +459,44 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             atomicExch(&P.ws->timeout_where, where);
         }
     };
+    // Error path.  Once one of this thread's waits has given up, the thread waits on nothing more
+    // (the CTA leaves at its next abort check, all threads at the same barrier).  A phase counter
+    // advances only when its wait succeeds, so thread 0's counters are the phases it saw complete.
+    // Before the CTA frees its tensor memory and exits, thread 0 -- the only thread that issues TMA
+    // loads and MMAs -- waits for everything it issued: one more commit covers all its MMAs, and on
+    // the two TMA barriers every phase between its counter and the loads it issued (s_iss), so no
+    // bulk copy or MMA is left writing into shared or tensor memory that is no longer the CTA's.
+    bool dead = false;
+    __shared__ uint32_t s_iss[2];
+    if (tid == 0) s_iss[0] = s_iss[1] = 0;
+    auto wait_bar = [&](uint64_t *bar, uint32_t &ph, int where) {
+        if (!dead) {
+            if (kwait<TW>(bar, ph & 1, kWaitIters, P.wait_iters)) ++ph;
+            else {
+                dead = true;
+                fail(where);
+            }
+        }
+    };
+    // bar_all that also tells every thread, uniformly, whether the CTA is aborting
+    auto abort_check = [&] { return bar_sync_or(1, kThreads, *reinterpret_cast<volatile int *>(&s_abort) != 0); };
     auto wait_mma = [&](int where) {
-        if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(where);
-        ++ph_mma;
+        wait_bar(&bar_mma, ph_mma, where);
         __syncwarp();            // reconverge before warp-collective tcgen05.ld/st
         tc_fence_after();
     };
     auto wait_mma2 = [&](int where) {
-        if (!mbar_wait(&bar_mma2, ph_mma2 & 1, kWaitIters)) fail(where);
-        ++ph_mma2;
+        wait_bar(&bar_mma2, ph_mma2, where);
         __syncwarp();
         tc_fence_after();
     };
+    auto commit_mma = [&] { mma_commit(&bar_mma); };   // thread 0
 
     // Issue the TMA loads of chunk m of unit U (control lane 0).  group A: [Q;K] and, for a
     // response chunk, [q~;.] and v~;  group B: V and, for a response chunk, [k~;.].
     auto issue_a = [&](const Unit &U, int m, bool nz) {
         const int cstart = U.s + U.prompt + CH * m;
+        ++s_iss[0];
         mbar_arrive_expect_tx(&bar_a, 32768u + (nz ? 65536u : 0u));
         for (int hf = 0; hf < 2; ++hf) {
             tma_load_3d(sm + OFF_QK + hf * 16384, &M.q, &bar_a, hf * 64, U.h, cstart);
@@ -788,6 +514,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     };
     auto issue_b = [&](const Unit &U, int m, bool nz) {
         const int cstart = U.s + U.prompt + CH * m;
+        ++s_iss[1];
         mbar_arrive_expect_tx(&bar_b, 16384u + (nz ? 32768u : 0u));
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_V + hf * 8192, &M.v, &bar_b, hf * 64, U.h, cstart);
         if (nz) {
@@ -915,6 +642,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     // uneven documents no longer pile up on the CTAs that a fixed stride would give them).
     const int parts = P.parts;
     __shared__ int s_next;
+    bool stop = false;        // uniform over the CTA: leave the work loop (a wait gave up)
     for (int w = blockIdx.x; w < P.num_units * parts; w = next_work_item(P.ws, &s_next)) {
         const int u = w / parts, part = w % parts;
         const Unit U = make_unit(P, u);
@@ -979,11 +707,9 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 cp_async_commit();
             }
             // ---- wait for this chunk's tiles ----
-            if (!mbar_wait(&bar_a, ph_a & 1, kWaitIters)) fail(1);
-            ++ph_a;
+            wait_bar(&bar_a, ph_a, 1);
             if (conv) {
-                if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
-                ++ph_b;
+                wait_bar(&bar_b, ph_b, 2);
                 cp_async_wait_all();
                 // The state rows wait in tensor memory (columns free until the batch MMAs) while
                 // the conv needs the registers.
@@ -1008,8 +734,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 }
             }
             __syncwarp();
-            bar_all();
-            if (s_abort) break;
+            if ((stop = abort_check())) break;
             const bool fact = s_okw[cb][0] && s_okw[cb][1];
 
             // ================= PK1: [Q;K]K^T now, the noisy products once group B is in ========
@@ -1020,7 +745,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     mma_bf16(tb + TM_TK, dK_qk + (off >> 4), dK_qk + ((8192 + off) >> 4),
                              make_idesc_bf16(128, 64, 0, 0), kk > 0);
                 }
-                mma_commit(&bar_mma);
+                commit_mma();
             }
             __syncwarp();
             // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout), on
@@ -1039,10 +764,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 }
             };
             if constexpr (!kKhatLate) build_khat();
-            if (!conv) {                                  // V and [k~0;k~1]
-                if (!mbar_wait(&bar_b, ph_b & 1, kWaitIters)) fail(2);
-                ++ph_b;
-            }
+            if (!conv) wait_bar(&bar_b, ph_b, 2);   // V and [k~0;k~1]
             __syncwarp();
             if (noisy && tid == 0) {
                 for (int kk = 0; kk < 8; ++kk) {
@@ -1118,7 +840,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                         mma_bf16_ts(tb + TM_R1, tb + TM_TK + 64 + kk * 8, dM_nk + ((kk * 2048) >> 4),
                                     make_idesc_bf16(128, 128, 0, 1), kk > 0);
                 }
-                mma_commit(&bar_mma);
+                commit_mma();
             }
             __syncwarp();
             solve_T(scratch, wstage, tid, warp);
@@ -1168,8 +890,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
-            bar_all();
-            if (s_abort) break;
+            if ((stop = abort_check())) break;
 
             // ================= PK2 =================
             if (tid == 0) {
@@ -1184,7 +905,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                                  make_idesc_bf16(128, 64, 0, 0), kk > 0);
                     }
                 }
-                mma_commit(&bar_mma);
+                commit_mma();
             }
             __syncwarp();
             wait_mma(20);
@@ -1212,13 +933,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
                         *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
                 } else {
-                    mz_rows_exact(sm, tmem_addr(tb, q * 32, TM_ZK + 32 * ch), rho, ch, e, s_gam, s_E);
+                    mz_rows_exact(sm + OFF_NK, sm + OFF_NQ, tmem_addr(tb, q * 32, TM_ZK + 32 * ch), rho, ch, e, s_gam, s_E);
                 }
             }
             fence_async_smem();
             tc_fence_before();
-            bar_all();
-            if (s_abort) break;
+            if ((stop = abort_check())) break;
 
             // ================= S2: [PT;T] R and the noisy rows' state product =================
             if (tid == 0) {
@@ -1233,11 +953,15 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                                  make_idesc_bf16(128, 128, 0, 1), 1u);
                     }
                 }
-                mma_commit(&bar_mma);
+                commit_mma();
                 // prefetch group A of the next chunk once [Q;K] and Z are consumed
-                if (!kKhatLate && !last) {
-                    if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(40);
-                    else issue_a(U, m + 1, chunk_noisy(ci + 1));
+                if (!kKhatLate && !last && !dead) {
+                    if (!kwait<TW>(&bar_mma, ph_mma & 1, kWaitIters, P.wait_iters)) {
+                        dead = true;
+                        fail(40);
+                    } else {
+                        issue_a(U, m + 1, chunk_noisy(ci + 1));
+                    }
                 }
             }
             __syncwarp();
@@ -1249,9 +973,13 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     bar_arrive_khat();
                 } else {
                     bar_sync_khat();
-                    if (tid == 0 && !last) {
-                        if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(40);
-                        else issue_a(U, m + 1, chunk_noisy(ci + 1));
+                    if (tid == 0 && !last && !dead) {
+                        if (!kwait<TW>(&bar_mma, ph_mma & 1, kWaitIters, P.wait_iters)) {
+                            dead = true;
+                            fail(40);
+                        } else {
+                            issue_a(U, m + 1, chunk_noisy(ci + 1));
+                        }
                     }
                     __syncwarp();
                 }
@@ -1295,8 +1023,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             }
             fence_async_smem();
             tc_fence_before();
-            bar_all();
-            if (s_abort) break;
+            if ((stop = abort_check())) break;
 
             // ================= S3 =================
             if (tid == 0) {
@@ -1309,10 +1036,14 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                         mma_bf16(tb + TM_N, dK_nk + ((kk * 32) >> 4), dM_v + ((kk * 2048) >> 4),
                                  make_idesc_bf16(128, 128, 0, 1), 1u);
                 }
-                mma_commit(&bar_mma);
-                if (!last) {
-                    if (!mbar_wait(&bar_mma, ph_mma & 1, kWaitIters)) fail(50);
-                    else issue_b(U, m + 1, chunk_noisy(ci + 1));
+                commit_mma();
+                if (!last && !dead) {
+                    if (!kwait<TW>(&bar_mma, ph_mma & 1, kWaitIters, P.wait_iters)) {
+                        dead = true;
+                        fail(50);
+                    } else {
+                        issue_b(U, m + 1, chunk_noisy(ci + 1));
+                    }
                 }
             }
             __syncwarp();
@@ -1363,41 +1094,27 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             }
             fence_async_smem();
             tc_fence_before();
-            bar_all();
             cb ^= 1;
-            if (s_abort) break;
+            if ((stop = abort_check())) break;
         }
-        if (s_abort) break;
+        if (stop) break;
     }
+    // Drain (a no-op unless a wait gave up; thread 0): every TMA phase issued but not seen complete
+    // is waited for, in order, with the normal bound (a phase's parity can repeat two phases later,
+    // so an in-order wait can only return late, never early); one more commit covers every MMA.
+    // Then the cp.async groups.
+    if (tid == 0) {
+        for (uint32_t p = ph_a; p < s_iss[0]; ++p) mbar_wait(&bar_a, p & 1, kDrainWaitIters);
+        for (uint32_t p = ph_b; p < s_iss[1]; ++p) mbar_wait(&bar_b, p & 1, kDrainWaitIters);
+        if (stop) {
+            mma_commit(&bar_drain);
+            mbar_wait(&bar_drain, 0, kDrainWaitIters);
+        }
+    }
+    cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tb, 512);
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult qr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-            qr == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 3-D map over a [rows, H, 128] bf16 tensor; box = 64 rows x 1 head x 64 columns, 128B swizzle.
-bool encode_map(CUtensorMap *m, const void *ptr, int H, int64_t rows) {
-    auto enc = get_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    cuuint32_t box[3] = {64, 1, 64};
-    cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -1406,9 +1123,11 @@ bool chunked_supported(int dtype, int d, int B, int conv_width) {
     return dtype == GDN_BF16 && d == D && (conv_width == 0 || conv_width == 4) && B >= 1 && B <= 32 && (32 % B) == 0;
 }
 
-cudaError_t launch_chunked(const Params &p, cudaStream_t stream) {
-    if (p.num_units == 0) return cudaSuccess;
-    if (p.V > 2 || p.T == 0) return cudaErrorNotSupported;
+namespace {
+
+// One launch over at most two noisy views: the pipelined kernel, or this file's in-order kernel.
+cudaError_t launch_chunked_views(const Params &p, bool pipelined, cudaStream_t stream) {
+    if (pipelined) return launch_pipe(p, stream);
     Maps maps;
     const bool noisy = p.V > 0 && p.TR > 0;
     if (!encode_map(&maps.q, p.q, p.H, p.T) || !encode_map(&maps.k, p.k, p.H, p.T) ||
@@ -1432,7 +1151,8 @@ cudaError_t launch_chunked(const Params &p, cudaStream_t stream) {
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
         cudaError_t e = cudaSuccess;
         for (auto fn : {gdn_chunked_kernel<1>, gdn_chunked_kernel<2>, gdn_chunked_kernel<4>,
-                        gdn_chunked_kernel<8>, gdn_chunked_kernel<16>, gdn_chunked_kernel<32>}) {
+                        gdn_chunked_kernel<8>, gdn_chunked_kernel<16>, gdn_chunked_kernel<32>,
+                        gdn_chunked_kernel<4, true>}) {
             cudaError_t r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
             if (r != cudaSuccess) e = r;
         }
@@ -1444,6 +1164,11 @@ cudaError_t launch_chunked(const Params &p, cudaStream_t stream) {
     Params q = p;
     q.parts = (noisy && 2 * p.num_units <= sms) ? 2 : 1;
     const int grid = std::min(p.num_units * q.parts, sms);
+    if (p.wait_test) {           // the test entry point: B = 4 only
+        if (p.B != 4) return cudaErrorNotSupported;
+        gdn_chunked_kernel<4, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);
+        return cudaGetLastError();
+    }
     switch (p.B) {
         case 1: gdn_chunked_kernel<1><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
         case 2: gdn_chunked_kernel<2><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
@@ -1454,6 +1179,36 @@ cudaError_t launch_chunked(const Params &p, cudaStream_t stream) {
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunked(const Params &p, bool pipelined, cudaStream_t stream) {
+    if (p.num_units == 0) return cudaSuccess;
+    // Every document empty: nothing to read, and each final state is the zero initial state.
+    if (p.T == 0) return cudaMemsetAsync(p.final_state, 0, (size_t)p.num_units * D * D * sizeof(float), stream);
+    if (p.V <= 2) return launch_chunked_views(p, pipelined, stream);
+    // More than two views: one launch per pair of views.  Each launch recomputes the clean
+    // stream (the views only share the clean boundary states) and rewrites the same clean
+    // outputs; the work counter in the workspace restarts at zero for every launch.
+    const int64_t row = p.TR * p.H;          // elements of one view's [T_R, H] plane
+    for (int v0 = 0; v0 < p.V; v0 += 2) {
+        Params q = p;
+        q.V = std::min(2, p.V - v0);
+        q.qn = static_cast<const __nv_bfloat16 *>(p.qn) + v0 * row * D;
+        q.kn = static_cast<const __nv_bfloat16 *>(p.kn) + v0 * row * D;
+        q.vn = static_cast<const __nv_bfloat16 *>(p.vn) + v0 * row * D;
+        q.gn = p.gn + v0 * row;
+        q.betan = p.betan + v0 * row;
+        q.out_noisy = static_cast<__nv_bfloat16 *>(p.out_noisy) + v0 * row * D;
+        if (v0 > 0) {
+            cudaError_t e = cudaMemsetAsync(&p.ws->next_unit, 0, sizeof(int32_t), stream);
+            if (e != cudaSuccess) return e;
+        }
+        cudaError_t e = launch_chunked_views(q, pipelined, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace gdn

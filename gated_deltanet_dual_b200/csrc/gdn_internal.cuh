@@ -14,6 +14,13 @@ namespace gdn {
 // host-to-device copy and no allocation.  1024 documents keep the parameter block ~16 KB.
 constexpr int kMaxDocs = 1024;
 
+// Iteration bound of every device-side mbarrier wait (each iteration is one try_wait, which
+// itself may suspend the thread for a while), and of the drain of outstanding copies and MMAs
+// after a wait gave up.  Kernels take the bound of their ordinary waits from their parameters,
+// so that a test can make a wait give up on purpose.
+constexpr uint32_t kWaitIters = 1u << 22;
+constexpr uint32_t kDrainWaitIters = 1u << 22;
+
 // Device-side status words at the start of the workspace.
 struct WorkspaceHeader {
     int32_t status;         // GDN_OK or GDN_ERR_TIMEOUT, written by kernels
@@ -36,6 +43,8 @@ struct Params {
     int32_t N, H, dk, dv, V, B, conv_width, num_units;
     int32_t parts;                    // chunked kernel: CTAs per unit (1, or 2 when units are few)
     float scale;                      // 1 / sqrt(d_k)
+    uint32_t wait_iters;              // test entry point only: bound of the mbarrier waits, in polls
+    uint32_t wait_test;               // 1: launch the kernels' test instantiation (polling waits)
     int32_t doc_start[kMaxDocs + 1];  // token offset of each document (doc_offsets)
     int32_t doc_prompt[kMaxDocs];     // prompt length of each document
     int32_t resp_off[kMaxDocs + 1];   // first packed noisy row of each document
@@ -44,7 +53,10 @@ struct Params {
 
 // Launchers (one per kernel family).  Return a CUDA error code; the caller maps it.
 cudaError_t launch_sequential(const Params &p, int dtype, cudaStream_t stream);
-cudaError_t launch_chunked(const Params &p, cudaStream_t stream);
+// pipelined: the warp-specialised variant (no ShortConv), else the in-order kernel.
+cudaError_t launch_chunked(const Params &p, bool pipelined, cudaStream_t stream);
+// The warp-specialised pipelined variant of the chunked kernel (no ShortConv, at most two views).
+cudaError_t launch_pipe(const Params &p, cudaStream_t stream);
 // Route I: clean chain writing block-boundary states into `states`, then block refinement.
 cudaError_t launch_route1(const Params &p, int dtype, float *states, cudaStream_t stream);
 bool chunked_supported(int dtype, int d, int B, int conv_width);

@@ -44,12 +44,59 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait on the phase with the given parity.  Returns false if it gave up.
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on the phase with the given parity.  Returns false if it gave up.  Each iteration is
+// one try_wait, which may itself suspend the thread for a while.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t max_iters) {
     for (uint32_t it = 0; it < max_iters; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
     }
     return false;
+}
+
+// The same bound made of non-blocking test_waits: a small bound gives up as soon as the phase is
+// not complete (the kernels' test instantiations, which exercise the give-up path).
+__device__ __forceinline__ bool mbar_poll(uint64_t *bar, uint32_t parity, uint32_t max_iters) {
+    for (uint32_t it = 0; it < max_iters; ++it) {
+        if (mbar_test_wait(bar, parity)) return true;
+    }
+    return false;
+}
+
+// The wait of a kernel instantiation: the normal bound with try_wait, or (TW, test instantiations)
+// the caller's bound with polls.
+template <bool TW>
+__device__ __forceinline__ bool kwait(uint64_t *bar, uint32_t parity, uint32_t normal_iters, uint32_t test_iters) {
+    if constexpr (TW) return mbar_poll(bar, parity, test_iters);
+    else return mbar_wait(bar, parity, normal_iters);
+}
+
+// ------------------------------------------------------------------ named barriers
+// bar.sync on named barrier `id` over `nthreads` threads that also ORs `pred` across them: every
+// participating thread gets the same result, so a decision taken on it (leave a loop) is uniform.
+__device__ __forceinline__ bool bar_sync_or(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
 
 // ------------------------------------------------------------------ proxies / fences

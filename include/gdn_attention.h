@@ -67,6 +67,16 @@ gdn_status gdn_attn_forward(const gdn_attn_desc *desc, const void *q, const void
                             void *out, void *out_noisy, void *workspace, size_t workspace_bytes,
                             gdn_stream_t stream);
 
+/* FOR TESTS of the bounded-wait error path only: gdn_attn_forward with every device-side wait
+ * bounded by `wait_iters` non-blocking polls (>= 1).  A wait that gives up records
+ * GDN_ERR_TIMEOUT in the workspace; the kernel then waits with the normal bound for every copy
+ * and MMA it issued before it leaves; outputs are unspecified.  (No counterpart in the notes.) */
+gdn_status gdn_attn_forward_test_wait_limit(const gdn_attn_desc *desc, const void *q, const void *k,
+                                            const void *v, const void *qn, const void *kn, const void *vn,
+                                            const int32_t *doc_offsets, const int32_t *prompt_len,
+                                            void *out, void *out_noisy, void *workspace, size_t workspace_bytes,
+                                            uint32_t wait_iters, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

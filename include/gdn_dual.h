@@ -40,7 +40,8 @@
  * Errors: every entry point returns a gdn_status.  Bad arguments are rejected on the host
  * before anything is enqueued (no partial writes).  CUDA launch failures return
  * GDN_ERR_CUDA.  Device code never traps or asserts; bounded waits inside kernels record
- * GDN_ERR_TIMEOUT in the workspace (see gdn_dual_read_device_status).
+ * GDN_ERR_TIMEOUT in the workspace (see gdn_dual_read_device_status); a kernel whose wait gave
+ * up first waits for every copy and MMA it had issued, then leaves.
  */
 #ifndef GDN_DUAL_H
 #define GDN_DUAL_H
@@ -64,17 +65,24 @@ typedef enum {
 typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 
 typedef enum {
-    GDN_ALGO_AUTO = 0,        /* chunked tensor-core kernel when supported, else sequential */
+    GDN_ALGO_AUTO = 0,        /* the in-order chunked kernel when supported, else the sequential one */
     GDN_ALGO_SEQUENTIAL = 1,  /* token-sequential CUDA-core kernel, fp32 state (any dtype) */
-    GDN_ALGO_CHUNKED = 2,     /* chunked WY/UT tcgen05 kernel (bf16, d_k = d_v = 128) */
-    GDN_ALGO_ROUTE1 = 3       /* chunk-then-refine (Route I of the notes, Key design 2), a measured
+    GDN_ALGO_CHUNKED = 2,     /* chunked WY/UT tcgen05 kernel, chunks in order (bf16,
+                                 d_k = d_v = 128, B | 32, ShortConv off or width 4) */
+    GDN_ALGO_ROUTE1 = 3,      /* chunk-then-refine (Route I of the notes, Key design 2), a measured
                                  comparison: a clean pass writes the state before every response
                                  block into the workspace, then each (view, block) is refined from
                                  its stored state; CUDA cores; no ShortConv; never chosen by AUTO */
+    GDN_ALGO_PIPELINED = 4    /* the chunked WY/UT tcgen05 kernel pipelined across chunks: helper
+                                 warps prepare chunk c+1's state-independent products (the
+                                 triangular solve among them) while the main warps run chunk c's
+                                 state chain (bf16, d_k = d_v = 128, B | 32, no ShortConv); a
+                                 measured alternative, slower than GDN_ALGO_CHUNKED on B200, never
+                                 chosen by AUTO */
 } gdn_algo;
 
 /* Problem descriptor.  num_docs N >= 1; num_heads H >= 1; d_k == d_v in {32, 64, 128};
- * num_views V in [0, 8]; block_size B >= 1 (the chunked kernel needs B | 64); dtype a
+ * num_views V in [0, 8]; block_size B >= 1 (the chunked kernel needs B | 32); dtype a
  * gdn_dtype; conv_width 0 (off) or 4; algo a gdn_algo; reserved must be 0. */
 typedef struct {
     int32_t num_docs;
@@ -175,7 +183,13 @@ gdn_status gdn_dual_backward(const gdn_dual_desc *desc,
  *   Sharing: all calls on a device share the array, which keeps the last call's contents; the
  *     status words are cleared on `stream` at the start of every call.  Calls whose work
  *     overlaps on the GPU (e.g. on two streams at once) race on the array: serialise them.
- *   Errors: as gdn_dual_forward, plus GDN_ERR_CUDA if the set-up lookup fails.
+ *     The address is kept per device ordinal for the life of the process, so it belongs to the
+ *     device's primary context (the CUDA runtime's); do not call this from another context, or
+ *     after cudaDeviceReset.
+ *   Errors: as gdn_dual_forward, plus GDN_ERR_CUDA if the set-up lookup fails, and
+ *     GDN_ERR_UNSUPPORTED for GDN_ALGO_ROUTE1 (its block-boundary states need far more scratch
+ *     than the array holds).  A bounded device-side wait that gives up is recorded in the array,
+ *     not returned here: read it with gdn_dual_noalloc_read_device_status.
  */
 gdn_status gdn_dual_forward_noalloc(const gdn_dual_desc *desc,
                                     const void *q, const void *k, const void *v,
@@ -187,10 +201,38 @@ gdn_status gdn_dual_forward_noalloc(const gdn_dual_desc *desc,
                                     void *out, void *out_noisy, float *final_state,
                                     gdn_stream_t stream);
 
+/* The device-side status recorded by the last gdn_dual_forward_noalloc on the current device
+ * (GDN_OK or GDN_ERR_TIMEOUT): synchronises `stream` and reads the status word at the start of
+ * the library's fixed scratch array.  No allocation.  (The FLARE notes have no counterpart.) */
+gdn_status gdn_dual_noalloc_read_device_status(gdn_stream_t stream);
+
 /* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
  * last gdn_dual_forward on it (GDN_OK or GDN_ERR_TIMEOUT), or GDN_ERR_CUDA if the sync fails.
  * For debugging and tests; the forward path itself never synchronises. */
 gdn_status gdn_dual_read_device_status(const void *workspace, gdn_stream_t stream);
+
+/* As gdn_dual_read_device_status, and, when `where` is not NULL, stores the diagnostic code of
+ * the wait that gave up (0 when none did). */
+gdn_status gdn_dual_read_device_status_where(const void *workspace, int32_t *where, gdn_stream_t stream);
+
+/* FOR TESTS of the bounded-wait error path only: gdn_dual_forward with every device-side
+ * mbarrier wait bounded by `wait_iters` non-blocking polls (>= 1) instead of the library's
+ * normal bound.  A tiny bound makes a wait give up while its copy or MMA is still in flight: the
+ * kernel then records GDN_ERR_TIMEOUT (and where) in the workspace, waits with the normal bound
+ * for every copy and MMA it has issued, and leaves; outputs are unspecified.  The next ordinary
+ * call is unaffected.  The tensor-core kernels have this test variant for B = 4 only (other block
+ * sizes on them: GDN_ERR_UNSUPPORTED).  (The FLARE notes have no counterpart: this exercises the failure
+ * detection of this library.) */
+gdn_status gdn_dual_forward_test_wait_limit(const gdn_dual_desc *desc,
+                                            const void *q, const void *k, const void *v,
+                                            const float *g, const float *beta,
+                                            const void *qn, const void *kn, const void *vn,
+                                            const float *gn, const float *betan,
+                                            const int32_t *doc_offsets, const int32_t *prompt_len,
+                                            const float *conv_w,
+                                            void *out, void *out_noisy, float *final_state,
+                                            void *workspace, size_t workspace_bytes,
+                                            uint32_t wait_iters, gdn_stream_t stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gdn_status_string(gdn_status status);

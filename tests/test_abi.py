@@ -375,3 +375,25 @@ def test_backward_more_documents_than_supported():
     st = lib.gdn_dual_backward(ctypes.byref(d), *ptr[:10], offs.ctypes.data_as(ip), pl.ctypes.data_as(ip),
                                *ptr[10:23], ptr[23], ctypes.c_size_t(nb), None)
     assert st == b.GDN_ERR_UNSUPPORTED
+
+
+def test_noalloc_rejects_route1_and_invalid_descriptors():
+    """The no-allocation entry point refuses on the host, before any device work: Route I (its
+    block-boundary states need far more than the fixed scratch array) is GDN_ERR_UNSUPPORTED, a
+    NULL or invalid descriptor GDN_ERR_INVALID_ARG."""
+    lib = b.load_library()
+    offs = np.array([0, 64], np.int32)
+    pl = np.array([32], np.int32)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    fn = lib.gdn_dual_forward_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.POINTER(b.Desc)] + [ctypes.c_void_p] * 10 + [ip, ip] + [ctypes.c_void_p] * 5
+
+    def call(desc):
+        ref = None if desc is None else ctypes.byref(desc)
+        return fn(ref, *([None] * 10), offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), *([None] * 5))
+
+    assert call(b.make_desc(1, 2, 128, 128, 2, 4, b.GDN_BF16, algo=b.ALGO_ROUTE1)) == b.GDN_ERR_UNSUPPORTED
+    assert call(None) == b.GDN_ERR_INVALID_ARG
+    assert call(b.make_desc(1, 2, 128, 128, 9, 4, b.GDN_BF16)) == b.GDN_ERR_INVALID_ARG    # views > 8
+    assert call(b.make_desc(0, 2, 128, 128, 2, 4, b.GDN_BF16)) == b.GDN_ERR_INVALID_ARG    # no documents
