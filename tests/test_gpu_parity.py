@@ -59,8 +59,9 @@ def test_head_dims_and_dtypes(d, dtype):
 
 
 def algos_for(conv):
-    """Both kernels implement bf16 d=128 problems, with or without the ShortConv prologue."""
-    return [b.ALGO_SEQUENTIAL, b.ALGO_CHUNKED]
+    """The sequential and the in-order chunked kernels implement bf16 d=128 problems with or without
+    the ShortConv prologue; the pipelined chunked kernel without it."""
+    return [b.ALGO_SEQUENTIAL, b.ALGO_CHUNKED] + ([b.ALGO_PIPELINED] if conv == 0 else [])
 
 
 @pytest.mark.parametrize("B", [1, 2, 4, 8, 16, 32])
@@ -82,10 +83,35 @@ def test_view_counts(V):
     check(prob, "fp32", b.ALGO_AUTO)
 
 
+@pytest.mark.parametrize("algo", [b.ALGO_CHUNKED, b.ALGO_PIPELINED])
 @pytest.mark.parametrize("V", [0, 1, 2])
-def test_view_counts_chunked(V):
+def test_view_counts_chunked(V, algo):
     prob = small([200, 136], [72, 8], H=2, d=128, V=V, dtype="bf16", seed=20 + V)
-    check(prob, "bf16", b.ALGO_CHUNKED)
+    check(prob, "bf16", algo)
+
+
+@pytest.mark.parametrize("V", [3, 8])
+@pytest.mark.parametrize("conv", [0, 4])
+def test_more_than_two_views_auto(V, conv):
+    """V = 3 and V = 8 (the header's maximum) at bf16, d = 128, algo AUTO: the tensor-core kernel
+    is selected and runs the views in pairs."""
+    prob = small([200, 136], [72, 8], H=2, d=128, V=V, dtype="bf16", conv=conv, seed=30 + V + conv)
+    desc = b.make_desc(prob.num_docs, 2, 128, 128, V, 4, b.GDN_BF16, conv)
+    assert b.select_algo(desc) == b.ALGO_CHUNKED
+    check(prob, "bf16", b.ALGO_AUTO)
+    if conv == 0:
+        check(prob, "bf16", b.ALGO_PIPELINED)
+
+
+@pytest.mark.parametrize("d,dtype", [(128, "bf16"), (32, "fp32")])
+def test_all_documents_empty(d, dtype):
+    """Every document empty (T = 0 with N x H > 0): GDN_OK and zero final states."""
+    prob = small([0, 0, 0], [0, 0, 0], H=2, d=d, dtype=dtype)
+    fs = torch.full((3, 2, d, d), float("nan"), device="cuda")
+    ws = b.Workspace(256)
+    _, _, fs = b.forward_problem(prob, final_state=fs, workspace=ws)
+    assert b.read_device_status(ws) == b.GDN_OK
+    assert bool((fs == 0).all())
 
 
 @pytest.mark.parametrize("conv", [0, 4])
@@ -106,20 +132,22 @@ def test_strong_gates_and_large_beta():
         check(prob, "bf16", algo)
 
 
+@pytest.mark.parametrize("algo", [b.ALGO_CHUNKED, b.ALGO_PIPELINED])
 @pytest.mark.parametrize("B", [4, 16, 32])
-def test_extreme_gates_take_the_exact_decay_paths(B):
+def test_extreme_gates_take_the_exact_decay_paths(B, algo):
     """g ~ U(-8, 0): a chunk's cumulative decay leaves the range in which e^{gamma_t - gamma_i}
     factorises as E_t F_i (|gamma| >= 100 in log2 units), so the chunked kernel exponentiates every
     difference (P and A rows, M'_Z and, for B >= 16, the noisy block coefficients)."""
     prob = small([640, 384], [128, 64], H=2, d=128, B=B, dtype="bf16", seed=41 + B, g_lo=-8.0)
-    check(prob, "bf16", b.ALGO_CHUNKED)
+    check(prob, "bf16", algo)
 
 
-def test_chunked_matches_sequential_kernel():
-    """The two CUDA kernels agree with each other on a multi-unit problem (both fp32 state)."""
+@pytest.mark.parametrize("algo", [b.ALGO_CHUNKED, b.ALGO_PIPELINED])
+def test_chunked_matches_sequential_kernel(algo):
+    """The CUDA kernels agree with each other on a multi-unit problem (all fp32 state)."""
     prob = small([1000, 1536, 520], [232, 512, 8], H=4, d=128, B=4, dtype="bf16", seed=31)
     a = [t.float().clone() for t in b.forward_problem(prob, algo=b.ALGO_SEQUENTIAL)]
-    c = [t.float().clone() for t in b.forward_problem(prob, algo=b.ALGO_CHUNKED)]
+    c = [t.float().clone() for t in b.forward_problem(prob, algo=algo)]
     torch.cuda.synchronize()
     for x, y in zip(a, c):
         assert float((x - y).abs().max()) <= 2e-2 * float(x.abs().max())
