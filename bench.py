@@ -33,17 +33,19 @@ from gated_deltanet_dual_b200 import binding as gb  # noqa: E402
 from gated_deltanet_dual_b200 import replicas  # noqa: E402
 from gated_deltanet_dual_b200 import synth  # noqa: E402
 
-DEFAULT_WORKLOAD = "train_8x4096_h16_d128"
+DEFAULT_WORKLOAD = "large_32x8192_h32_d128"   # the largest single-GPU workload
 METRIC = "dual-stream GDN fwd tokens/s on 1 B200 and % of roofline (HBM/tensor)"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = {
     gb.ALGO_SEQUENTIAL: ["gated_deltanet_dual_b200/csrc/gdn_sequential.cu"],
-    gb.ALGO_CHUNKED: ["gated_deltanet_dual_b200/csrc/gdn_chunked.cu"],
+    gb.ALGO_CHUNKED: ["gated_deltanet_dual_b200/csrc/gdn_chunked.cu", "gated_deltanet_dual_b200/csrc/gdn_chunk_common.cuh"],
+    gb.ALGO_PIPELINED: ["gated_deltanet_dual_b200/csrc/gdn_pipe.cu", "gated_deltanet_dual_b200/csrc/gdn_chunk_common.cuh"],
     gb.ALGO_ROUTE1: ["gated_deltanet_dual_b200/csrc/gdn_decode.cu"],
     "attention": ["gated_deltanet_dual_b200/csrc/gdn_attention.cu"],
 }
 KERNEL_NAMES = {gb.ALGO_SEQUENTIAL: "gdn_sequential_kernel", gb.ALGO_CHUNKED: "gdn_chunked_kernel",
+                gb.ALGO_PIPELINED: "gdn_pipe_kernel",
                 gb.ALGO_ROUTE1: "gdn_route1_chain_kernel + gdn_decode_kernel (block end)",
                 "attention": "gdn_attention_kernel"}
 
@@ -86,16 +88,24 @@ def kernel_hash(algo) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(algo, workload):
+def profiled_traffic(algo, workload, alg_bytes=None):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
-    kernel source (same hash) for this workload; else None."""
+    kernel source (same hash) for this workload; else None.  A record may instead name a
+    smaller captured workload of the same kernel (`scaled_from`, for a workload too large to
+    capture): its traffic is then scaled by the ratio of the two workloads' algorithmic bytes."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     try:
-        rec = json.load(open(path)).get(f"{KERNEL_NAMES[algo]}:{workload}")
+        recs = json.load(open(path))
     except Exception:
         return None
+    rec = recs.get(f"{KERNEL_NAMES[algo]}:{workload}")
+    if rec and rec.get("scaled_from") and alg_bytes:
+        src = recs.get(f"{KERNEL_NAMES[algo]}:{rec['scaled_from']}")
+        if not src or src.get("kernel_hash") != kernel_hash(algo) or not src.get("algorithmic_bytes"):
+            return None
+        return int(src["dram_bytes_per_launch"] * alg_bytes / src["algorithmic_bytes"])
     if not rec or rec.get("kernel_hash") != kernel_hash(algo):
         return None
     return rec.get("dram_bytes_per_launch")
@@ -786,7 +796,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--algo", default="auto", choices=["auto", "sequential", "chunked", "route1"])
+    ap.add_argument("--algo", default="auto", choices=["auto", "sequential", "chunked", "route1", "pipelined"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -811,7 +821,7 @@ def main():
     dev = torch.device("cuda", local)
     replicas.init(world, backend="nccl", device=dev)
     algo = {"auto": gb.ALGO_AUTO, "sequential": gb.ALGO_SEQUENTIAL, "chunked": gb.ALGO_CHUNKED,
-            "route1": gb.ALGO_ROUTE1}[args.algo]
+            "route1": gb.ALGO_ROUTE1, "pipelined": gb.ALGO_PIPELINED}[args.algo]
 
     prob = synth.make_problem(wl, seed=replicas.replica_seed(0, rank), device=dev)
     T, TR, V, H, d = prob.T, prob.T_R, prob.num_views, prob.num_heads, prob.d_k
@@ -863,7 +873,7 @@ def main():
     value = replicas.throughput(prob.tokens(), world, args.steps, elapsed_ms)
     peaks = measured_peaks()
     achieved_gbs = work["bytes"] / (kernel_ms / 1e3) / 1e9
-    traffic = profiled_traffic(used_algo, wl.name)
+    traffic = profiled_traffic(used_algo, wl.name, work["bytes"])
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
                 "peak_source": peaks["source"], "kernel": KERNEL_NAMES.get(used_algo),
@@ -911,8 +921,8 @@ def main():
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        max_units = units_for_seconds(wl, target_s=10.0)
-        cb = time_oracle(wl, steps=1, warmup=0, max_units=max_units)
+        max_units = units_for_seconds(wl, target_s=8.0)
+        cb = time_oracle(wl, steps=1, warmup=1, max_units=max_units)
         cpu_baseline = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
     replicas.shutdown(world)
@@ -924,7 +934,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": wl.name, "docs": prob.num_docs, "tokens_clean": T, "tokens_noisy": V * TR,
                        "heads": H, "d": d, "block_size": prob.block_size, "views": V, "conv_width": prob.conv_width,
-                       "algo": {1: "sequential", 2: "chunked", 3: "route1"}.get(used_algo, str(used_algo)),
+                       "algo": {1: "sequential", 2: "chunked", 3: "route1", 4: "pipelined"}.get(used_algo, str(used_algo)),
                        "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush)"},
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks.summary(),
