@@ -26,7 +26,8 @@ EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device
             "gdn_attn_forward", "gdn_attn_workspace_size", "gdn_dual_backward",
             "gdn_dual_backward_workspace_size", "gdn_dual_forward_noalloc",
             "gdn_dual_noalloc_read_device_status", "gdn_dual_forward_test_wait_limit",
-            "gdn_dual_read_device_status_where", "gdn_attn_forward_test_wait_limit")
+            "gdn_dual_read_device_status_where", "gdn_attn_forward_test_wait_limit",
+            "gdn_dual_backward_conv", "gdn_dual_backward_conv_workspace_size")
 
 
 class GdnError(RuntimeError):
@@ -478,10 +479,11 @@ def backward_workspace_size(desc: Desc, doc_offsets) -> int:
 
 
 def backward(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, block_size, d_out, d_out_noisy,
-             d_final_state=None, *, workspace=None, stream=None):
+             d_final_state=None, *, conv_w=None, workspace=None, stream=None):
     """Gradients of <d_out, out> + <d_out_noisy, out_noisy> + <d_final_state, final_state> with
-    respect to every input of the dual-stream forward (gdn_dual_backward), fp32.  Returns a dict
-    dq, dk, dv, dg, dbeta, dqn, dkn, dvn, dgn, dbetan."""
+    respect to every input of the dual-stream forward, fp32 (gdn_dual_backward; with conv_w, the
+    width-4 ShortConv prologue: gdn_dual_backward_conv, gradients of the raw inputs plus dconv_w).
+    Returns a dict dq, dk, dv, dg, dbeta, dqn, dkn, dvn, dgn, dbetan (and dconv_w)."""
     dev = q.device
     if dev.type != "cuda":
         raise ValueError("inputs must be CUDA tensors")
@@ -504,25 +506,49 @@ def backward(q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, b
                                (d_out_noisy, "d_out_noisy", (V, TR, H, dv_), io),
                                (d_final_state, "d_final_state", (N, H, dk_, dv_), f32)):
         _check(t, name, shape, dt, dev)
+    conv_width = 0
+    if conv_w is not None:
+        conv_width = int(conv_w.shape[-1])
+        _check(conv_w, "conv_w", (3, H * dk_, conv_width), f32, dev)
     out = {n: torch.empty(x.shape, dtype=f32, device=dev) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dg", g),
                                                                          ("dbeta", beta), ("dqn", qn), ("dkn", kn),
                                                                          ("dvn", vn), ("dgn", gn), ("dbetan", betan))}
-    desc = make_desc(N, H, dk_, dv_, V, int(block_size), _dtype_code(q))
+    desc = make_desc(N, H, dk_, dv_, V, int(block_size), _dtype_code(q), conv_width)
+    lib = load_library()
     ws = workspace
     if ws is None:
-        nbytes = backward_workspace_size(desc, offs)
+        nbytes = backward_workspace_size(desc, offs) if conv_w is None else backward_conv_workspace_size(desc, offs)
         if nbytes:
             ws = Workspace(nbytes, device=dev).tensor
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     noisy = V > 0 and TR > 0
     nz = lambda t: _ptr(t) if noisy else None
     ip = ctypes.POINTER(ctypes.c_int32)
-    st = load_library().gdn_dual_backward(
-        ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), nz(qn), nz(kn), nz(vn), nz(gn), nz(betan),
-        offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(d_out), nz(d_out_noisy), _ptr(d_final_state),
-        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
-        nz(out["dqn"]), nz(out["dkn"]), nz(out["dvn"]), nz(out["dgn"]), nz(out["dbetan"]),
-        _ptr(ws), ctypes.c_size_t(ws_bytes), _stream(stream))
+    head = [ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), nz(qn), nz(kn), nz(vn), nz(gn),
+            nz(betan), offs.ctypes.data_as(ip), pl.ctypes.data_as(ip)]
+    grads = [_ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+             nz(out["dqn"]), nz(out["dkn"]), nz(out["dvn"]), nz(out["dgn"]), nz(out["dbetan"])]
+    ups = [_ptr(d_out), nz(d_out_noisy), _ptr(d_final_state)]
+    if conv_w is None:
+        st = lib.gdn_dual_backward(*head, *ups, *grads, _ptr(ws), ctypes.c_size_t(ws_bytes), _stream(stream))
+        name = "gdn_dual_backward"
+    else:
+        out["dconv_w"] = torch.empty_like(conv_w)
+        fn = lib.gdn_dual_backward_conv
+        fn.restype = ctypes.c_int
+        vp = ctypes.c_void_p
+        fn.argtypes = [ctypes.POINTER(Desc)] + [vp] * 10 + [ip, ip] + [vp] * 4 + [vp] * 10 + [vp, vp, ctypes.c_size_t, vp]
+        st = fn(*head, _ptr(conv_w), *ups, *grads, _ptr(out["dconv_w"]), _ptr(ws), ctypes.c_size_t(ws_bytes),
+                _stream(stream))
+        name = "gdn_dual_backward_conv"
     if st != GDN_OK:
-        raise GdnError(st, f"gdn_dual_backward failed: {status_string(st)}")
+        raise GdnError(st, f"{name} failed: {status_string(st)}")
     return out
+
+
+def backward_conv_workspace_size(desc: Desc, doc_offsets) -> int:
+    offs = np.ascontiguousarray(doc_offsets, dtype=np.int32)
+    fn = load_library().gdn_dual_backward_conv_workspace_size
+    fn.restype = ctypes.c_size_t
+    fn.argtypes = [ctypes.POINTER(Desc), ctypes.POINTER(ctypes.c_int32)]
+    return int(fn(ctypes.byref(desc), offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))))

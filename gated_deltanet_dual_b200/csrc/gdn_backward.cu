@@ -15,7 +15,9 @@
 // Lam.  One CTA takes one (document, head, slice of 32 columns); two threads per column hold half
 // of its rows of S and of Lam in registers (a pair shuffle completes the k^T S and k^T Lam dot
 // products).  Gradients that sum over columns (dq, dk, dg, dbeta) are reduced over the CTA's 32
-// columns in shared memory and added into the fp32 outputs with atomics (one add per slice).
+// columns in shared memory and stored as the slice's partial in the workspace; a second kernel
+// adds the d/32 partials of every element in slice order, so the results are the same on every
+// call (no atomics).
 //   pass 1: the clean chain, writing the state before every 16th token into the workspace
 //   pass 2: 16-token segments from the last: the segment's states are rebuilt from its
 //           checkpoint, 4 tokens at a time into shared memory, and the adjoint runs backwards
@@ -23,6 +25,7 @@
 //           is rebuilt from that token's state (token by token, from the start for every step)
 //           and run backwards, and its initial-state gradient joins Lam.
 // The work per token is a few dot products of length d per column: CUDA cores, not tensor cores.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -40,6 +43,7 @@ struct BwdParams {
     const float *g, *beta, *gn, *betan, *dsf;
     float *dq, *dk, *dv, *dg, *dbeta, *dqn, *dkn, *dvn, *dgn, *dbetan;
     float *ck;                        // checkpoints [ck index][H][slice][R2][64]
+    int64_t pst_vec, pst_sc, pst_nvec, pst_nsc;   // slice strides of the partial buffers (floats)
     int64_t TR;
     int32_t N, H, V, B;
     float scale;
@@ -75,6 +79,11 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
     const int roff = P.resp_off[n];
     const float sc = P.scale;
     auto at = [&](float *buf, int i) -> float & { return buf[i * kBwdThreads + tid]; };
+    // this slice's partial buffers (P.dq ... point at slice 0)
+    float *const pdq = P.dq + js * P.pst_vec, *const pdk = P.dk + js * P.pst_vec;
+    float *const pdg = P.dg + js * P.pst_sc, *const pdbeta = P.dbeta + js * P.pst_sc;
+    float *const pdqn = P.dqn + js * P.pst_nvec, *const pdkn = P.dkn + js * P.pst_nvec;
+    float *const pdgn = P.dgn + js * P.pst_nsc, *const pdbetan = P.dbetan + js * P.pst_nsc;
 
     // this thread's rows of a k or q vector (clean row, or noisy packed row), as 16-byte loads
     // (the rows start 32-byte aligned: D >= 32 and the tensors are 16-byte aligned)
@@ -123,11 +132,11 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
             for (int cc = 0; cc < 32; ++cc) a4[cc & 3] += red[cc * (D + 2) + r];
             const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
             if (r < D) {
-                if (out_vec) atomicAdd(out_vec + r, acc);
+                if (out_vec) out_vec[r] = acc;
             } else if (r == D) {
-                if (sc0) atomicAdd(sc0, acc);
+                if (sc0) *sc0 = acc;
             } else if (sc1) {
-                atomicAdd(sc1, acc);
+                *sc1 = acc;
             }
         }
         __syncthreads();
@@ -191,7 +200,7 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
                 kq(P.qn, row, qq);
 #pragma unroll
                 for (int i = 0; i < R2; ++i) lt[i] = fmaf(qq[i], dd * sc, lt[i]);
-                dq_rows(sw, dd, P.dqn + (row * H + h) * D);
+                dq_rows(sw, dd, pdqn + (row * H + h) * D);
             }
             // steps from the last: rebuild the state before step j from the block start
             for (int j = P.B - 1; j >= 0; --j) {
@@ -209,7 +218,7 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
                 bwd(lt, sw, kk, ld<TIO>(P.vn, (row * H + h) * D + col), expf(P.gn[row * H + h]),
                     P.betan[row * H + h], &dvc);
                 if (hf == 0) P.dvn[(row * H + h) * D + col] = dvc;
-                reduce_add(P.dkn + (row * H + h) * D, P.dgn + row * H + h, P.dbetan + row * H + h);
+                reduce_add(pdkn + (row * H + h) * D, pdgn + row * H + h, pdbetan + row * H + h);
             }
 #pragma unroll
             for (int i = 0; i < R2; ++i) at(lmb, i) += lt[i];
@@ -281,7 +290,7 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
                         lam[i] = at(lmb, i);
                     }
                 }
-                dq_rows(sp, dd, P.dq + (row * H + h) * D);
+                dq_rows(sp, dd, pdq + (row * H + h) * D);
                 // the state before token t
 #pragma unroll
                 for (int i = 0; i < R2; ++i) sp[i] = at(seg, (t - u0) * R2 + i);
@@ -290,7 +299,7 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
                 bwd(lam, sp, kk, ld<TIO>(P.v, (row * H + h) * D + col), expf(P.g[row * H + h]),
                     P.beta[row * H + h], &dvc);
                 if (hf == 0) P.dv[(row * H + h) * D + col] = dvc;
-                reduce_add(P.dk + (row * H + h) * D, P.dg + row * H + h, P.dbeta + row * H + h);
+                reduce_add(pdk + (row * H + h) * D, pdg + row * H + h, pdbeta + row * H + h);
             }
         }
     }
@@ -303,6 +312,23 @@ gdn_backward_kernel(const __grid_constant__ BwdParams P) {
         }
         noisy_block(0, sp, lam);
     }
+}
+
+// out[i] = sum over the ns slice partials part[s * stride + i], in slice order.
+__global__ void reduce_slices_kernel(const float *__restrict__ part, float *__restrict__ out, int64_t n,
+                                     int64_t stride, int ns) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = part[i];
+        for (int s = 1; s < ns; ++s) acc += part[s * stride + i];
+        out[i] = acc;
+    }
+}
+
+cudaError_t reduce_slices(const float *part, float *out, int64_t n, int64_t stride, int ns, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
+    reduce_slices_kernel<<<(unsigned)blocks, 256, 0, st>>>(part, out, n, stride, ns);
+    return cudaGetLastError();
 }
 
 template <typename TIO, int D>
@@ -325,6 +351,14 @@ int64_t bwd_checkpoints(const gdn_dual_desc *d, const int32_t *offs) {
     return nck;
 }
 
+// Partial buffers of the column-summed gradients: per slice, [dq | dk] (T H d each), [dg | dbeta]
+// (T H each), and for the noisy stream the same over V T rows (T_R <= T: the size needs no prompt
+// lengths).  Returns floats per slice; *strides gets the four per-slice offsets and strides.
+int64_t bwd_partial_floats(const gdn_dual_desc *d, int64_t T) {
+    const int64_t th = T * d->num_heads, V = d->num_views;
+    return 2 * th * d->d_k + 2 * th + (V > 0 ? 2 * V * th * d->d_k + 2 * V * th : 0);
+}
+
 bool bwd_desc_ok(const gdn_dual_desc *d) {
     return d && d->num_docs >= 1 && d->num_heads >= 1 && d->d_k >= 1 && d->d_v >= 1 &&
            d->num_views >= 0 && d->block_size >= 1 && (d->dtype == GDN_BF16 || d->dtype == GDN_FP32) &&
@@ -334,6 +368,79 @@ bool bwd_desc_ok(const gdn_dual_desc *d) {
 }  // namespace
 }  // namespace gdn
 
+
+namespace gdn {
+
+// The backward on validated arguments: dtype is the element type of q, k, v, their noisy twins
+// and the upstream gradients (the ShortConv entry point passes fp32 copies).  The workspace holds
+// the checkpoints, then the slice partials.
+gdn_status run_backward(const gdn_dual_desc *desc, int dtype, const void *q, const void *k, const void *v,
+                        const float *g, const float *beta, const void *qn, const void *kn, const void *vn,
+                        const float *gn, const float *betan, const int32_t *doc_offsets, const int32_t *prompt_len,
+                        const void *d_out, const void *d_out_noisy, const float *d_final_state, float *dq,
+                        float *dk, float *dv, float *dg, float *dbeta, float *dqn, float *dkn, float *dvn,
+                        float *dgn, float *dbetan, void *workspace, cudaStream_t st) {
+    const int N = desc->num_docs, H = desc->num_heads, B = desc->block_size, D = desc->d_k;
+    int64_t TR = 0;
+    for (int n = 0; n < N; ++n) TR += (int64_t)doc_offsets[n + 1] - doc_offsets[n] - prompt_len[n];
+    const int64_t T = doc_offsets[N];
+    const bool noisy = desc->num_views > 0 && TR > 0;
+    const int ns = D / 32;
+    const int64_t nck = bwd_checkpoints(desc, doc_offsets);
+    float *ck = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + 256);
+    float *part = ck + nck * H * D * D;
+    const int64_t th = T * H, V = desc->num_views;
+    // slice-0 bases and slice strides of the partials (bwd_partial_floats layout)
+    const int64_t per_slice = bwd_partial_floats(desc, T);
+    float *p_dq = part, *p_dk = part + th * D, *p_dg = part + 2 * th * D, *p_dbeta = p_dg + th;
+    float *p_dqn = p_dbeta + th, *p_dkn = p_dqn + V * th * D, *p_dgn = p_dkn + V * th * D, *p_dbetan = p_dgn + V * th;
+
+    BwdParams P;
+    std::memset(&P, 0, sizeof(P));
+    P.q = q; P.k = k; P.v = v; P.qn = qn; P.kn = kn; P.vn = vn; P.dout = d_out; P.doutn = d_out_noisy;
+    P.g = g; P.beta = beta; P.gn = gn; P.betan = betan; P.dsf = d_final_state;
+    P.dq = p_dq; P.dk = p_dk; P.dv = dv; P.dg = p_dg; P.dbeta = p_dbeta;
+    P.dqn = p_dqn; P.dkn = p_dkn; P.dvn = dvn; P.dgn = p_dgn; P.dbetan = p_dbetan;
+    P.pst_vec = P.pst_sc = P.pst_nvec = P.pst_nsc = per_slice;
+    P.ck = ck;
+    P.TR = TR; P.N = N; P.H = H; P.V = noisy ? desc->num_views : 0; P.B = B;
+    P.scale = (float)(1.0 / std::sqrt((double)D));
+    int64_t roff = 0, ckn = 0;
+    for (int n = 0; n <= N; ++n) {
+        P.doc_start[n] = doc_offsets[n];
+        P.resp_off[n] = (int32_t)roff;
+        P.ck_off[n] = (int32_t)ckn;
+        if (n < N) {
+            P.doc_prompt[n] = prompt_len[n];
+            roff += (int64_t)doc_offsets[n + 1] - doc_offsets[n] - prompt_len[n];
+            ckn += ((int64_t)doc_offsets[n + 1] - doc_offsets[n] + kCk - 1) / kCk;
+        }
+    }
+    cudaError_t e;
+    const bool bf = dtype == GDN_BF16;
+    switch (D) {
+        case 32: e = bf ? launch_bwd<__nv_bfloat16, 32>(P, st) : launch_bwd<float, 32>(P, st); break;
+        case 64: e = bf ? launch_bwd<__nv_bfloat16, 64>(P, st) : launch_bwd<float, 64>(P, st); break;
+        default: e = bf ? launch_bwd<__nv_bfloat16, 128>(P, st) : launch_bwd<float, 128>(P, st); break;
+    }
+    // the slice partials, added in slice order
+    const int64_t nn = (noisy ? V * TR : 0) * H;
+    if (e == cudaSuccess) e = reduce_slices(p_dq, dq, th * D, per_slice, ns, st);
+    if (e == cudaSuccess) e = reduce_slices(p_dk, dk, th * D, per_slice, ns, st);
+    if (e == cudaSuccess) e = reduce_slices(p_dg, dg, th, per_slice, ns, st);
+    if (e == cudaSuccess) e = reduce_slices(p_dbeta, dbeta, th, per_slice, ns, st);
+    if (noisy) {
+        // the noisy partials are laid out over V x T_R rows inside their V x T row sections
+        if (e == cudaSuccess) e = reduce_slices(p_dqn, dqn, nn * D, per_slice, ns, st);
+        if (e == cudaSuccess) e = reduce_slices(p_dkn, dkn, nn * D, per_slice, ns, st);
+        if (e == cudaSuccess) e = reduce_slices(p_dgn, dgn, nn, per_slice, ns, st);
+        if (e == cudaSuccess) e = reduce_slices(p_dbetan, dbetan, nn, per_slice, ns, st);
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace gdn
+
 using namespace gdn;
 
 extern "C" size_t gdn_dual_backward_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host) {
@@ -341,7 +448,9 @@ extern "C" size_t gdn_dual_backward_workspace_size(const gdn_dual_desc *desc, co
     for (int n = 0; n < desc->num_docs; ++n)
         if (doc_offsets_host[n + 1] < doc_offsets_host[n]) return 0;
     const int64_t nck = bwd_checkpoints(desc, doc_offsets_host);
-    return (size_t)nck * desc->num_heads * desc->d_k * desc->d_v * sizeof(float) + 256;
+    const int ns = desc->d_k >= 32 ? desc->d_k / 32 : 1;
+    const int64_t part = (int64_t)ns * bwd_partial_floats(desc, doc_offsets_host[desc->num_docs]);
+    return ((size_t)nck * desc->num_heads * desc->d_k * desc->d_v + (size_t)part) * sizeof(float) + 256;
 }
 
 extern "C" gdn_status gdn_dual_backward(const gdn_dual_desc *desc, const void *q, const void *k, const void *v,
@@ -353,7 +462,7 @@ extern "C" gdn_status gdn_dual_backward(const gdn_dual_desc *desc, const void *q
                                         float *dqn, float *dkn, float *dvn, float *dgn, float *dbetan,
                                         void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
     if (!bwd_desc_ok(desc) || !doc_offsets || !prompt_len || doc_offsets[0] != 0) return GDN_ERR_INVALID_ARG;
-    const int N = desc->num_docs, H = desc->num_heads, B = desc->block_size, D = desc->d_k;
+    const int N = desc->num_docs, B = desc->block_size, D = desc->d_k;
     int64_t TR = 0;
     for (int n = 0; n < N; ++n) {
         const int64_t len = (int64_t)doc_offsets[n + 1] - doc_offsets[n];
@@ -378,43 +487,7 @@ extern "C" gdn_status gdn_dual_backward(const gdn_dual_desc *desc, const void *q
         return GDN_ERR_UNSUPPORTED;
     if (T == 0) return GDN_OK;
 
-    BwdParams P;
-    std::memset(&P, 0, sizeof(P));
-    P.q = q; P.k = k; P.v = v; P.qn = qn; P.kn = kn; P.vn = vn; P.dout = d_out; P.doutn = d_out_noisy;
-    P.g = g; P.beta = beta; P.gn = gn; P.betan = betan; P.dsf = d_final_state;
-    P.dq = dq; P.dk = dk; P.dv = dv; P.dg = dg; P.dbeta = dbeta;
-    P.dqn = dqn; P.dkn = dkn; P.dvn = dvn; P.dgn = dgn; P.dbetan = dbetan;
-    P.ck = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + 256);
-    P.TR = TR; P.N = N; P.H = H; P.V = noisy ? desc->num_views : 0; P.B = B;
-    P.scale = (float)(1.0 / std::sqrt((double)D));
-    int64_t roff = 0, ck = 0;
-    for (int n = 0; n <= N; ++n) {
-        P.doc_start[n] = doc_offsets[n];
-        P.resp_off[n] = (int32_t)roff;
-        P.ck_off[n] = (int32_t)ck;
-        if (n < N) {
-            P.doc_prompt[n] = prompt_len[n];
-            roff += (int64_t)doc_offsets[n + 1] - doc_offsets[n] - prompt_len[n];
-            ck += ((int64_t)doc_offsets[n + 1] - doc_offsets[n] + kCk - 1) / kCk;
-        }
-    }
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // the column-summed gradients are accumulated with atomics
-    const size_t tok = (size_t)T * H, ntok = (size_t)(noisy ? desc->num_views : 0) * TR * H;
-    if (cudaMemsetAsync(dq, 0, tok * D * 4, st) != cudaSuccess || cudaMemsetAsync(dk, 0, tok * D * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(dg, 0, tok * 4, st) != cudaSuccess || cudaMemsetAsync(dbeta, 0, tok * 4, st) != cudaSuccess)
-        return GDN_ERR_CUDA;
-    if (noisy) {
-        if (cudaMemsetAsync(dqn, 0, ntok * D * 4, st) != cudaSuccess || cudaMemsetAsync(dkn, 0, ntok * D * 4, st) != cudaSuccess ||
-            cudaMemsetAsync(dgn, 0, ntok * 4, st) != cudaSuccess || cudaMemsetAsync(dbetan, 0, ntok * 4, st) != cudaSuccess)
-            return GDN_ERR_CUDA;
-    }
-    cudaError_t e;
-    const bool bf = desc->dtype == GDN_BF16;
-    switch (D) {
-        case 32: e = bf ? launch_bwd<__nv_bfloat16, 32>(P, st) : launch_bwd<float, 32>(P, st); break;
-        case 64: e = bf ? launch_bwd<__nv_bfloat16, 64>(P, st) : launch_bwd<float, 64>(P, st); break;
-        default: e = bf ? launch_bwd<__nv_bfloat16, 128>(P, st) : launch_bwd<float, 128>(P, st); break;
-    }
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return gdn::run_backward(desc, desc->dtype, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len,
+                             d_out, d_out_noisy, d_final_state, dq, dk, dv, dg, dbeta, dqn, dkn, dvn, dgn, dbetan,
+                             workspace, reinterpret_cast<cudaStream_t>(stream));
 }

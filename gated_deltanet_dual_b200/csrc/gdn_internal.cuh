@@ -60,6 +60,14 @@ cudaError_t launch_pipe(const Params &p, cudaStream_t stream);
 // Route I: clean chain writing block-boundary states into `states`, then block refinement.
 cudaError_t launch_route1(const Params &p, int dtype, float *states, cudaStream_t stream);
 bool chunked_supported(int dtype, int d, int B, int conv_width);
+// The backward on validated arguments, inputs and upstream gradients of element type `dtype`;
+// the workspace must hold gdn_dual_backward_workspace_size() bytes for the descriptor.
+gdn_status run_backward(const gdn_dual_desc *desc, int dtype, const void *q, const void *k, const void *v,
+                        const float *g, const float *beta, const void *qn, const void *kn, const void *vn,
+                        const float *gn, const float *betan, const int32_t *doc_offsets, const int32_t *prompt_len,
+                        const void *d_out, const void *d_out_noisy, const float *d_final_state, float *dq,
+                        float *dk, float *dv, float *dg, float *dbeta, float *dqn, float *dkn, float *dvn,
+                        float *dgn, float *dbetan, void *workspace, cudaStream_t st);
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

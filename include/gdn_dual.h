@@ -149,11 +149,12 @@ gdn_status gdn_dual_forward(const gdn_dual_desc *desc,
  * with respect to every input, all fp32 in the inputs' layouts: dq dk dv [T, H, d], dg dbeta
  * [T, H], dqn dkn dvn [V, T_R, H, d], dgn dbetan [V, T_R, H] (fully overwritten; the noisy ones
  * may be NULL when there are no noisy rows).  The workspace holds the clean states at every
- * 16th token: at least gdn_dual_backward_workspace_size() bytes.  Host validation as for the
- * forward; GDN_ERR_UNSUPPORTED for ShortConv (conv_width != 0), d_k != d_v or d not in
- * {32, 64, 128}.  CUDA-core kernel (one CTA per (document, head, 32 state columns)); the
- * column-summed gradients are accumulated with fp32 atomics, so their last bits may vary from
- * call to call.
+ * 16th token and the per-slice partial sums below: at least gdn_dual_backward_workspace_size()
+ * bytes.  Host validation as for the forward; GDN_ERR_UNSUPPORTED for ShortConv (conv_width != 0:
+ * use gdn_dual_backward_conv), d_k != d_v or d not in {32, 64, 128}.  CUDA-core kernel (one CTA
+ * per (document, head, 32 state columns)); the column-summed gradients (dq, dk, dg, dbeta and
+ * their noisy twins) are stored per 32-column slice and added in slice order by a second kernel,
+ * so the results are the same on every call.
  */
 size_t gdn_dual_backward_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host);
 gdn_status gdn_dual_backward(const gdn_dual_desc *desc,
@@ -166,6 +167,33 @@ gdn_status gdn_dual_backward(const gdn_dual_desc *desc,
                              float *dq, float *dk, float *dv, float *dg, float *dbeta,
                              float *dqn, float *dkn, float *dvn, float *dgn, float *dbetan,
                              void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * Backward pass of gdn_dual_forward with the width-4 ShortConv prologue (desc->conv_width == 4;
+ * Method > Key design 3 of the FLARE notes: depthwise causal conv of q, k, v, tap 3 = the current
+ * token, the same weights for both streams, a noisy tap before its block start reads the clean raw
+ * input, no tap across a document start).  Arguments as gdn_dual_backward, plus:
+ *   conv_w    device fp32 [3, H*d_k, 4], the forward's weights;
+ *   dconv_w   device fp32 [3, H*d_k, 4] output, the gradient of the weights.
+ * dq dk dv (dqn dkn dvn) are the gradients of the RAW (unconvolved) inputs.  The workspace must
+ * hold gdn_dual_backward_conv_workspace_size() bytes (the convolved inputs and their gradients in
+ * fp32, besides the backward's own checkpoints).  Every sum runs in a fixed order, so the results
+ * are the same on every call.  GDN_ERR_UNSUPPORTED unless conv_width == 4, d_k == d_v in
+ * {32, 64, 128}.  CUDA cores: the conv, the backward of the recurrence on the convolved fp32
+ * inputs, then the transposed taps and the weight sums.
+ */
+size_t gdn_dual_backward_conv_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host);
+gdn_status gdn_dual_backward_conv(const gdn_dual_desc *desc,
+                                  const void *q, const void *k, const void *v,
+                                  const float *g, const float *beta,
+                                  const void *qn, const void *kn, const void *vn,
+                                  const float *gn, const float *betan,
+                                  const int32_t *doc_offsets, const int32_t *prompt_len,
+                                  const float *conv_w,
+                                  const void *d_out, const void *d_out_noisy, const float *d_final_state,
+                                  float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                                  float *dqn, float *dkn, float *dvn, float *dgn, float *dbetan,
+                                  float *dconv_w, void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /*
  * gdn_dual_forward without a workspace argument, for callers that cannot allocate device

@@ -349,8 +349,12 @@ def test_backward_host_validation():
                                      *ptr[10:23], ptr[23], ctypes.c_size_t(nb), None)
 
     d = b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32)
-    # 73 tokens in 16-token checkpoints: 3 + 3 per head, 64 x 64 fp32 each, plus 256 bytes
-    assert b.backward_workspace_size(d, offs) == 256 + 6 * 2 * 64 * 64 * 4
+    # 73 tokens in 16-token checkpoints: 3 + 3 per head, 64 x 64 fp32 each, plus 256 bytes; then the
+    # column-summed gradients' partials, per 32-column slice (2 here): [dq | dk] (T H d each) and
+    # [dg | dbeta] (T H each), and the same for the noisy stream over V x T rows
+    th = 73 * 2
+    partial = 2 * (2 * th * 64 + 2 * th) * (1 + 2)
+    assert b.backward_workspace_size(d, offs) == 256 + 6 * 2 * 64 * 64 * 4 + partial * 4
     assert call(d, ws_bytes=1024) == b.GDN_ERR_INVALID_ARG
     assert call(d, over={0: None}) == b.GDN_ERR_INVALID_ARG                  # q
     assert call(d, over={3: base + 4}) == b.GDN_ERR_ALIGNMENT                # g
@@ -397,3 +401,35 @@ def test_noalloc_rejects_route1_and_invalid_descriptors():
     assert call(None) == b.GDN_ERR_INVALID_ARG
     assert call(b.make_desc(1, 2, 128, 128, 9, 4, b.GDN_BF16)) == b.GDN_ERR_INVALID_ARG    # views > 8
     assert call(b.make_desc(0, 2, 128, 128, 2, 4, b.GDN_BF16)) == b.GDN_ERR_INVALID_ARG    # no documents
+
+
+@no_gpu
+def test_backward_conv_host_validation():
+    """gdn_dual_backward_conv refuses on the host: conv width other than 4, NULL weights or weight
+    gradient, a workspace smaller than gdn_dual_backward_conv_workspace_size."""
+    base = 0x7f0000000000
+    lib = b.load_library()
+    offs = np.array([0, 40, 73], np.int32)
+    pl = np.array([8, 1], np.int32)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    fn = lib.gdn_dual_backward_conv
+    fn.restype = ctypes.c_int
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(b.Desc)] + [vp] * 10 + [ip, ip] + [vp] * 4 + [vp] * 10 + [vp, vp, ctypes.c_size_t, vp]
+
+    def call(desc, ws_bytes=None, over=None):
+        ptr = [ctypes.c_void_p(base + 0x10000000 * i) for i in range(26)]   # 10 in, conv_w, 3 up, 10 grads, dw, ws
+        for i, v in (over or {}).items():
+            ptr[i] = None if v is None else ctypes.c_void_p(v)
+        nb = b.backward_conv_workspace_size(desc, offs) if ws_bytes is None else ws_bytes
+        return fn(ctypes.byref(desc), *ptr[:10], offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), *ptr[10:25],
+                  ptr[25], ctypes.c_size_t(nb), None)
+
+    d = b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32, conv_width=4)
+    need = b.backward_conv_workspace_size(d, offs)
+    assert need > b.backward_workspace_size(b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32), offs)
+    assert call(d, ws_bytes=need - 16) == b.GDN_ERR_INVALID_ARG
+    assert call(d, over={10: None}) == b.GDN_ERR_INVALID_ARG                 # conv_w
+    assert call(d, over={24: None}) == b.GDN_ERR_INVALID_ARG                 # dconv_w
+    assert call(b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32, conv_width=3)) == b.GDN_ERR_UNSUPPORTED
+    assert call(b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32)) == b.GDN_ERR_UNSUPPORTED   # no conv: gdn_dual_backward

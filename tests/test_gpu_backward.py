@@ -15,11 +15,11 @@ TOL = 1e-4
 GRADS = ("dq", "dk", "dv", "dg", "dbeta", "dqn", "dkn", "dvn", "dgn", "dbetan")
 
 
-def problem(lens, prompts, B, d=64, H=2, V=2, dtype="fp32", seed=0, g_lo=-0.1):
+def problem(lens, prompts, B, d=64, H=2, V=2, dtype="fp32", seed=0, g_lo=-0.1, conv=0):
     offs = np.zeros(len(lens) + 1, np.int32)
     offs[1:] = np.cumsum(lens)
     return synth.make_problem_from_layout(offs, prompts, num_heads=H, d_k=d, d_v=d, block_size=B, num_views=V,
-                                          dtype=dtype, seed=seed, g_lo=g_lo, device="cuda")
+                                          dtype=dtype, seed=seed, g_lo=g_lo, conv_width=conv, device="cuda")
 
 
 def upstream(pr, seed, final=True):
@@ -35,12 +35,16 @@ def upstream(pr, seed, final=True):
 def check(pr, seed=1, final=True):
     do, don, dsf = upstream(pr, seed, final)
     got = b.backward(pr.q, pr.k, pr.v, pr.g, pr.beta, pr.qn, pr.kn, pr.vn, pr.gn, pr.betan, pr.doc_offsets,
-                     pr.prompt_len, pr.block_size, do, don, dsf)
+                     pr.prompt_len, pr.block_size, do, don, dsf, conv_w=pr.conv_w)
     torch.cuda.synchronize()
-    ref = ob.dual_backward(pr.q, pr.k, pr.v, pr.g, pr.beta, pr.qn, pr.kn, pr.vn, pr.gn, pr.betan, pr.doc_offsets,
-                           pr.prompt_len, pr.block_size, do, don, dsf)
+    if pr.conv_w is None:
+        ref = ob.dual_backward(pr.q, pr.k, pr.v, pr.g, pr.beta, pr.qn, pr.kn, pr.vn, pr.gn, pr.betan,
+                               pr.doc_offsets, pr.prompt_len, pr.block_size, do, don, dsf)
+    else:
+        ref = ob.dual_backward_conv(pr.q, pr.k, pr.v, pr.g, pr.beta, pr.qn, pr.kn, pr.vn, pr.gn, pr.betan,
+                                    pr.doc_offsets, pr.prompt_len, pr.block_size, pr.conv_w, do, don, dsf)
     errs = {}
-    for n in GRADS:
+    for n in GRADS + (("dconv_w",) if pr.conv_w is not None else ()):
         r = ref[n]
         if r.size == 0:
             continue
@@ -105,3 +109,31 @@ def test_invalid_arguments():
         b.backward(pr.q, pr.k, pr.v, pr.g, pr.beta, pr.qn, pr.kn, pr.vn, pr.gn, pr.betan, pr.doc_offsets,
                    [10, -1], 4, do, don, dsf)
     assert e.value.status == b.GDN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B", [1, 4, 8, 32])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_shortconv_backward(B, dtype):
+    """gdn_dual_backward_conv against the oracle's conv backward (Key design 3): ragged documents, a
+    prompt shorter than the conv, an empty prompt (the first block's taps before the document read
+    nothing), a prompt-only document; gradients of the raw inputs and of the weights."""
+    R = lambda r: (r // B) * B
+    lens = [2 + R(40), 69 + R(3), 20]
+    prompts = [2, 5, 20]
+    lens[1] = 5 + R(64)
+    check(problem(lens, prompts, B, d=64, dtype=dtype, seed=40 + B, conv=4))
+
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_backward_is_deterministic(conv):
+    """Two calls on the same inputs give bit-identical gradients (no atomics: per-slice partials
+    added in a fixed order)."""
+    pr = problem([200, 136], [72, 8], 4, d=128, dtype="bf16", seed=50 + conv, conv=conv)
+    do, don, dsf = upstream(pr, 5)
+    run = lambda: b.backward(pr.q, pr.k, pr.v, pr.g, pr.beta, pr.qn, pr.kn, pr.vn, pr.gn, pr.betan, pr.doc_offsets,
+                             pr.prompt_len, pr.block_size, do, don, dsf, conv_w=pr.conv_w)
+    a = {n: t.clone() for n, t in run().items()}
+    c = run()
+    torch.cuda.synchronize()
+    for n in a:
+        assert torch.equal(a[n], c[n]), n
