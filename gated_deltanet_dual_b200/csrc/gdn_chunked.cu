@@ -459,24 +459,23 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             atomicExch(&P.ws->timeout_where, where);
         }
     };
-    // Error path.  Once one of this thread's waits has given up, the thread waits on nothing more
-    // (the CTA leaves at its next abort check, all threads at the same barrier).  A phase counter
-    // advances only when its wait succeeds, so thread 0's counters are the phases it saw complete.
-    // Before the CTA frees its tensor memory and exits, thread 0 -- the only thread that issues TMA
-    // loads and MMAs -- waits for everything it issued: one more commit covers all its MMAs, and on
-    // the two TMA barriers every phase between its counter and the loads it issued (s_iss), so no
-    // bulk copy or MMA is left writing into shared or tensor memory that is no longer the CTA's.
+    // Error path.  A wait that gives up records GDN_ERR_TIMEOUT, and the CTA leaves its loop at the
+    // next abort check (all threads at the same barrier).  Thread 0, the only thread that issues TMA
+    // loads and MMAs, issues no further TMA load once one of its own waits has given up (`dead`), so
+    // on each TMA barrier at most the last load it issued can still be in flight when the CTA leaves
+    // (every earlier one was waited for: a prefetch is only issued after the previous load's wait).
+    // Before the CTA frees its tensor memory, thread 0 waits for that last load (s_iss counts the
+    // loads) and, with one more commit, for every MMA it issued, so no bulk copy or MMA is left
+    // writing into shared or tensor memory that is no longer the CTA's.
     bool dead = false;
     __shared__ uint32_t s_iss[2];
     if (tid == 0) s_iss[0] = s_iss[1] = 0;
     auto wait_bar = [&](uint64_t *bar, uint32_t &ph, int where) {
-        if (!dead) {
-            if (kwait<TW>(bar, ph & 1, kWaitIters, P.wait_iters)) ++ph;
-            else {
-                dead = true;
-                fail(where);
-            }
+        if (!kwait<TW>(bar, ph & 1, kWaitIters, P.wait_iters)) {
+            fail(where);
+            dead = true;
         }
+        ++ph;
     };
     // bar_all that also tells every thread, uniformly, whether the CTA is aborting
     auto abort_check = [&] { return bar_sync_or(1, kThreads, *reinterpret_cast<volatile int *>(&s_abort) != 0); };
@@ -1099,13 +1098,11 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         }
         if (stop) break;
     }
-    // Drain (a no-op unless a wait gave up; thread 0): every TMA phase issued but not seen complete
-    // is waited for, in order, with the normal bound (a phase's parity can repeat two phases later,
-    // so an in-order wait can only return late, never early); one more commit covers every MMA.
-    // Then the cp.async groups.
+    // Drain (thread 0; immediate unless a wait gave up): the last TMA load on each barrier, then,
+    // with one more commit, every MMA.  Then the cp.async groups.
     if (tid == 0) {
-        for (uint32_t p = ph_a; p < s_iss[0]; ++p) mbar_wait(&bar_a, p & 1, kDrainWaitIters);
-        for (uint32_t p = ph_b; p < s_iss[1]; ++p) mbar_wait(&bar_b, p & 1, kDrainWaitIters);
+        if (s_iss[0] > 0) mbar_wait(&bar_a, (s_iss[0] - 1) & 1, kDrainWaitIters);
+        if (s_iss[1] > 0) mbar_wait(&bar_b, (s_iss[1] - 1) & 1, kDrainWaitIters);
         if (stop) {
             mma_commit(&bar_drain);
             mbar_wait(&bar_drain, 0, kDrainWaitIters);
