@@ -38,6 +38,13 @@ bool desc_supported(const gdn_dual_desc *d) {
     return true;
 }
 
+// AUTO with ShortConv on the chunked path runs the conv as a pass of its own (into the workspace)
+// when the workspace has room for the convolved inputs; else the chunked kernel's fused prologue.
+bool conv_pass_wanted(const gdn_dual_desc *d) {
+    return d->algo == GDN_ALGO_AUTO && d->conv_width == 4 &&
+           gdn::chunked_supported(d->dtype, d->d_k, d->block_size, d->conv_width) && d->d_k == d->d_v;
+}
+
 int select_algo(const gdn_dual_desc *d) {
     if (d->algo != GDN_ALGO_AUTO) return d->algo;
     return gdn::chunked_supported(d->dtype, d->d_k, d->block_size, d->conv_width) ? GDN_ALGO_CHUNKED
@@ -73,6 +80,11 @@ size_t gdn_dual_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_off
     for (int n = 0; n < desc->num_docs; ++n)
         if (doc_offsets_host[n + 1] < doc_offsets_host[n]) return 0;
     if (desc->algo == GDN_ALGO_ROUTE1) return 0;   // needs the prompt lengths: the _route1 variant
+    if (conv_pass_wanted(desc)) {                  // room for the convolved inputs (T_R <= T)
+        const int64_t T = doc_offsets_host[desc->num_docs];
+        return sizeof(gdn::WorkspaceHeader) +
+               gdn::conv_pass_bytes(T, T, desc->num_heads, desc->d_k, desc->num_views);
+    }
     return sizeof(gdn::WorkspaceHeader);
 }
 
@@ -175,12 +187,30 @@ gdn_status forward_impl(const gdn_dual_desc *desc,
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, sizeof(gdn::WorkspaceHeader), st) != cudaSuccess) return GDN_ERR_CUDA;
     cudaError_t err;
-    if (algo == GDN_ALGO_CHUNKED || algo == GDN_ALGO_PIPELINED)
+    const size_t pass_bytes = gdn::conv_pass_bytes(T, TR, H, desc->d_k, P.V);
+    if (algo == GDN_ALGO_CHUNKED && conv_pass_wanted(desc) && !P.wait_test &&
+        workspace_bytes >= sizeof(gdn::WorkspaceHeader) + pass_bytes) {
+        // the conv pass, then the chunked kernel without its prologue on the convolved inputs
+        uint8_t *buf = static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader);
+        err = gdn::launch_conv_pass(P, buf, st);
+        if (err == cudaSuccess) {
+            const int64_t clean = T * H * desc->d_k, nz = (int64_t)P.V * TR * H * desc->d_k;
+            const __nv_bfloat16 *y = reinterpret_cast<const __nv_bfloat16 *>(buf);
+            gdn::Params Q = P;
+            Q.q = y; Q.k = y + clean; Q.v = y + 2 * clean;
+            Q.qn = y + 3 * clean; Q.kn = y + 3 * clean + nz; Q.vn = y + 3 * clean + 2 * nz;
+            Q.conv_width = 0;
+            Q.conv_w = nullptr;
+            err = gdn::launch_chunked(Q, false, st);
+        }
+    } else if (algo == GDN_ALGO_CHUNKED || algo == GDN_ALGO_PIPELINED) {
         err = gdn::launch_chunked(P, algo == GDN_ALGO_PIPELINED, st);
-    else if (algo == GDN_ALGO_ROUTE1)
+    } else if (algo == GDN_ALGO_ROUTE1) {
         err = gdn::launch_route1(P, desc->dtype,
                                  reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader)), st);
-    else err = gdn::launch_sequential(P, desc->dtype, st);
+    } else {
+        err = gdn::launch_sequential(P, desc->dtype, st);
+    }
     if (err == cudaErrorNotSupported) return GDN_ERR_UNSUPPORTED;
     return err == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

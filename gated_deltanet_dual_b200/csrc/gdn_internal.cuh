@@ -57,6 +57,10 @@ cudaError_t launch_sequential(const Params &p, int dtype, cudaStream_t stream);
 cudaError_t launch_chunked(const Params &p, bool pipelined, cudaStream_t stream);
 // The warp-specialised pipelined variant of the chunked kernel (no ShortConv, at most two views).
 cudaError_t launch_pipe(const Params &p, cudaStream_t stream);
+// ShortConv as a pass of its own: the convolved bf16 q, k, v (T H d each, in that order) and
+// their noisy twins (V T_R H d each) into `buf` (conv_pass_bytes of them).
+size_t conv_pass_bytes(int64_t T, int64_t TR, int H, int d, int V);
+cudaError_t launch_conv_pass(const Params &p, void *buf, cudaStream_t stream);
 // Route I: clean chain writing block-boundary states into `states`, then block refinement.
 cudaError_t launch_route1(const Params &p, int dtype, float *states, cudaStream_t stream);
 bool chunked_supported(int dtype, int d, int B, int conv_width);

@@ -13,7 +13,9 @@
 namespace {
 
 // Fixed scratch: 4096 bytes.  Every GPU that loads this library holds it until the process
-// exits.  The kernels currently need 256 bytes of it.
+// exits.  The kernels need 256 bytes of it (their status words and work counter); with ShortConv
+// the conv then runs in the chunked kernel's prologue (the separate conv pass would need room for
+// the convolved inputs).
 constexpr size_t kNoAllocScratchBytes = 4096;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -53,9 +55,8 @@ extern "C" gdn_status gdn_dual_forward_noalloc(const gdn_dual_desc *desc,
     if (!desc || !doc_offsets) return GDN_ERR_INVALID_ARG;
     // Route I keeps every block-boundary state in its workspace: far more than the array holds.
     if (desc->algo == GDN_ALGO_ROUTE1) return GDN_ERR_UNSUPPORTED;
-    const size_t need = gdn_dual_workspace_size(desc, doc_offsets);
-    if (need == 0) return GDN_ERR_INVALID_ARG;
-    if (need > kNoAllocScratchBytes) return GDN_ERR_UNSUPPORTED;   // problem needs more scratch than the array holds
+    if (gdn_dual_workspace_size(desc, doc_offsets) == 0) return GDN_ERR_INVALID_ARG;
+    static_assert(sizeof(gdn::WorkspaceHeader) <= kNoAllocScratchBytes, "the status words fit the array");
     void *scratch = nullptr;
     const gdn_status st = scratch_address(&scratch);
     if (st != GDN_OK) return st;

@@ -100,9 +100,13 @@ typedef struct {
 /* Same object as cudaStream_t; NULL is the legacy default stream. */
 typedef struct CUstream_st *gdn_stream_t;
 
-/* Bytes of device workspace gdn_dual_forward needs for this problem (>= 256, a multiple of
+/* Bytes of device workspace gdn_dual_forward wants for this problem (>= 256, a multiple of
  * 256).  doc_offsets_host: HOST array [N+1].  Returns 0 if the descriptor or offsets are
- * invalid.  For GDN_ALGO_ROUTE1 it adds the materialised block-boundary states, T_R / B x H x
+ * invalid.  Any workspace of at least 256 bytes is accepted; the size returned here also covers
+ * the convolved inputs of a GDN_ALGO_AUTO call with ShortConv on the chunked path (bf16, 3 T H d
+ * plus 3 V T H d elements): with that much, the conv runs as a pass of its own over every SM
+ * before the chunked kernel; with less, inside the chunked kernel's prologue (same results up to
+ * the accumulation order of the chunked products).  For GDN_ALGO_ROUTE1 it adds the materialised block-boundary states, T_R / B x H x
  * d_k x d_v fp32 (all documents' responses, T_R from doc_offsets and the prompt lengths); for
  * that algorithm prompt_len must be known, so use gdn_dual_workspace_size_route1. */
 size_t gdn_dual_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host);
@@ -203,8 +207,9 @@ gdn_status gdn_dual_backward_conv(const gdn_dual_desc *desc,
  * semantics and host validation as gdn_dual_forward.
  *   Scratch: a fixed 4096-byte array in the library's own device memory (a file-scope
  *     __device__ array; every GPU that loads the library holds it until the process exits).
- *     A problem whose gdn_dual_workspace_size() exceeds 4096 bytes returns
- *     GDN_ERR_UNSUPPORTED (the current kernels need 256 bytes).
+ *     The kernels need 256 bytes of it; with ShortConv the conv runs in the chunked kernel's
+ *     prologue (the separate conv pass needs room for the convolved inputs, which the array does
+ *     not have).
  *   Allocation: none, on any call (no cudaMalloc or cudaFree).
  *   Set-up: the first call on a device, with that device current, looks up the array's device
  *     address (cudaGetSymbolAddress); make that first call before any stream capture.

@@ -433,3 +433,16 @@ def test_backward_conv_host_validation():
     assert call(d, over={24: None}) == b.GDN_ERR_INVALID_ARG                 # dconv_w
     assert call(b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32, conv_width=3)) == b.GDN_ERR_UNSUPPORTED
     assert call(b.make_desc(2, 2, 64, 64, 2, 4, b.GDN_FP32)) == b.GDN_ERR_UNSUPPORTED   # no conv: gdn_dual_backward
+
+
+def test_workspace_size_covers_the_conv_pass():
+    """With ShortConv, AUTO on the chunked path asks for room for the convolved bf16 inputs
+    (3 T H d clean + 3 V T H d noisy elements, T_R bounded by T); an explicit algorithm needs the
+    256-byte header only."""
+    offs = [0, 64, 192]
+    T, H, d, V = 192, 2, 128, 2
+    auto = b.make_desc(2, H, d, d, V, 4, b.GDN_BF16, conv_width=4)
+    conv_bytes = 3 * (T * H * d + V * T * H * d) * 2
+    assert b.workspace_size(auto, offs) == 256 + (conv_bytes + 255) // 256 * 256
+    assert b.workspace_size(b.make_desc(2, H, d, d, V, 4, b.GDN_BF16, conv_width=4, algo=b.ALGO_CHUNKED), offs) == 256
+    assert b.workspace_size(b.make_desc(2, H, d, d, V, 4, b.GDN_BF16), offs) == 256
