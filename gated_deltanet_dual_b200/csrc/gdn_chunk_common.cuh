@@ -20,6 +20,7 @@ constexpr int CH = 64;                 // chunk length
 
 struct Maps {
     CUtensorMap q, k, v, qn, kn, vn;
+    CUtensorMap o, on;            // outputs (TMA stores of whole chunks)
 };
 
 __device__ __forceinline__ uint4 pack8(const float *f) {

@@ -29,7 +29,10 @@
 //   S2   [P T; T] R                                                (needs R)
 //   S3   Khat^T U,  M'_Z U (+=)                                    (needs U)
 // Inputs of the next chunk are prefetched by TMA while the current chunk's S-dependent phases
-// run.  All waits are bounded; on timeout the kernel records GDN_ERR_TIMEOUT, waits for the
+// run.  Outputs of chunks that lie inside their document leave by TMA stores from tiles that are
+// free at that point (O in the [P;T] tile, the noisy rows in the K-hat and [P;T] tiles), not as
+// row-per-lane global stores; chunks at a document edge store row by row, so that no store
+// reaches into a neighbouring document.  All waits are bounded; on timeout the kernel records GDN_ERR_TIMEOUT, waits for the
 // copies and MMAs it has issued, and exits.
 #include <algorithm>
 #include <cudaTypedefs.h>
@@ -407,6 +410,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bar_a, bar_b, bar_mma, bar_mma2;   // bar_mma2: the noisy half of PK1 only
     __shared__ uint64_t bar_drain;                         // error path: all MMAs of thread 0 done
+    __shared__ uint64_t bar_ost;                           // thread 0: the O tile's store has read [P;T]
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     // Per-chunk scalars, double-buffered so the next chunk's are prepared while this chunk's
@@ -434,6 +438,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         mbar_init(&bar_mma, 1);
         mbar_init(&bar_mma2, 1);
         mbar_init(&bar_drain, 1);
+        mbar_init(&bar_ost, 1);
         fence_mbar_init();
         s_abort = 0;
     }
@@ -451,7 +456,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     tc_fence_after();
     const uint32_t tb = s_tmem;
     // Every mbarrier has at most one outstanding phase when it is waited on, so parities never alias.
-    uint32_t ph_a = 0, ph_b = 0, ph_mma = 0, ph_mma2 = 0;
+    uint32_t ph_a = 0, ph_b = 0, ph_mma = 0, ph_mma2 = 0, ph_ost = 0;
 
     auto fail = [&](int where) {
         if (atomicExch(&s_abort, 1) == 0) {
@@ -633,8 +638,6 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     // for a clean-only chunk costing kCleanCost of a full one (lower for long blocks, whose noisy
     // work weighs more).
     constexpr float kCleanCost = B >= 32 ? 0.42f : (B >= 16 ? 0.55f : 0.65f);   // measured balance
-    // B >= 16: the noisy block coefficients are staged in the Khat buffer, so Khat is built late.
-    constexpr bool kKhatLate = B >= 16;
     static_assert(4 * kAtQuadBytes<B> <= 16384, "block coefficients must fit the Khat buffer");
     // Work items are (unit, part), longest documents first; each CTA starts with item blockIdx.x and
     // then takes the next untaken item from a counter in the workspace (greedy list scheduling:
@@ -688,6 +691,11 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             const bool noisy = chunk_noisy(ci);
             const bool last = ci == ci_end - 1;
             const int cstart = U.s + U.prompt + CH * m;   // global token of chunk row 0
+            // whole chunks inside the document leave by TMA stores staged in free tiles: O in
+            // the [P;T] tile after S2, the noisy rows in the K-hat and [P;T] tiles after S3 (not
+            // with the in-kernel conv, whose weights live in the K-hat tile at the chunk top)
+            const bool o_tma = cstart >= U.s && cstart + CH <= U.s + U.len && ci >= ci_full;
+            const bool n_tma = noisy && !conv && CH * m + CH <= U.R;
             float *s_gam = s_sc[cb] + SC_GAM, *s_beta = s_sc[cb] + SC_BETA;
             float *s_E = s_sc[cb] + SC_E, *s_F = s_sc[cb] + SC_F;
             float *s_ngam = s_sc[cb] + SC_NGAM, *s_nbeta = s_sc[cb] + SC_NBETA;
@@ -744,12 +752,16 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     mma_bf16(tb + TM_TK, dK_qk + (off >> 4), dK_qk + ((8192 + off) >> 4),
                              make_idesc_bf16(128, 64, 0, 0), kk > 0);
                 }
+                // the last chunk's output stores have read the K-hat and [P;T] tiles before this
+                // barrier completes: those tiles are next written after it
+                bulk_wait_read_all();
                 commit_mma();
             }
             __syncwarp();
-            // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout), on
-            // warps 1..7.  With B >= 16 its buffer first stages the noisy block coefficients and
-            // Khat is built in the S2 phase instead, before the next chunk's tiles replace K.
+            // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout), built by
+            // warps 1..7 in the S2 phase, before the next chunk's tiles replace K: until PK1
+            // completes its buffer still feeds the last chunk's noisy output stores, and with
+            // B >= 16 it then stages the noisy block coefficients.
             auto build_khat = [&] {
                 const float gC = s_gam[CH - 1];
                 for (int it = tid - 32; it >= 0 && it < 64 * 16; it += kMathThreads - 32) {
@@ -762,7 +774,6 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     *reinterpret_cast<uint4 *>(sm + OFF_KH + hf * 8192 + sw128_off(t, c8)) = pack8(f);
                 }
             };
-            if constexpr (!kKhatLate) build_khat();
             if (!conv) wait_bar(&bar_b, ph_b, 2);   // V and [k~0;k~1]
             __syncwarp();
             if (noisy && tid == 0) {
@@ -953,8 +964,16 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     }
                 }
                 commit_mma();
-                // prefetch group A of the next chunk once [Q;K] and Z are consumed
-                if (!kKhatLate && !last && !dead) {
+            }
+            __syncwarp();
+            // Khat reads K from the [Q;K] tile: warps 1..7 build it, then signal warp 0, whose
+            // lane 0 lets the next chunk's group A overwrite the tile once [Q;K] and Z are consumed.
+            if (warp > 0) {
+                build_khat();
+                bar_arrive_khat();
+            } else {
+                bar_sync_khat();
+                if (tid == 0 && !last && !dead) {
                     if (!kwait<TW>(&bar_mma, ph_mma & 1, kWaitIters, P.wait_iters)) {
                         dead = true;
                         fail(40);
@@ -962,26 +981,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                         issue_a(U, m + 1, chunk_noisy(ci + 1));
                     }
                 }
-            }
-            __syncwarp();
-            if constexpr (kKhatLate) {
-                // Khat reads K from the [Q;K] tile: warps 1..7 build it, then signal warp 0,
-                // whose lane 0 lets the next chunk's group A overwrite the tile.
-                if (warp > 0) {
-                    build_khat();
-                    bar_arrive_khat();
-                } else {
-                    bar_sync_khat();
-                    if (tid == 0 && !last && !dead) {
-                        if (!kwait<TW>(&bar_mma, ph_mma & 1, kWaitIters, P.wait_iters)) {
-                            dead = true;
-                            fail(40);
-                        } else {
-                            issue_a(U, m + 1, chunk_noisy(ci + 1));
-                        }
-                    }
-                    __syncwarp();
-                }
+                __syncwarp();
             }
             if (!last && warp > 0) prep_scalars(U, m + 1, cb ^ 1);   // next chunk's scalars meanwhile
             wait_mma(40);
@@ -999,7 +999,11 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     tmem_wait_ld();
 #pragma unroll
                     for (int x = 0; x < 32; ++x) qs[x] = (Gt * qs[x] + pu[x]) * scale;
-                    if (ok) {
+                    if (o_tma) {
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            *reinterpret_cast<uint4 *>(sm + OFF_Y + ch * 8192 + sw128_off(t, 4 * hf + c4)) = pack8(qs + 8 * c4);
+                    } else if (ok) {
 #pragma unroll
                         for (int c4 = 0; c4 < 4; ++c4)
                             *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(qs + 8 * c4);
@@ -1027,6 +1031,11 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // ================= S3 =================
             if (tid == 0) {
                 tc_fence_after();
+                if (o_tma && !dead) {
+                    tma_store_3d(&M.o, sm + OFF_Y, 0, U.h, cstart);
+                    tma_store_3d(&M.o, sm + OFF_Y + 8192, 64, U.h, cstart);
+                    bulk_commit();
+                }
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16(tb + TM_R0, dM_kh + ((kk * 2048) >> 4), dM_v + ((kk * 2048) >> 4),
                              make_idesc_bf16(128, 128, 1, 1), kk > 0);
@@ -1043,6 +1052,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     } else {
                         issue_b(U, m + 1, chunk_noisy(ci + 1));
                     }
+                }
+                if (o_tma && n_tma) {          // the noisy rows are staged over the O tile
+                    bulk_wait_read_all();
+                    mbar_arrive(&bar_ost);
                 }
             }
             __syncwarp();
@@ -1069,6 +1082,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 for (int c = 0; c < 64; c += 4)
                     *reinterpret_cast<float4 *>(fs + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
             }
+            if (o_tma && n_tma) {
+                wait_bar(&bar_ost, ph_ost, 60);
+                __syncwarp();            // reconverge before the warp-collective tcgen05.ld
+            }
             if (noisy) {
                 const int vw = rho >> 6, jj = rho & 63;
                 const int rr = CH * m + jj;
@@ -1084,7 +1101,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                     float (&on)[32] = onb[hf];
 #pragma unroll
                     for (int x = 0; x < 32; ++x) on[x] *= scale;
-                    if (ok) {
+                    if (n_tma) {            // view vw's tile: 16 KB at K-hat (view 0) / [P;T] (view 1)
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            *reinterpret_cast<uint4 *>(sm + OFF_KH + vw * 16384 + ch * 8192 + sw128_off(jj, 4 * hf + c4)) =
+                                pack8(on + 8 * c4);
+                    } else if (ok) {
 #pragma unroll
                         for (int c4 = 0; c4 < 4; ++c4)
                             *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(on + 8 * c4);
@@ -1095,12 +1117,20 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             tc_fence_before();
             cb ^= 1;
             if ((stop = abort_check())) break;
+            if (tid == 0 && n_tma && !dead) {
+                for (int vw = 0; vw < V && vw < 2; ++vw)
+                    for (int hf = 0; hf < 2; ++hf)
+                        tma_store_3d(&M.on, sm + OFF_KH + vw * 16384 + hf * 8192, hf * 64, U.h,
+                                     vw * (int)TR + U.roff + CH * m);
+                bulk_commit();
+            }
         }
         if (stop) break;
     }
     // Drain (thread 0; immediate unless a wait gave up): the last TMA load on each barrier, then,
     // with one more commit, every MMA.  Then the cp.async groups.
     if (tid == 0) {
+        bulk_wait_all();
         if (s_iss[0] > 0) mbar_wait(&bar_a, (s_iss[0] - 1) & 1, kDrainWaitIters);
         if (s_iss[1] > 0) mbar_wait(&bar_b, (s_iss[1] - 1) & 1, kDrainWaitIters);
         if (stop) {
@@ -1128,16 +1158,18 @@ cudaError_t launch_chunked_views(const Params &p, bool pipelined, cudaStream_t s
     Maps maps;
     const bool noisy = p.V > 0 && p.TR > 0;
     if (!encode_map(&maps.q, p.q, p.H, p.T) || !encode_map(&maps.k, p.k, p.H, p.T) ||
-        !encode_map(&maps.v, p.v, p.H, p.T))
+        !encode_map(&maps.v, p.v, p.H, p.T) || !encode_map(&maps.o, p.out, p.H, p.T))
         return cudaErrorInvalidValue;
     if (noisy) {
         if (!encode_map(&maps.qn, p.qn, p.H, (int64_t)p.V * p.TR) || !encode_map(&maps.kn, p.kn, p.H, (int64_t)p.V * p.TR) ||
-            !encode_map(&maps.vn, p.vn, p.H, (int64_t)p.V * p.TR))
+            !encode_map(&maps.vn, p.vn, p.H, (int64_t)p.V * p.TR) ||
+            !encode_map(&maps.on, p.out_noisy, p.H, (int64_t)p.V * p.TR))
             return cudaErrorInvalidValue;
     } else {
         maps.qn = maps.q;
         maps.kn = maps.k;
         maps.vn = maps.v;
+        maps.on = maps.o;
     }
     static int num_sms = 0;
     static std::once_flag once;
