@@ -88,6 +88,8 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bar_q, bar_k, bar_v, bar_s, bar_o;
+    __shared__ uint64_t bar_drain;          // error path: every MMA thread 0 issued has completed
+    __shared__ uint32_t s_kflag, s_vflag;   // error path: thread 0's waits of the last tile (see below)
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
@@ -136,6 +138,8 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
         mbar_init(&bar_v, 1);
         mbar_init(&bar_s, 1);
         mbar_init(&bar_o, 1);
+        mbar_init(&bar_drain, 1);
+        s_kflag = s_vflag = 0u;
         fence_mbar_init();
         s_abort = 0;
     }
@@ -155,34 +159,31 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
             atomicExch(&P.ws->timeout_where, where);
         }
     };
-    // Error path (as in the chunked kernel): after one of its waits gave up, a thread waits on
-    // nothing more; thread 0, which issues every TMA load and MMA commit, counts per mbarrier the
-    // phases it issued and those it saw complete, and drains the rest before the CTA frees its
-    // tensor memory.
-    bool dead = false;
-    uint32_t iss_q = 0, iss_k = 0, iss_v = 0, iss_s = 0, iss_o = 0;
-    uint32_t ok_q = 0, ok_k = 0, ok_v = 0, ok_s = 0, ok_o = 0;
-    auto wait_bar = [&](uint64_t *bar, uint32_t parity, uint32_t &ok, int where) {
-        if (!dead && *reinterpret_cast<volatile int *>(&s_abort)) dead = true;
-        if (dead) return;
-        if (kwait<TW>(bar, parity, kAWaitIters, P.wait_iters)) ++ok;
-        else {
-            dead = true;
-            fail(where);
-        }
+    // Error path (as in the chunked kernel): a wait that gives up records its site, and the CTA
+    // leaves the key loop at the next uniform barrier, before another key tile starts.  Thread 0,
+    // which issues every TMA load and MMA, decides each issue on the waits of the same tile: it
+    // refills a buffer only after seeing its last load arrive and the MMA that read it complete,
+    // so no mbarrier ever has two phases outstanding.  It leaves the outcome of its waits of the
+    // current tile in shared memory (s_kflag after the S half, s_vflag after the PV half, each
+    // tagged with the tile); when the CTA stops, it works out from them which load may still be
+    // arriving on each mbarrier, waits for those and, through one more commit, for its MMAs
+    // before the CTA frees tensor memory.  (Counting the issued loads in registers instead, or
+    // bookkeeping inside the loop's exits, cost about 5 % of the kernel's time.)
+    auto wait_ok = [&](uint64_t *bar, uint32_t parity, int where) {
+        const bool ok = kwait<TW>(bar, parity, kAWaitIters, P.wait_iters);
+        if (!ok) fail(where);
+        return ok;
     };
     // key tile j: clean keys [s + 128 j, +128) or (j == nkc) the tile's own noisy rows
     auto issue_tile = [&](uint8_t *dst, const CUtensorMap *clean, const CUtensorMap *noisy, uint64_t *bar, int j) {
         const CUtensorMap *map = j < nkc ? clean : noisy;
         const int row0 = j < nkc ? s + AT * j : (int)nrow0;
-        ++(bar == &bar_k ? iss_k : iss_v);
         mbar_arrive_expect_tx(bar, 32768u);
         for (int hf = 0; hf < 2; ++hf)
             for (int rh = 0; rh < 2; ++rh)
                 tma_load_3d(dst + hf * 16384 + rh * 8192, map, bar, hf * 64, hk, row0 + 64 * rh);
     };
     if (tid == 0) {
-        ++iss_q;
         mbar_arrive_expect_tx(&bar_q, 32768u);
         const CUtensorMap *qm = kind == 0 ? &M.q : &M.qn;
         for (int hf = 0; hf < 2; ++hf)
@@ -205,27 +206,32 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
     const float sl2 = P.scale_log2;
     bool stop = false;        // uniform over the CTA: leave the key loop (a wait gave up)
 
-    for (int j = 0; j < nk; ++j) {
+    int j = 0;
+    for (; j < nk; ++j) {
         // ---- S = Q K_j^T
+        bool q_ok = true, k_ok = true;    // thread 0: Q and K_j arrived
         if (tid == 0) {
-            if (j == 0) wait_bar(&bar_q, 0, ok_q, 1);
-            wait_bar(&bar_k, j & 1, ok_k, 2);
-            tc_fence_after();
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16(tb + TA_S, dQ + (off >> 4), dK + (off >> 4), idesc, kk > 0);
+            q_ok = j > 0 || wait_ok(&bar_q, 0, 1);
+            k_ok = wait_ok(&bar_k, j & 1, 2) && q_ok;
+            if (k_ok) {
+                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_bf16(tb + TA_S, dQ + (off >> 4), dK + (off >> 4), idesc, kk > 0);
+                }
+                mma_commit(&bar_s);
             }
-            mma_commit(&bar_s);
-            ++iss_s;
         }
         __syncwarp();
-        {
-            uint32_t okv = 0;
-            wait_bar(&bar_s, j & 1, tid == 0 ? ok_s : okv, 3);
-        }
+        const bool s_ok = wait_ok(&bar_s, j & 1, 3);
         __syncwarp();
         tc_fence_after();
-        if (tid == 0 && j + 1 < nk && !dead) issue_tile(sm + A_OFF_K, &M.k, &M.kn, &bar_k, j + 1);
+        if (tid == 0) {
+            const bool kn = k_ok && s_ok && j + 1 < nk;                // K_{j+1} goes out
+            if (kn) issue_tile(sm + A_OFF_K, &M.k, &M.kn, &bar_k, j + 1);
+            // bit 0 Q missing, bit 1 K_{j+1} issued, bit 2 K_j missing; tile j + 1 above bit 8
+            s_kflag = (q_ok ? 0u : 1u) | (kn ? 2u : 0u) | (k_ok ? 0u : 4u) | ((uint32_t)(j + 1) << 8);
+        }
         // visible columns of this row in tile j: [lo, hi)
         int lo = 0, hi;
         if (j < nkc) hi = kind == 0 ? AT * (tile - j) + r + 1 : Pn + b0 - AT * j;
@@ -294,22 +300,26 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
         tc_fence_before();
         if ((stop = __syncthreads_or(*reinterpret_cast<volatile int *>(&s_abort) != 0))) break;
         // ---- O += P V_j
+        bool v_ok = true;                 // thread 0: V_j arrived
         if (tid == 0) {
             tc_fence_after();
-            wait_bar(&bar_v, j & 1, ok_v, 4);
-            for (int kk = 0; kk < 8; ++kk)
-                mma_bf16_ts(tb + TA_O, tb + TA_S + kk * 8, dV + ((kk * 2048) >> 4), idesc_pv, (j > 0 || kk > 0));
-            mma_commit(&bar_o);
-            ++iss_o;
+            v_ok = wait_ok(&bar_v, j & 1, 4);
+            if (v_ok) {
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tb + TA_O, tb + TA_S + kk * 8, dV + ((kk * 2048) >> 4), idesc_pv, (j > 0 || kk > 0));
+                mma_commit(&bar_o);
+            }
         }
         __syncwarp();
-        {
-            uint32_t okv = 0;
-            wait_bar(&bar_o, j & 1, tid == 0 ? ok_o : okv, 5);
-        }
+        const bool o_ok = wait_ok(&bar_o, j & 1, 5);
         __syncwarp();
         tc_fence_after();
-        if (tid == 0 && j + 1 < nk && !dead) issue_tile(sm + A_OFF_V, &M.v, &M.vn, &bar_v, j + 1);
+        if (tid == 0) {
+            const bool vn = v_ok && o_ok && j + 1 < nk;               // V_{j+1} goes out
+            if (vn) issue_tile(sm + A_OFF_V, &M.v, &M.vn, &bar_v, j + 1);
+            // bit 1 V_{j+1} issued, bit 2 V_j missing; tile j + 1 above bit 8
+            s_vflag = (vn ? 2u : 0u) | (v_ok ? 0u : 4u) | ((uint32_t)(j + 1) << 8);
+        }
         if ((stop = __syncthreads_or(*reinterpret_cast<volatile int *>(&s_abort) != 0))) break;
     }
 
@@ -338,15 +348,20 @@ gdn_attention_kernel(const __grid_constant__ AttnParams P, const __grid_constant
             }
         }
     }
-    // Drain (a no-op unless a wait gave up): every phase thread 0 issued but did not see
-    // complete, in order, with the normal limit.
-    if (tid == 0) {
+    // Drain (only when the CTA stopped early), with the normal limit: the loads that may still be
+    // arriving (a completed phase passes at once), then thread 0's MMAs.
+    if (stop && tid == 0) {
         const uint32_t lim = kDrainWaitIters;
-        for (uint32_t p = ok_q; p < iss_q; ++p) mbar_wait(&bar_q, p & 1, lim);
-        for (uint32_t p = ok_k; p < iss_k; ++p) mbar_wait(&bar_k, p & 1, lim);
-        for (uint32_t p = ok_v; p < iss_v; ++p) mbar_wait(&bar_v, p & 1, lim);
-        for (uint32_t p = ok_s; p < iss_s; ++p) mbar_wait(&bar_s, p & 1, lim);
-        for (uint32_t p = ok_o; p < iss_o; ++p) mbar_wait(&bar_o, p & 1, lim);
+        // The loop stopped in tile j.  K: K_{j+1} if it went out, else K_j unless it was seen to
+        // arrive.  V: after the PV half of tile j (s_vflag tagged j + 1) the same; before it,
+        // V_j went out (before the loop or in tile j - 1) and was not waited for.
+        const uint32_t kf = s_kflag, vf = s_vflag;
+        if (kf & 1u) mbar_wait(&bar_q, 0, lim);
+        if (kf & 6u) mbar_wait(&bar_k, ((kf & 2u) ? j + 1 : j) & 1, lim);
+        if ((vf >> 8) != (uint32_t)(j + 1)) mbar_wait(&bar_v, j & 1, lim);
+        else if (vf & 6u) mbar_wait(&bar_v, ((vf & 2u) ? j + 1 : j) & 1, lim);
+        mma_commit(&bar_drain);
+        mbar_wait(&bar_drain, 0, lim);
     }
     tc_fence_before();
     __syncthreads();
