@@ -637,7 +637,8 @@ def run_attention(args, name, rank, world, local):
 
 # ----------------------------------------------------------------------------- backward
 BWD_METRIC = "dual-stream GDN backward tokens/s on 1 B200 and % of HBM roofline"
-BWD_WORKLOADS = {"bwd_train_8x4096_h16_d128": "train_8x4096_h16_d128"}
+BWD_WORKLOADS = {"bwd_train_8x4096_h16_d128": "train_8x4096_h16_d128",
+                 "bwd_conv_4x8192_h16_d128_B4": "conv_4x8192_h16_d128_B4"}
 
 
 def backward_bytes(prob) -> int:
@@ -647,7 +648,8 @@ def backward_bytes(prob) -> int:
     s = prob.q.element_size()
     d = prob.d_k
     toks = (prob.T + prob.num_views * prob.T_R) * prob.num_heads
-    return int(toks * (4 * d * s + 8 + 3 * d * 4 + 8) + prob.num_docs * prob.num_heads * d * d * 4)
+    conv = 3 * prob.num_heads * d * 4 * 4 * 2 if prob.conv_width else 0       # weights in, dconv_w out
+    return int(toks * (4 * d * s + 8 + 3 * d * 4 + 8) + prob.num_docs * prob.num_heads * d * d * 4 + conv)
 
 
 def time_backward_oracle(prob, min_seconds=2.0):
@@ -663,9 +665,12 @@ def time_backward_oracle(prob, min_seconds=2.0):
         sn = lambda t: t[:, r0:r1, :1]
         do = np.ones((e - s, 1, prob.d_v))
         don = np.ones((prob.num_views, r1 - r0, 1, prob.d_v))
-        ob.dual_backward(sl(prob.q), sl(prob.k), sl(prob.v), sl(prob.g), sl(prob.beta), sn(prob.qn), sn(prob.kn),
-                         sn(prob.vn), sn(prob.gn), sn(prob.betan), [0, e - s], prob.prompt_len[d_:d_ + 1],
-                         prob.block_size, do, don, None)
+        args_ = (sl(prob.q), sl(prob.k), sl(prob.v), sl(prob.g), sl(prob.beta), sn(prob.qn), sn(prob.kn),
+                 sn(prob.vn), sn(prob.gn), sn(prob.betan), [0, e - s], prob.prompt_len[d_:d_ + 1], prob.block_size)
+        if prob.conv_width:     # head 0's weights: conv_w is [3, H d, W]
+            ob.dual_backward_conv(*args_, prob.conv_w[:, :prob.d_k, :], do, don, None)
+        else:
+            ob.dual_backward(*args_, do, don, None)
         toks += (e - s) + prob.num_views * (r1 - r0)
         n += 1
         el = time.perf_counter() - t0
@@ -701,15 +706,18 @@ def run_backward(args, name, rank, world, local):
     do = torch.randn(prob.T, prob.num_heads, prob.d_v, generator=gen, device=dev).to(prob.q.dtype)
     don = torch.randn(prob.num_views, prob.T_R, prob.num_heads, prob.d_v, generator=gen, device=dev).to(prob.q.dtype)
     desc = gb.make_desc(prob.num_docs, prob.num_heads, prob.d_k, prob.d_v, prob.num_views, prob.block_size,
-                        gb._dtype_code(prob.q))
-    ws = gb.Workspace(gb.backward_workspace_size(desc, prob.doc_offsets), device=dev).tensor
+                        gb._dtype_code(prob.q), prob.conv_width)
+    wsize = (gb.backward_conv_workspace_size(desc, prob.doc_offsets) if prob.conv_width
+             else gb.backward_workspace_size(desc, prob.doc_offsets))
+    ws = gb.Workspace(wsize, device=dev).tensor
     names = ("q", "k", "v", "g", "beta", "qn", "kn", "vn", "gn", "betan")
     ins = [getattr(prob, n) for n in names]
     stream = torch.cuda.current_stream(dev)
 
     def step(inputs=None, d_o=None, d_on=None):
         return gb.backward(*(inputs or ins), prob.doc_offsets, prob.prompt_len, prob.block_size,
-                           do if d_o is None else d_o, don if d_on is None else d_on, None, workspace=ws)
+                           do if d_o is None else d_o, don if d_on is None else d_on, None,
+                           conv_w=prob.conv_w, workspace=ws)
 
     steps = max(1, args.steps)
     for _ in range(args.warmup):
@@ -734,7 +742,8 @@ def run_backward(args, name, rank, world, local):
     gbps = nbytes / (ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": gbps, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbps / peaks["hbm_gbs"], "traffic": None, "peak_source": peaks["source"],
-                "kernel": "gdn_backward_kernel", "algorithmic_bytes": nbytes}
+                "kernel": "gdn_backward_kernel" + (" (+ ShortConv forward, backward and weight-gradient kernels)"
+                                                   if prob.conv_width else ""), "algorithmic_bytes": nbytes}
     toks = prob.tokens() * world
     value = toks / (ms / 1e3)
     e2e = None

@@ -1127,8 +1127,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
         }
         if (stop) break;
     }
-    // Drain (thread 0; immediate unless a wait gave up): the last TMA load on each barrier, then,
-    // with one more commit, every MMA.  Then the cp.async groups.
+    // Drain (thread 0): the output stores complete; then (immediate unless a wait gave up) the last
+    // TMA load on each barrier and, with one more commit, every MMA.  Then the cp.async groups.
     if (tid == 0) {
         bulk_wait_all();
         if (s_iss[0] > 0) mbar_wait(&bar_a, (s_iss[0] - 1) & 1, kDrainWaitIters);
