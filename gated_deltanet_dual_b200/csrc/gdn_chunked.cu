@@ -695,6 +695,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // the [P;T] tile after S2, the noisy rows in the K-hat and [P;T] tiles after S3 (not
             // with the in-kernel conv, whose weights live in the K-hat tile at the chunk top)
             const bool o_tma = cstart >= U.s && cstart + CH <= U.s + U.len && ci >= ci_full;
+            // a clean-only chunk of a split unit only carries the state: no P, PT or O
+            const bool need_o = ci >= ci_full;
             const bool n_tma = noisy && !conv && CH * m + CH <= U.R;
             float *s_gam = s_sc[cb] + SC_GAM, *s_beta = s_sc[cb] + SC_BETA;
             float *s_E = s_sc[cb] + SC_E, *s_F = s_sc[cb] + SC_F;
@@ -801,7 +803,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
                         const int i = 32 * ch + c;
-                        tk[c] = (i <= t) ? tk[c] * (Et * s_F[i]) : 0.f;
+                        tk[c] = (i <= t && need_o) ? tk[c] * (Et * s_F[i]) : 0.f;
                     }
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) ppk[c4] = pack8(tk + 8 * c4);
@@ -902,53 +904,55 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             tc_fence_before();
             if ((stop = abort_check())) break;
 
-            // ================= PK2 =================
-            if (tid == 0) {
-                tc_fence_after();
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tb + TM_TK, dK_y + ((kk * 32) >> 4),
-                             dM_t + ((kk * 2048) >> 4), make_idesc_bf16(128, 64, 0, 1), kk > 0);
-                if (noisy) {
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        mma_bf16(tb + TM_ZK, dK_nq + (off >> 4), dK_qk + ((8192 + off) >> 4),
-                                 make_idesc_bf16(128, 64, 0, 0), kk > 0);
+            // ================= PK2 (not in a clean-only chunk: PT feeds only O) =================
+            if (need_o) {
+                if (tid == 0) {
+                    tc_fence_after();
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tb + TM_TK, dK_y + ((kk * 32) >> 4),
+                                 dM_t + ((kk * 2048) >> 4), make_idesc_bf16(128, 64, 0, 1), kk > 0);
+                    if (noisy) {
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                            mma_bf16(tb + TM_ZK, dK_nq + (off >> 4), dK_qk + ((8192 + off) >> 4),
+                                     make_idesc_bf16(128, 64, 0, 0), kk > 0);
+                        }
                     }
+                    commit_mma();
                 }
-                commit_mma();
-            }
-            __syncwarp();
-            wait_mma(20);
-            if (rho < 64) {
-                float pt[32];
-                tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), pt);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(pt + 8 * c4);
-            }
-            if (noisy) {
-                const int e = ((rho & 63) / B) * B - 1;   // chunk-local boundary row (-1: S0)
-                if (fact) {
-                    float zk[32];
-                    tmem_ld32(tmem_addr(tb, q * 32, TM_ZK + 32 * ch), zk);
+                __syncwarp();
+                wait_mma(20);
+                if (rho < 64) {
+                    float pt[32];
+                    tmem_ld32(tmem_addr(tb, q * 32, TM_TK + 32 * ch), pt);
                     tmem_wait_ld();
-                    // the rows already hold Gamma_e Z: M'_Z = (Gamma_e Z K^T) e^{-gamma_i} [i <= e]
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int i = 32 * ch + c;
-                        zk[c] = (i <= e) ? zk[c] * s_F[i] : 0.f;
-                    }
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
-                        *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
-                } else {
-                    mz_rows_exact(sm + OFF_NK, sm + OFF_NQ, tmem_addr(tb, q * 32, TM_ZK + 32 * ch), rho, ch, e, s_gam, s_E);
+                    for (int c4 = 0; c4 < 4; ++c4)
+                        *reinterpret_cast<uint4 *>(sm + OFF_Y + sw128_off(rho, 4 * ch + c4)) = pack8(pt + 8 * c4);
                 }
+                if (noisy) {
+                    const int e = ((rho & 63) / B) * B - 1;   // chunk-local boundary row (-1: S0)
+                    if (fact) {
+                        float zk[32];
+                        tmem_ld32(tmem_addr(tb, q * 32, TM_ZK + 32 * ch), zk);
+                        tmem_wait_ld();
+                        // the rows already hold Gamma_e Z: M'_Z = (Gamma_e Z K^T) e^{-gamma_i} [i <= e]
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int i = 32 * ch + c;
+                            zk[c] = (i <= e) ? zk[c] * s_F[i] : 0.f;
+                        }
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)    // M'_Z: K-major 128 x 64 in d-half 0 of the k~ tile
+                            *reinterpret_cast<uint4 *>(sm + OFF_NK + sw128_off(rho, 4 * ch + c4)) = pack8(zk + 8 * c4);
+                    } else {
+                        mz_rows_exact(sm + OFF_NK, sm + OFF_NQ, tmem_addr(tb, q * 32, TM_ZK + 32 * ch), rho, ch, e, s_gam, s_E);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                if ((stop = abort_check())) break;
             }
-            fence_async_smem();
-            tc_fence_before();
-            if ((stop = abort_check())) break;
 
             // ================= S2: [PT;T] R and the noisy rows' state product =================
             if (tid == 0) {
@@ -986,27 +990,29 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             if (!last && warp > 0) prep_scalars(U, m + 1, cb ^ 1);   // next chunk's scalars meanwhile
             wait_mma(40);
             if (rho < 64) {
-                const int t = rho;
-                const int tok = cstart + t;
-                const bool ok = tok >= U.s && tok < U.s + U.len && ci >= ci_full;
-                const float Gt = s_E[t];
-                __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(P.out) + ((int64_t)tok * H + U.h) * D + 64 * ch;
+                if (need_o) {
+                    const int t = rho;
+                    const int tok = cstart + t;
+                    const bool ok = tok >= U.s && tok < U.s + U.len && ci >= ci_full;
+                    const float Gt = s_E[t];
+                    __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(P.out) + ((int64_t)tok * H + U.h) * D + 64 * ch;
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    float qs[32], pu[32];
-                    tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32 * hf), qs);
-                    tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32 * hf), pu);
-                    tmem_wait_ld();
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float qs[32], pu[32];
+                        tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch + 32 * hf), qs);
+                        tmem_ld32(tmem_addr(tb, q * 32, TM_R1 + 64 * ch + 32 * hf), pu);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) qs[x] = (Gt * qs[x] + pu[x]) * scale;
-                    if (o_tma) {
+                        for (int x = 0; x < 32; ++x) qs[x] = (Gt * qs[x] + pu[x]) * scale;
+                        if (o_tma) {
 #pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4)
-                            *reinterpret_cast<uint4 *>(sm + OFF_Y + ch * 8192 + sw128_off(t, 4 * hf + c4)) = pack8(qs + 8 * c4);
-                    } else if (ok) {
+                            for (int c4 = 0; c4 < 4; ++c4)
+                                *reinterpret_cast<uint4 *>(sm + OFF_Y + ch * 8192 + sw128_off(t, 4 * hf + c4)) = pack8(qs + 8 * c4);
+                        } else if (ok) {
 #pragma unroll
-                        for (int c4 = 0; c4 < 4; ++c4)
-                            *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(qs + 8 * c4);
+                            for (int c4 = 0; c4 < 4; ++c4)
+                                *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(qs + 8 * c4);
+                        }
                     }
                 }
             } else {
