@@ -17,7 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdn_dual.so")
 
-GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_ALIGNMENT, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(6)
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_ALIGNMENT, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, GDN_ERR_BOUNDS = range(7)
 GDN_BF16, GDN_FP32 = 0, 1
 ALGO_AUTO, ALGO_SEQUENTIAL, ALGO_CHUNKED, ALGO_ROUTE1, ALGO_PIPELINED = 0, 1, 2, 3, 4
 EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device_status",

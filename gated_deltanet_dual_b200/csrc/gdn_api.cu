@@ -63,6 +63,7 @@ const char *gdn_status_string(gdn_status s) {
         case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
         case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
         case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+        case GDN_ERR_BOUNDS: return "GDN_ERR_BOUNDS";
     }
     return "GDN_ERR_UNKNOWN";
 }

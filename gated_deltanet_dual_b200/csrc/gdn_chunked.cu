@@ -576,6 +576,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             }
         }
         (void)buf;
+        if (nb && !GDN_IN_RANGE(P.ws, sr < CH ? (gp - P.g) < P.T * H : (gp - P.gn) < (int64_t)V * TR * H, 201)) nb = 0;
         cp_async4(&s_raw[0][sr], gp, nb);
         cp_async4(&s_raw[1][sr], bp, nb);
         cp_async_commit();
@@ -676,7 +677,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8) *reinterpret_cast<uint4 *>(s0 + sw128_off(rho, c8)) = z;
             fence_async_smem();
-            if (U.nchunks == 0 && final_part) {
+            if (U.nchunks == 0 && final_part && GDN_IN_RANGE(P.ws, U.n < P.N && U.h < H, 203)) {
                 float *fs = P.final_state + ((int64_t)U.n * H + U.h) * D * D + (int64_t)rho * D + 64 * ch;
 #pragma unroll
                 for (int c = 0; c < 64; c += 4) *reinterpret_cast<float4 *>(fs + c) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -711,7 +712,8 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 for (int it = tid; it < 3 * 128 * 4; it += kThreads) {   // (tensor X, channel c, tap j)
                     const int X = it >> 9, c = (it >> 2) & 127, j = it & 3;
                     const int dst = (X * 128 + ((c & 7) >> 1) * 32 + (j >> 1) * 16 + (c >> 3)) * 4 + (j & 1) * 2 + (c & 1);
-                    cp_async4(sm + OFF_CW + dst * 4, P.conv_w + (((int64_t)X * H + U.h) * 128 + c) * 4 + j, 4);
+                    const int64_t wi = (((int64_t)X * H + U.h) * 128 + c) * 4 + j;
+                    cp_async4(sm + OFF_CW + dst * 4, P.conv_w + wi, GDN_IN_RANGE(P.ws, wi < 3LL * H * 128 * 4, 202) ? 4 : 0);
                 }
                 cp_async_commit();
             }
@@ -1008,7 +1010,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
 #pragma unroll
                             for (int c4 = 0; c4 < 4; ++c4)
                                 *reinterpret_cast<uint4 *>(sm + OFF_Y + ch * 8192 + sw128_off(t, 4 * hf + c4)) = pack8(qs + 8 * c4);
-                        } else if (ok) {
+                        } else if (ok && GDN_IN_RANGE(P.ws, tok >= 0 && tok < P.T, 205)) {
 #pragma unroll
                             for (int c4 = 0; c4 < 4; ++c4)
                                 *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(qs + 8 * c4);
@@ -1037,7 +1039,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // ================= S3 =================
             if (tid == 0) {
                 tc_fence_after();
-                if (o_tma && !dead) {
+                if (o_tma && !dead && GDN_IN_RANGE(P.ws, cstart >= 0 && cstart + CH <= P.T, 206)) {
                     tma_store_3d(&M.o, sm + OFF_Y, 0, U.h, cstart);
                     tma_store_3d(&M.o, sm + OFF_Y + 8192, 64, U.h, cstart);
                     bulk_commit();
@@ -1082,7 +1084,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
 #pragma unroll
             for (int c8 = 0; c8 < 8; ++c8)
                 *reinterpret_cast<uint4 *>(srow + sw128_off(rho, c8)) = pack8(S + 8 * c8);
-            if (last && final_part) {
+            if (last && final_part && GDN_IN_RANGE(P.ws, U.n < P.N && U.h < H, 204)) {
                 float *fs = P.final_state + ((int64_t)U.n * H + U.h) * D * D + (int64_t)rho * D + 64 * ch;
 #pragma unroll
                 for (int c = 0; c < 64; c += 4)
@@ -1112,7 +1114,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                         for (int c4 = 0; c4 < 4; ++c4)
                             *reinterpret_cast<uint4 *>(sm + OFF_KH + vw * 16384 + ch * 8192 + sw128_off(jj, 4 * hf + c4)) =
                                 pack8(on + 8 * c4);
-                    } else if (ok) {
+                    } else if (ok && GDN_IN_RANGE(P.ws, (int64_t)vw * TR + U.roff + rr < (int64_t)V * TR, 207)) {
 #pragma unroll
                         for (int c4 = 0; c4 < 4; ++c4)
                             *reinterpret_cast<uint4 *>(orow + 32 * hf + 8 * c4) = pack8(on + 8 * c4);
@@ -1124,10 +1126,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             cb ^= 1;
             if ((stop = abort_check())) break;
             if (tid == 0 && n_tma && !dead) {
-                for (int vw = 0; vw < V && vw < 2; ++vw)
+                for (int vw = 0; vw < V && vw < 2; ++vw) {
+                    const int64_t row0 = (int64_t)vw * TR + U.roff + CH * m;
+                    if (!GDN_IN_RANGE(P.ws, row0 >= 0 && row0 + CH <= (int64_t)V * TR, 208)) continue;
                     for (int hf = 0; hf < 2; ++hf)
-                        tma_store_3d(&M.on, sm + OFF_KH + vw * 16384 + hf * 8192, hf * 64, U.h,
-                                     vw * (int)TR + U.roff + CH * m);
+                        tma_store_3d(&M.on, sm + OFF_KH + vw * 16384 + hf * 8192, hf * 64, U.h, (int)row0);
+                }
                 bulk_commit();
             }
         }

@@ -43,6 +43,7 @@ struct ConvPassParams {
     const __nv_bfloat16 *x[3], *xn[3];     // raw clean [T, H, d] and noisy [V, T_R, H, d]
     __nv_bfloat16 *y[3], *yn[3];           // convolved (disjoint from the raw inputs)
     const float *w;                        // [3, H d, 4]
+    WorkspaceHeader *ws;                   // status words (range-checking build)
     int64_t T, TR;
     int32_t N, H, d, V, B;
     int32_t doc_start[kMaxDocs + 1];
@@ -101,7 +102,7 @@ __device__ __forceinline__ void conv_row(const uint4 (*cw)[3][kSliceGroups], con
 #pragma unroll
             for (int c = 0; c < 8; ++c) acc[c] = fmaf(wv[c], f[c], acc[c]);
         }
-        *reinterpret_cast<uint4 *>(dst[X]) = pack_bf16x8(acc);
+        *reinterpret_cast<uint4 *>(dst[X]) = pack_bf16x8(acc);   // dst checked by the caller
     }
 }
 
@@ -148,7 +149,8 @@ __global__ void __launch_bounds__(kPassThreads) conv_pass_kernel(const __grid_co
         // clean window: row k holds position a - 3 + k
         for (int t = warp; t < kWin * 3; t += kPassWarps) {
             const int k = t / 3, X = t - 3 * (t / 3), pos = a - (kTaps - 1) + k;
-            if (lane_on && pos >= 0 && pos < len) cp_async16(&cw[k][X][lane], P.x[X] + (s + pos) * hd + col);
+            if (lane_on && pos >= 0 && pos < len && GDN_IN_RANGE(P.ws, s + pos < P.T, 301))
+                cp_async16(&cw[k][X][lane], P.x[X] + (s + pos) * hd + col);
         }
         for (int vw = 0; vw < P.V && nlo < nhi; ++vw) {
             if (vw > 0) __syncthreads();                          // view vw-1 is done with nw
@@ -156,7 +158,8 @@ __global__ void __launch_bounds__(kPassThreads) conv_pass_kernel(const __grid_co
             // noisy window: row k holds response index i0 - 3 + k
             for (int t = warp; t < kWin * 3; t += kPassWarps) {
                 const int k = t / 3, X = t - 3 * (t / 3), i = i0 - (kTaps - 1) + k;
-                if (lane_on && i >= 0 && i < L) cp_async16(&nw[k][X][lane], P.xn[X] + (vbase + i) * hd + col);
+                if (lane_on && i >= 0 && i < L && GDN_IN_RANGE(P.ws, vbase + i < (int64_t)P.V * P.TR, 302))
+                    cp_async16(&nw[k][X][lane], P.xn[X] + (vbase + i) * hd + col);
             }
             cp_async_commit();
             cp_async_wait_all();
@@ -170,7 +173,7 @@ __global__ void __launch_bounds__(kPassThreads) conv_pass_kernel(const __grid_co
                         __nv_bfloat16 *dst[3];
 #pragma unroll
                         for (int X = 0; X < 3; ++X) dst[X] = P.y[X] + (s + a + r) * hd + col;
-                        conv_row(cw, nw, w_s, lane, r + kTaps - 1, kind, dst);
+                        if (GDN_IN_RANGE(P.ws, s + a + r < P.T, 303)) conv_row(cw, nw, w_s, lane, r + kTaps - 1, kind, dst);
                     }
                 }
                 for (int r = warp; r < kTile; r += kPassWarps) {
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(kPassThreads) conv_pass_kernel(const __grid_co
                     __nv_bfloat16 *dst[3];
 #pragma unroll
                     for (int X = 0; X < 3; ++X) dst[X] = P.yn[X] + (vbase + i) * hd + col;
-                    conv_row(cw, nw, w_s, lane, r + kTaps - 1, kind, dst);
+                    if (GDN_IN_RANGE(P.ws, vbase + i < (int64_t)P.V * P.TR, 304)) conv_row(cw, nw, w_s, lane, r + kTaps - 1, kind, dst);
                 }
             }
         }
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(kPassThreads) conv_pass_kernel(const __grid_co
                     __nv_bfloat16 *dst[3];
 #pragma unroll
                     for (int X = 0; X < 3; ++X) dst[X] = P.y[X] + (s + a + r) * hd + col;
-                    conv_row(cw, nw, w_s, lane, r + kTaps - 1, kind, dst);
+                    if (GDN_IN_RANGE(P.ws, s + a + r < P.T, 303)) conv_row(cw, nw, w_s, lane, r + kTaps - 1, kind, dst);
                 }
         }
         __syncthreads();                                          // windows free for the next tile
@@ -226,6 +229,7 @@ cudaError_t launch_conv_pass(const Params &p, void *buf, cudaStream_t stream) {
         C.yn[X] = b + 3 * clean + X * noisy;
     }
     C.w = p.conv_w;
+    C.ws = p.ws;
     C.T = p.T; C.TR = p.TR; C.N = p.N; C.H = p.H; C.d = p.dk; C.V = p.V; C.B = p.B;
     std::memcpy(C.doc_start, p.doc_start, sizeof(C.doc_start));
     std::memcpy(C.doc_prompt, p.doc_prompt, sizeof(C.doc_prompt));

@@ -25,10 +25,26 @@ constexpr uint32_t kDrainWaitIters = 1u << 22;
 struct WorkspaceHeader {
     int32_t status;         // GDN_OK or GDN_ERR_TIMEOUT, written by kernels
     int32_t next_unit;      // dynamic work counter of the persistent kernel
-    int32_t timeout_where;  // diagnostic: which wait gave up
+    int32_t timeout_where;  // diagnostic: which wait gave up (or, range-checking build, which check failed)
     int32_t pad[61];        // header is 256 bytes
 };
 static_assert(sizeof(WorkspaceHeader) == 256, "workspace header is 256 bytes");
+
+// Range checks of the debug build (compiled with -DGDN_DEBUG_BOUNDS, libgdn_dual_debug.so): a
+// failed check records GDN_ERR_BOUNDS and its site in the workspace status words, and the access
+// it guards is skipped.  In the normal build a check is `true` and its condition is not evaluated.
+#ifdef GDN_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(WorkspaceHeader *ws, bool ok, int where) {
+    if (!ok) {
+        atomicCAS(&ws->status, 0, (int)GDN_ERR_BOUNDS);
+        atomicCAS(&ws->timeout_where, 0, where);
+    }
+    return ok;
+}
+#define GDN_IN_RANGE(ws, cond, where) ::gdn::bounds_ok((ws), (cond), (where))
+#else
+#define GDN_IN_RANGE(ws, cond, where) true
+#endif
 
 struct Params {
     const void *q, *k, *v;

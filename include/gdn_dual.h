@@ -59,7 +59,12 @@ typedef enum {
     GDN_ERR_ALIGNMENT = 2,     /* a tensor pointer is not 16-byte aligned */
     GDN_ERR_UNSUPPORTED = 3,   /* valid but not implemented here (d, dtype, conv width, algo) */
     GDN_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
-    GDN_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (reported by the device) */
+    GDN_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (reported by the device) */
+    GDN_ERR_BOUNDS = 6         /* range-checking build only (libgdn_dual_debug.so, compiled with
+                                  GDN_DEBUG_BOUNDS): a device-side index check failed and the
+                                  access was skipped; the check's site is the `where` code of
+                                  gdn_dual_read_device_status_where (201-209 chunked kernel,
+                                  301-304 ShortConv pass) */
 } gdn_status;
 
 typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;

@@ -39,11 +39,20 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), f"{name} declared in include/ but not exported"
 
 
+def test_range_checking_build_exports_every_declared_symbol():
+    """libgdn_dual_debug.so (GDN_DEBUG_BOUNDS) is a drop-in replacement: same C ABI."""
+    import ctypes
+    from gated_deltanet_dual_b200 import build as gbuild
+    lib = ctypes.CDLL(gbuild.build_debug())
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported by the range-checking build"
+
+
 def test_version_and_status_strings():
     lib = b.load_library()
     assert lib.gdn_dual_version() >= 100
     for code, name in enumerate(["GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_ALIGNMENT", "GDN_ERR_UNSUPPORTED",
-                                 "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT"]):
+                                 "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT", "GDN_ERR_BOUNDS"]):
         assert b.status_string(code) == name
     assert b.status_string(99) == "GDN_ERR_UNKNOWN"
 
