@@ -403,7 +403,9 @@ __device__ __noinline__ int next_work_item(WorkspaceHeader *ws, int *s_next) {
 }
 
 // TW: the test instantiation, whose waits poll with the caller's bound (gdn_dual_forward_test_wait_limit).
-template <int B, bool TW = false>
+// CONV: the instantiation with the fused ShortConv prologue (the other one has no conv code at
+// all, which keeps its loop body smaller for the instruction cache).
+template <int B, bool TW = false, bool CONV = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps M) {
     extern __shared__ uint8_t smraw[];
@@ -430,7 +432,7 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
     const int H = P.H, V = P.V;
     const int64_t TR = P.TR;
     const float scale = P.scale;
-    const bool conv = P.conv_width > 0;
+    constexpr bool conv = CONV;   // the host launches CONV exactly when P.conv_width > 0
 
     if (tid == 0) {
         mbar_init(&bar_a, 1);
@@ -1191,7 +1193,10 @@ cudaError_t launch_chunked_views(const Params &p, bool pipelined, cudaStream_t s
         cudaError_t e = cudaSuccess;
         for (auto fn : {gdn_chunked_kernel<1>, gdn_chunked_kernel<2>, gdn_chunked_kernel<4>,
                         gdn_chunked_kernel<8>, gdn_chunked_kernel<16>, gdn_chunked_kernel<32>,
-                        gdn_chunked_kernel<4, true>}) {
+                        gdn_chunked_kernel<1, false, true>, gdn_chunked_kernel<2, false, true>,
+                        gdn_chunked_kernel<4, false, true>, gdn_chunked_kernel<8, false, true>,
+                        gdn_chunked_kernel<16, false, true>, gdn_chunked_kernel<32, false, true>,
+                        gdn_chunked_kernel<4, true>, gdn_chunked_kernel<4, true, true>}) {
             cudaError_t r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
             if (r != cudaSuccess) e = r;
         }
@@ -1203,20 +1208,28 @@ cudaError_t launch_chunked_views(const Params &p, bool pipelined, cudaStream_t s
     Params q = p;
     q.parts = (noisy && 2 * p.num_units <= sms) ? 2 : 1;
     const int grid = std::min(p.num_units * q.parts, sms);
+    const bool conv = p.conv_width > 0;
     if (p.wait_test) {           // the test entry point: B = 4 only
         if (p.B != 4) return cudaErrorNotSupported;
-        gdn_chunked_kernel<4, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);
+        if (conv) gdn_chunked_kernel<4, true, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);
+        else gdn_chunked_kernel<4, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);
         return cudaGetLastError();
     }
+#define GDN_CHUNKED_CASE(b)                                                                        \
+    case b:                                                                                        \
+        if (conv) gdn_chunked_kernel<b, false, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); \
+        else gdn_chunked_kernel<b><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);              \
+        break;
     switch (p.B) {
-        case 1: gdn_chunked_kernel<1><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
-        case 2: gdn_chunked_kernel<2><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
-        case 4: gdn_chunked_kernel<4><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
-        case 8: gdn_chunked_kernel<8><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
-        case 16: gdn_chunked_kernel<16><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
-        case 32: gdn_chunked_kernel<32><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps); break;
+        GDN_CHUNKED_CASE(1)
+        GDN_CHUNKED_CASE(2)
+        GDN_CHUNKED_CASE(4)
+        GDN_CHUNKED_CASE(8)
+        GDN_CHUNKED_CASE(16)
+        GDN_CHUNKED_CASE(32)
         default: return cudaErrorInvalidValue;
     }
+#undef GDN_CHUNKED_CASE
     return cudaGetLastError();
 }
 
