@@ -206,6 +206,20 @@ gdn_status forward_impl(const gdn_dual_desc *desc,
         }
     } else if (algo == GDN_ALGO_CHUNKED || algo == GDN_ALGO_PIPELINED) {
         err = gdn::launch_chunked(P, algo == GDN_ALGO_PIPELINED, st);
+    } else if (algo == GDN_ALGO_ROUTE1 && P.V > 0 && !P.wait_test &&
+               gdn::route1_tc_supported(desc->dtype, desc->d_k, B, desc->conv_width) && desc->d_k == desc->d_v) {
+        // Route I on tensor cores: the clean stream exporting the state before every response
+        // block (bf16 blobs of 32 KB, in the space the fp32 states take otherwise), then the refine
+        // kernel over every (block, head, pair of views)
+        gdn::Params Q = P;
+        Q.states = static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader);
+        Q.V = 0;
+        err = gdn::launch_chunked(Q, false, st);
+        if (err == cudaSuccess) {
+            cudaMemsetAsync(&static_cast<gdn::WorkspaceHeader *>(workspace)->next_unit, 0, sizeof(int32_t), st);
+            Q.V = P.V;
+            err = gdn::launch_route1_refine(Q, st);
+        }
     } else if (algo == GDN_ALGO_ROUTE1) {
         err = gdn::launch_route1(P, desc->dtype,
                                  reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader)), st);

@@ -71,6 +71,8 @@ constexpr uint32_t TM_R1 = 128;    // k~k~^T | [P U; U]
 constexpr uint32_t TM_N = 256;     // noisy accumulator (WV + Gamma_e Z S0 + M'_Z U)
 constexpr uint32_t TM_TK = 384;    // [Q;K]K^T | P T
 constexpr uint32_t TM_ZK = 448;    // Z K^T
+// Route I export j (the block starting at row j B): free columns once S2's products are read
+__device__ __forceinline__ uint32_t export_col(int j) { return j == 1 ? TM_N : (j == 2 ? TM_R1 : TM_TK); }
 
 __device__ __forceinline__ void bar_all() { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); }
 __device__ __forceinline__ void bar_math() { bar_all(); }
@@ -405,7 +407,13 @@ __device__ __noinline__ int next_work_item(WorkspaceHeader *ws, int *s_next) {
 // TW: the test instantiation, whose waits poll with the caller's bound (gdn_dual_forward_test_wait_limit).
 // CONV: the instantiation with the fused ShortConv prologue (the other one has no conv code at
 // all, which keeps its loop body smaller for the instruction cache).
-template <int B, bool TW = false, bool CONV = false>
+// EXPORT: Route I's first stage (no noisy views; B = 16 or 32): besides the clean outputs, the
+// state before every response block, S_e = Gamma_e S0 + Khat_e^T U with Khat_e,i =
+// e^{gamma_e - gamma_i} k_i (i <= e), is written to P.states as a 32 KB blob in the bf16 S0 tile
+// layout (the kernels' MMA B operand): the chunk's own S0 for the block at its row 0, and one
+// more MMA per later block start, into tensor-memory columns and shared tiles that carry the
+// noisy rows when there are views.
+template <int B, bool TW = false, bool CONV = false, bool EXPORT = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Maps M) {
     extern __shared__ uint8_t smraw[];
@@ -749,6 +757,19 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             __syncwarp();
             if ((stop = abort_check())) break;
             const bool fact = s_okw[cb][0] && s_okw[cb][1];
+            // Route I export: blocks that start in this chunk (its rows are response positions)
+            constexpr int kNbE = EXPORT ? CH / B : 0;
+            const int eb0 = (CH * m) / B, enb = U.R / B;     // first block of the chunk, blocks in all
+            const bool exporting = EXPORT && need_o && m >= 0;
+            auto blob = [&](int b) {
+                return static_cast<uint8_t *>(P.states) + ((int64_t)(U.roff / B + b) * H + U.h) * 32768;
+            };
+            if constexpr (EXPORT) {
+                if (tid == 0 && exporting && eb0 < enb && !dead) {   // the first block starts from S0
+                    bulk_store(blob(eb0), sm + OFF_S0, 32768);
+                    bulk_commit();
+                }
+            }
 
             // ================= PK1: [Q;K]K^T now, the noisy products once group B is in ========
             if (tid == 0) {
@@ -978,6 +999,27 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // lane 0 lets the next chunk's group A overwrite the tile once [Q;K] and Z are consumed.
             if (warp > 0) {
                 build_khat();
+                if constexpr (EXPORT) {
+                    // Khat_e for the block starting at row j B (e = j B - 1), j >= 1: K rows i <= e
+                    // scaled by e^{gamma_e - gamma_i}, the rest zero; MN-major A tiles at NQ
+                    if (exporting) {
+                        for (int it = tid - 32; it < 64 * 16; it += kMathThreads - 32) {
+                            const int t = it >> 4, c16 = it & 15, hf = c16 >> 3, c8 = c16 & 7;
+                            float f[8], g8[8];
+                            unpack8(*reinterpret_cast<const uint4 *>(sm + OFF_QK + hf * 16384 + sw128_off(64 + t, c8)), f);
+#pragma unroll
+                            for (int j = 1; j < kNbE; ++j) {
+                                const int e = j * B - 1;
+                                const float sc = t <= e ? exp2f(s_gam[e] - s_gam[t]) : 0.f;
+#pragma unroll
+                                for (int x = 0; x < 8; ++x) g8[x] = f[x] * sc;
+                                *reinterpret_cast<uint4 *>(sm + OFF_NQ + (j - 1) * 16384 + hf * 8192 + sw128_off(t, c8)) =
+                                    pack8(g8);
+                            }
+                        }
+                        fence_async_smem();
+                    }
+                }
                 bar_arrive_khat();
             } else {
                 bar_sync_khat();
@@ -1054,6 +1096,18 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                         mma_bf16(tb + TM_N, dK_nk + ((kk * 32) >> 4), dM_v + ((kk * 2048) >> 4),
                                  make_idesc_bf16(128, 128, 0, 1), 1u);
                 }
+                if constexpr (EXPORT) {
+                    if (exporting) {
+                        for (int j = 1; j < kNbE; ++j) {
+                            if (eb0 + j >= enb) break;
+                            const uint64_t dM_khe = make_sdesc(smem_u32(sm + OFF_NQ + (j - 1) * 16384), 8192, 1024);
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_bf16(tb + export_col(j), dM_khe + ((kk * 2048) >> 4), dM_v + ((kk * 2048) >> 4),
+                                         make_idesc_bf16(128, 128, 1, 1), kk > 0);
+                        }
+                    }
+                    bulk_wait_read_all();    // the S0 blob has been read before the update rewrites S0
+                }
                 commit_mma();
                 if (!last && !dead) {
                     if (!kwait<TW>(&bar_mma, ph_mma & 1, kWaitIters, P.wait_iters)) {
@@ -1072,6 +1126,26 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             wait_mma(50);
             const float GC = s_E[CH - 1];
             uint8_t *srow = sm + OFF_S0 + ch * 16384;
+            if constexpr (EXPORT) {
+                if (exporting) {
+                    for (int j = 1; j < kNbE; ++j) {
+                        if (eb0 + j >= enb) break;
+                        const float Ge = s_E[j * B - 1];
+                        uint8_t *st = sm + OFF_NQ + (j - 1) * 32768 + ch * 16384;
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            float ex[32];
+                            tmem_ld32(tmem_addr(tb, q * 32, export_col(j) + 64 * ch + 32 * hf), ex);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) ex[x] = fmaf(Ge, S[32 * hf + x], ex[x]);
+#pragma unroll
+                            for (int c4 = 0; c4 < 4; ++c4)
+                                *reinterpret_cast<uint4 *>(st + sw128_off(rho, 4 * hf + c4)) = pack8(ex + 8 * c4);
+                        }
+                    }
+                }
+            }
             {
                 float ds0[32], ds1[32];
                 tmem_ld32(tmem_addr(tb, q * 32, TM_R0 + 64 * ch), ds0);
@@ -1127,6 +1201,15 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             tc_fence_before();
             cb ^= 1;
             if ((stop = abort_check())) break;
+            if constexpr (EXPORT) {
+                if (tid == 0 && exporting && !dead) {
+                    for (int j = 1; j < kNbE; ++j) {
+                        if (eb0 + j >= enb) break;
+                        bulk_store(blob(eb0 + j), sm + OFF_NQ + (j - 1) * 32768, 32768);
+                    }
+                    bulk_commit();
+                }
+            }
             if (tid == 0 && n_tma && !dead) {
                 for (int vw = 0; vw < V && vw < 2; ++vw) {
                     const int64_t row0 = (int64_t)vw * TR + U.roff + CH * m;
@@ -1196,7 +1279,8 @@ cudaError_t launch_chunked_views(const Params &p, bool pipelined, cudaStream_t s
                         gdn_chunked_kernel<1, false, true>, gdn_chunked_kernel<2, false, true>,
                         gdn_chunked_kernel<4, false, true>, gdn_chunked_kernel<8, false, true>,
                         gdn_chunked_kernel<16, false, true>, gdn_chunked_kernel<32, false, true>,
-                        gdn_chunked_kernel<4, true>, gdn_chunked_kernel<4, true, true>}) {
+                        gdn_chunked_kernel<4, true>, gdn_chunked_kernel<4, true, true>,
+                        gdn_chunked_kernel<16, false, false, true>, gdn_chunked_kernel<32, false, false, true>}) {
             cudaError_t r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
             if (r != cudaSuccess) e = r;
         }
@@ -1206,9 +1290,16 @@ cudaError_t launch_chunked_views(const Params &p, bool pipelined, cudaStream_t s
     // Few units: two CTAs per unit (see the kernel's unit loop).
     const int sms = num_sms > 0 ? num_sms : 148;
     Params q = p;
-    q.parts = (noisy && 2 * p.num_units <= sms) ? 2 : 1;
+    q.parts = ((noisy || p.states) && 2 * p.num_units <= sms) ? 2 : 1;
     const int grid = std::min(p.num_units * q.parts, sms);
     const bool conv = p.conv_width > 0;
+    if (p.states) {              // Route I's first stage: no views, no ShortConv, B = 16 or 32
+        if (noisy || conv || p.wait_test) return cudaErrorNotSupported;
+        if (p.B == 16) gdn_chunked_kernel<16, false, false, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);
+        else if (p.B == 32) gdn_chunked_kernel<32, false, false, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);
+        else return cudaErrorNotSupported;
+        return cudaGetLastError();
+    }
     if (p.wait_test) {           // the test entry point: B = 4 only
         if (p.B != 4) return cudaErrorNotSupported;
         if (conv) gdn_chunked_kernel<4, true, true><<<grid, kThreads, SMEM_BYTES, stream>>>(q, maps);

@@ -55,6 +55,7 @@ struct Params {
     void *out, *out_noisy;
     float *final_state;
     WorkspaceHeader *ws;
+    void *states;           // Route I on tensor cores: the block-boundary state blobs (else NULL)
     int64_t T, TR;
     int32_t N, H, dk, dv, V, B, conv_width, num_units;
     int32_t parts;                    // chunked kernel: CTAs per unit (1, or 2 when units are few)
@@ -80,6 +81,11 @@ cudaError_t launch_conv_pass(const Params &p, void *buf, cudaStream_t stream);
 // Route I: clean chain writing block-boundary states into `states`, then block refinement.
 cudaError_t launch_route1(const Params &p, int dtype, float *states, cudaStream_t stream);
 bool chunked_supported(int dtype, int d, int B, int conv_width);
+// Route I on tensor cores (gdn_route1_tc.cu): bf16, d = 128, B = 16 or 32, no ShortConv.  Stage 1
+// is launch_chunked with P.states set and no views (the chunked kernel's EXPORT instantiation),
+// stage 2 refines every (boundary state, pair of views) from P.states.
+bool route1_tc_supported(int dtype, int d, int B, int conv_width);
+cudaError_t launch_route1_refine(const Params &p, cudaStream_t stream);
 // The backward on validated arguments, inputs and upstream gradients of element type `dtype`;
 // the workspace must hold gdn_dual_backward_workspace_size() bytes for the descriptor.
 gdn_status run_backward(const gdn_dual_desc *desc, int dtype, const void *q, const void *k, const void *v,

@@ -50,3 +50,31 @@ def test_route1_long_document_tiles():
     prob = synth.make_problem_from_layout(offs, [232], num_heads=2, d_k=128, d_v=128, block_size=16, num_views=2,
                                           dtype="bf16", seed=9, device="cuda")
     _check(prob, 2e-2)
+
+
+@pytest.mark.parametrize("B", [16, 32])
+@pytest.mark.parametrize("V", [1, 3])
+def test_route1_tensor_cores_odd_views_and_prompts(B, V):
+    """bf16, d = 128, B = 16 / 32: Route I on tensor cores (the chunked kernel exporting the state
+    before every response block, then the refine kernel by pairs of views; V odd leaves a pair with
+    one view).  Prompts that are not whole chunks, an empty response, and few units (split over two
+    CTAs)."""
+    lens, prompts = [40 + 4 * B, 96 + 6 * B, 72, 3 * B], [40, 96, 72, 0]
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    prob = synth.make_problem_from_layout(offs, prompts, num_heads=2, d_k=128, d_v=128, block_size=B, num_views=V,
+                                          dtype="bf16", seed=60 + B + V, device="cuda")
+    _check(prob, 2e-2)
+
+
+@pytest.mark.parametrize("wl", ["train_8x4096_h16_d128_B16", "train_8x4096_h16_d128_B32"])
+def test_route1_tensor_cores_match_fused_kernel_full_size(wl):
+    """The full training shape: Route I on tensor cores against the fused chunked kernel (both
+    checked against the oracle elsewhere), every output element, within the bf16 bar."""
+    prob = synth.make_problem(wl, device="cuda")
+    r1 = b.forward_problem(prob, algo=b.ALGO_ROUTE1)
+    r2 = b.forward_problem(prob, algo=b.ALGO_CHUNKED)
+    torch.cuda.synchronize()
+    for name, x, y in zip(("out", "out_noisy", "final_state"), r1, r2):
+        scale = float(y.abs().max())
+        err = float((x.float() - y.float()).abs().max())
+        assert err <= 2e-2 * scale, f"{name}: {err:.3e} vs {scale:.3e}"
