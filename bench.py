@@ -44,7 +44,7 @@ KERNEL_SOURCES = {
     gb.ALGO_PIPELINED: ["gated_deltanet_dual_b200/csrc/gdn_pipe.cu", "gated_deltanet_dual_b200/csrc/gdn_chunk_common.cuh"],
     gb.ALGO_ROUTE1: ["gated_deltanet_dual_b200/csrc/gdn_decode.cu"],
     "route1_tc": ["gated_deltanet_dual_b200/csrc/gdn_route1_tc.cu", "gated_deltanet_dual_b200/csrc/gdn_chunked.cu",
-                  "gated_deltanet_dual_b200/csrc/gdn_chunk_common.cuh"],
+                  "gated_deltanet_dual_b200/csrc/gdn_chunk_common.cuh", "gated_deltanet_dual_b200/csrc/gdn_conv.cu"],
     "attention": ["gated_deltanet_dual_b200/csrc/gdn_attention.cu"],
 }
 KERNEL_NAMES = {gb.ALGO_SEQUENTIAL: "gdn_sequential_kernel", gb.ALGO_CHUNKED: "gdn_chunked_kernel",
@@ -891,13 +891,14 @@ def main():
     # kernel on the convolved copies; the events time both, against the forward's algorithmic bytes
     conv_pass = (algo == gb.ALGO_AUTO and used_algo == gb.ALGO_CHUNKED and prob.conv_width == 4
                  and gb.workspace_size(desc, prob.doc_offsets) > 256)
-    # Route I on tensor cores (bf16, d = 128, B in {16, 32}, no ShortConv, at least one view)
+    # Route I on tensor cores (bf16, d = 128, B in {16, 32}; ShortConv as a pass of its own first)
     r1_tc = (used_algo == gb.ALGO_ROUTE1 and prob.q.dtype == torch.bfloat16 and d == 128
-             and prob.block_size in (16, 32) and prob.conv_width == 0 and V > 0)
+             and prob.block_size in (16, 32) and (V > 0 or prob.conv_width == 4))
     if r1_tc:
         traffic = profiled_traffic("route1_tc", wl.name, work["bytes"])
     kname = ("conv_pass_kernel + " + KERNEL_NAMES[used_algo] + " (one forward call)") if conv_pass \
-        else KERNEL_NAMES["route1_tc"] if r1_tc else KERNEL_NAMES.get(used_algo)
+        else ("conv_pass_kernel + " if prob.conv_width == 4 else "") + KERNEL_NAMES["route1_tc"] if r1_tc \
+        else KERNEL_NAMES.get(used_algo)
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
                 "peak_source": peaks["source"], "kernel": kname,

@@ -38,6 +38,11 @@ bool desc_supported(const gdn_dual_desc *d) {
     return true;
 }
 
+// GDN_ALGO_ROUTE1 on tensor cores (else the CUDA-core form)
+bool route1_tc_form(const gdn_dual_desc *d) {
+    return d->d_k == d->d_v && gdn::route1_tc_supported(d->dtype, d->d_k, d->block_size, d->conv_width);
+}
+
 // AUTO with ShortConv on the chunked path runs the conv as a pass of its own (into the workspace)
 // when the workspace has room for the convolved inputs; else the chunked kernel's fused prologue.
 bool conv_pass_wanted(const gdn_dual_desc *d) {
@@ -101,7 +106,11 @@ size_t gdn_dual_workspace_size_route1(const gdn_dual_desc *desc, const int32_t *
         TR += len - prompt_len_host[n];
     }
     const size_t states = (size_t)(TR / desc->block_size) * desc->num_heads * desc->d_k * desc->d_v * sizeof(float);
-    return sizeof(gdn::WorkspaceHeader) + ((states + 255) / 256) * 256;
+    size_t bytes = sizeof(gdn::WorkspaceHeader) + ((states + 255) / 256) * 256;
+    if (desc->conv_width > 0 && route1_tc_form(desc))   // its conv pass: the convolved copies follow the states
+        bytes += gdn::conv_pass_bytes(doc_offsets_host[desc->num_docs], TR, desc->num_heads, desc->d_k,
+                                      desc->num_views);
+    return bytes;
 }
 
 }  // extern "C"
@@ -139,8 +148,10 @@ gdn_status forward_impl(const gdn_dual_desc *desc,
     const bool noisy = V > 0 && TR > 0;
     if (noisy && (!qn || !kn || !vn || !gn || !betan || !out_noisy)) return GDN_ERR_INVALID_ARG;
     if (!workspace || workspace_bytes < sizeof(gdn::WorkspaceHeader)) return GDN_ERR_INVALID_ARG;
-    const size_t route1_states = (size_t)(TR / B) * H * desc->d_k * desc->d_v * sizeof(float);
-    if (desc->algo == GDN_ALGO_ROUTE1 && workspace_bytes < sizeof(gdn::WorkspaceHeader) + route1_states)
+    const size_t route1_states = (((size_t)(TR / B) * H * desc->d_k * desc->d_v * sizeof(float) + 255) / 256) * 256;
+    const size_t route1_conv =
+        desc->conv_width > 0 && route1_tc_form(desc) ? gdn::conv_pass_bytes(T, TR, H, desc->d_k, V) : 0;
+    if (desc->algo == GDN_ALGO_ROUTE1 && workspace_bytes < sizeof(gdn::WorkspaceHeader) + route1_states + route1_conv)
         return GDN_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, g, beta, qn, kn, vn, gn, betan, conv_w, out, out_noisy, final_state, workspace};
     for (const void *p : ptrs)
@@ -151,7 +162,11 @@ gdn_status forward_impl(const gdn_dual_desc *desc,
         !gdn::chunked_supported(desc->dtype, desc->d_k, B, desc->conv_width))
         return GDN_ERR_UNSUPPORTED;
     if (algo == GDN_ALGO_PIPELINED && desc->conv_width != 0) return GDN_ERR_UNSUPPORTED;
-    if (algo == GDN_ALGO_ROUTE1 && (desc->conv_width != 0 || B > 64)) return GDN_ERR_UNSUPPORTED;
+    // Route I: tensor cores for bf16, d = 128, B in {16, 32} (ShortConv through the conv pass);
+    // otherwise CUDA cores, without ShortConv
+    const bool route1_tc = algo == GDN_ALGO_ROUTE1 && route1_tc_form(desc);
+    if (algo == GDN_ALGO_ROUTE1 && (B > 64 || (desc->conv_width != 0 && (!route1_tc || wait_iters < gdn::kWaitIters))))
+        return GDN_ERR_UNSUPPORTED;
 
     gdn::Params P;
     std::memset(&P, 0, sizeof(P));
@@ -206,15 +221,26 @@ gdn_status forward_impl(const gdn_dual_desc *desc,
         }
     } else if (algo == GDN_ALGO_CHUNKED || algo == GDN_ALGO_PIPELINED) {
         err = gdn::launch_chunked(P, algo == GDN_ALGO_PIPELINED, st);
-    } else if (algo == GDN_ALGO_ROUTE1 && P.V > 0 && !P.wait_test &&
-               gdn::route1_tc_supported(desc->dtype, desc->d_k, B, desc->conv_width) && desc->d_k == desc->d_v) {
+    } else if (route1_tc && (P.V > 0 || desc->conv_width > 0) && !P.wait_test) {
         // Route I on tensor cores: the clean stream exporting the state before every response
         // block (bf16 blobs of 32 KB, in the space the fp32 states take otherwise), then the refine
-        // kernel over every (block, head, pair of views)
+        // kernel over every (block, head, pair of views).  With ShortConv, the conv pass first
+        // writes the convolved inputs after the states, and both stages read those.
         gdn::Params Q = P;
         Q.states = static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader);
+        err = cudaSuccess;
+        if (desc->conv_width > 0) {
+            uint8_t *buf = static_cast<uint8_t *>(workspace) + sizeof(gdn::WorkspaceHeader) + route1_states;
+            err = gdn::launch_conv_pass(P, buf, st);
+            const int64_t clean = T * H * desc->d_k, nz = (int64_t)P.V * TR * H * desc->d_k;
+            const __nv_bfloat16 *y = reinterpret_cast<const __nv_bfloat16 *>(buf);
+            Q.q = y; Q.k = y + clean; Q.v = y + 2 * clean;
+            Q.qn = y + 3 * clean; Q.kn = y + 3 * clean + nz; Q.vn = y + 3 * clean + 2 * nz;
+            Q.conv_width = 0;
+            Q.conv_w = nullptr;
+        }
         Q.V = 0;
-        err = gdn::launch_chunked(Q, false, st);
+        if (err == cudaSuccess) err = gdn::launch_chunked(Q, false, st);
         if (err == cudaSuccess) {
             cudaMemsetAsync(&static_cast<gdn::WorkspaceHeader *>(workspace)->next_unit, 0, sizeof(int32_t), st);
             Q.V = P.V;

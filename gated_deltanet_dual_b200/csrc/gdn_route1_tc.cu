@@ -475,8 +475,9 @@ cudaError_t launch_refine(const Params &p, cudaStream_t stream) {
 
 }  // namespace
 
+// (ShortConv runs as a pass of its own before both stages, so the kernels never see it)
 bool route1_tc_supported(int dtype, int d, int B, int conv_width) {
-    return dtype == GDN_BF16 && d == RD && (B == 16 || B == 32) && conv_width == 0;
+    return dtype == GDN_BF16 && d == RD && (B == 16 || B == 32) && (conv_width == 0 || conv_width == 4);
 }
 
 size_t route1_tc_state_bytes(int64_t TR, int H, int B) { return (size_t)(TR / B) * H * 32768; }

@@ -77,11 +77,12 @@ typedef enum {
     GDN_ALGO_ROUTE1 = 3,      /* chunk-then-refine (Route I of the notes, Key design 2), a measured
                                  comparison: a clean pass writes the state before every response
                                  block into the workspace, then each (view, block) is refined from
-                                 its stored state.  bf16, d_k = d_v = 128, B in {16, 32}, V >= 1,
-                                 no ShortConv: tensor cores (the chunked kernel exports bf16 states
-                                 from its intra-chunk products, then a tcgen05 refine kernel takes
-                                 two views of a block per item); otherwise CUDA cores (fp32 states).
-                                 No ShortConv; never chosen by AUTO */
+                                 its stored state.  bf16, d_k = d_v = 128, B in {16, 32}: tensor
+                                 cores (the chunked kernel exports bf16 states from its intra-chunk
+                                 products, then a tcgen05 refine kernel takes two views of a block
+                                 per item; ShortConv as a pass of its own into the workspace
+                                 first).  Otherwise CUDA cores (fp32 states), without ShortConv.
+                                 Never chosen by AUTO */
     GDN_ALGO_PIPELINED = 4    /* the chunked WY/UT tcgen05 kernel pipelined across chunks: helper
                                  warps prepare chunk c+1's state-independent products (the
                                  triangular solve among them) while the main warps run chunk c's
@@ -120,10 +121,11 @@ typedef struct CUstream_st *gdn_stream_t;
  * that algorithm prompt_len must be known, so use gdn_dual_workspace_size_route1. */
 size_t gdn_dual_workspace_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host);
 
-/* Workspace bytes for GDN_ALGO_ROUTE1: 256 + (T_R / B) * H * d_k * d_v * 4, where T_R is the total
- * response length (doc_offsets_host [N+1] and prompt_len_host [N] are HOST arrays); the
- * tensor-core form stores its bf16 states in the first half of that.  Returns 0 if the
- * descriptor, offsets or prompt lengths are invalid. */
+/* Workspace bytes for GDN_ALGO_ROUTE1: 256 + (T_R / B) * H * d_k * d_v * 4 (rounded up to 256),
+ * where T_R is the total response length (doc_offsets_host [N+1] and prompt_len_host [N] are HOST
+ * arrays); the tensor-core form stores its bf16 states in the first half of that.  With ShortConv
+ * it adds the convolved inputs, 3 (T + V T_R) H d bf16 elements.  Returns 0 if the descriptor,
+ * offsets or prompt lengths are invalid. */
 size_t gdn_dual_workspace_size_route1(const gdn_dual_desc *desc, const int32_t *doc_offsets_host,
                                       const int32_t *prompt_len_host);
 

@@ -255,6 +255,12 @@ def test_route1_workspace_and_validation():
     assert b.workspace_size_route1(d, offs, pl) == 256 + 6 * 4 * 64 * 64 * 4
     assert b.workspace_size_route1(d, offs, [30, 32]) == 0          # response not a multiple of B
     assert b.select_algo(b.make_desc(2, 4, 64, 64, 2, 16, b.GDN_BF16)) != b.ALGO_ROUTE1
+    # the tensor-core form with ShortConv (bf16, d = 128, B = 16) adds the conv pass's convolved
+    # copies, 3 (T + V T_R) H d bf16 elements; any other ShortConv case adds nothing (unsupported)
+    dt = b.make_desc(2, 4, 128, 128, 2, 16, b.GDN_BF16, conv_width=4, algo=b.ALGO_ROUTE1)
+    assert b.workspace_size_route1(dt, offs, pl) == 256 + 6 * 4 * 128 * 128 * 4 + 3 * (160 + 2 * 96) * 4 * 128 * 2
+    dc = b.make_desc(2, 4, 64, 64, 2, 16, b.GDN_BF16, conv_width=4, algo=b.ALGO_ROUTE1)
+    assert b.workspace_size_route1(dc, offs, pl) == 256 + 6 * 4 * 64 * 64 * 4
 
 
 @no_gpu
@@ -265,6 +271,12 @@ def test_route1_host_validation():
     dc = b.make_desc(2, 2, 32, 32, 2, 4, b.GDN_FP32, conv_width=4, algo=b.ALGO_ROUTE1)
     assert _call(dc, [0, 16, 40], [8, 4], conv_w=_Fake(0x7f0000000000), _ws_bytes=need) == b.GDN_ERR_UNSUPPORTED
     assert _call(d, [0, 16, 40], [8, 4], _ws_bytes=need) == b.GDN_ERR_CUDA              # valid; no device here
+    # the tensor-core form takes ShortConv; its workspace must hold the convolved copies too
+    dt = b.make_desc(2, 2, 128, 128, 2, 16, b.GDN_BF16, conv_width=4, algo=b.ALGO_ROUTE1)
+    offs, pl = [0, 48, 96], [16, 16]
+    need_t = b.workspace_size_route1(dt, offs, pl)
+    assert _call(dt, offs, pl, conv_w=_Fake(0x7f0000000000), _ws_bytes=need_t - 256) == b.GDN_ERR_INVALID_ARG
+    assert _call(dt, offs, pl, conv_w=_Fake(0x7f0000000000), _ws_bytes=need_t) == b.GDN_ERR_CUDA
 
 
 def _attn_call(desc, offs, pl, ws_bytes=None, **over):

@@ -66,10 +66,26 @@ def test_route1_tensor_cores_odd_views_and_prompts(B, V):
     _check(prob, 2e-2)
 
 
-@pytest.mark.parametrize("wl", ["train_8x4096_h16_d128_B16", "train_8x4096_h16_d128_B32"])
+@pytest.mark.parametrize("B", [16, 32])
+@pytest.mark.parametrize("V", [1, 2])
+def test_route1_tensor_cores_shortconv(B, V):
+    """Route I on tensor cores with the width-4 ShortConv (Key design 3 of the FLARE notes): the
+    conv pass writes the convolved inputs into the workspace, then both stages run on them.
+    Prompts of every kind, so that noisy taps before a block start read clean raw inputs and no
+    tap crosses a document start."""
+    lens, prompts = [40 + 4 * B, 2 * B, 96 + 3 * B], [40, 0, 96]
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    prob = synth.make_problem_from_layout(offs, prompts, num_heads=2, d_k=128, d_v=128, block_size=B, num_views=V,
+                                          dtype="bf16", conv_width=4, seed=80 + B + V, device="cuda")
+    _check(prob, 2e-2)
+
+
+@pytest.mark.parametrize("wl", ["train_8x4096_h16_d128_B16", "train_8x4096_h16_d128_B32",
+                                "conv_4x8192_h16_d128_B16", "conv_4x8192_h16_d128_B32"])
 def test_route1_tensor_cores_match_fused_kernel_full_size(wl):
-    """The full training shape: Route I on tensor cores against the fused chunked kernel (both
-    checked against the oracle elsewhere), every output element, within the bf16 bar."""
+    """The full training and ShortConv shapes: Route I on tensor cores against the fused chunked
+    kernel (both checked against the oracle elsewhere), every output element, within the bf16
+    bar."""
     prob = synth.make_problem(wl, device="cuda")
     r1 = b.forward_problem(prob, algo=b.ALGO_ROUTE1)
     r2 = b.forward_problem(prob, algo=b.ALGO_CHUNKED)
