@@ -810,6 +810,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--algo", default="auto", choices=["auto", "sequential", "chunked", "route1", "pipelined"])
+    ap.add_argument("--e2e-groups", type=int, default=8,
+                    help="document groups of the host-buffer call (its copies in and out overlap across groups)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -905,27 +907,27 @@ def main():
                 "algorithmic_bytes_per_launch": work["bytes"], "algorithmic_flops_per_launch": work["flops"],
                 "tensor_frac_at_algorithmic_flops": work["flops"] / (kernel_ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
 
-    # ---- end to end through the public API: pinned host inputs in, outputs back ----
+    # ---- end to end through the public API: pinned host inputs in, outputs back to pinned host
+    #      memory, by gdn_dual_forward_host (document groups pipelined across the host link) ----
     e2e = None
     if not args.no_e2e:
         names = ["q", "k", "v", "g", "beta", "qn", "kn", "vn", "gn", "betan"] + (["conv_w"] if prob.conv_w is not None else [])
         host = {n: getattr(prob, n).cpu().pin_memory() for n in names}
-        dbuf = {n: torch.empty_like(getattr(prob, n)) for n in names}
         h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         h_outn = torch.empty(out_n.shape, dtype=out_n.dtype, pin_memory=True)
         h_fs = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = sum(t.numel() * t.element_size() for t in (h_out, h_outn, h_fs))
+        staging = torch.empty(gb.host_staging_size(desc, prob.doc_offsets, prob.prompt_len, args.e2e_groups),
+                              dtype=torch.uint8, device=dev)
 
         def e2e_step():
-            for n in names:
-                dbuf[n].copy_(host[n], non_blocking=True)
-            gb.forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["qn"], dbuf["kn"], dbuf["vn"],
-                       dbuf["gn"], dbuf["betan"], prob.doc_offsets, prob.prompt_len, prob.block_size,
-                       conv_w=dbuf.get("conv_w"), algo=algo, out=out, out_noisy=out_n, final_state=fs, workspace=ws)
-            h_out.copy_(out, non_blocking=True)
-            h_outn.copy_(out_n, non_blocking=True)
-            h_fs.copy_(fs, non_blocking=True)
+            st = gb.forward_host_raw(desc, host["q"], host["k"], host["v"], host["g"], host["beta"], host["qn"],
+                                     host["kn"], host["vn"], host["gn"], host["betan"], prob.doc_offsets,
+                                     prob.prompt_len, host.get("conv_w"), h_out, h_outn, h_fs, staging,
+                                     args.e2e_groups, stream=stream.cuda_stream)
+            if st != gb.GDN_OK:
+                raise gb.GdnError(st, f"gdn_dual_forward_host failed: {gb.status_string(st)}")
 
         e2e_steps = max(3, min(args.steps, 10))
         for _ in range(3):
@@ -941,8 +943,10 @@ def main():
         barrier()
         e2e_ms = max_over_ranks(a.elapsed_time(z)) / e2e_steps
         e2e = {"value": toks_all / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms, "steps": e2e_steps}
-        del host, dbuf
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "api": "gdn_dual_forward_host", "groups": args.e2e_groups,
+               "host_status": gb.status_string(gb.read_host_device_status(staging, stream.cuda_stream)[0])}
+        del host, staging
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -27,7 +27,8 @@ EXPORTED = ("gdn_dual_forward", "gdn_dual_workspace_size", "gdn_dual_read_device
             "gdn_dual_backward_workspace_size", "gdn_dual_forward_noalloc",
             "gdn_dual_noalloc_read_device_status", "gdn_dual_forward_test_wait_limit",
             "gdn_dual_read_device_status_where", "gdn_attn_forward_test_wait_limit",
-            "gdn_dual_backward_conv", "gdn_dual_backward_conv_workspace_size")
+            "gdn_dual_backward_conv", "gdn_dual_backward_conv_workspace_size",
+            "gdn_dual_forward_host", "gdn_dual_host_staging_size", "gdn_dual_host_read_device_status")
 
 
 class GdnError(RuntimeError):
@@ -96,6 +97,13 @@ def load_library(path: str = LIB_PATH):
             lib.gdn_attn_workspace_size.argtypes = [ad, ip, ip]
             lib.gdn_attn_forward.restype = ctypes.c_int
             lib.gdn_attn_forward.argtypes = [ad, vp, vp, vp, vp, vp, vp, ip, ip, vp, vp, vp, ctypes.c_size_t, vp]
+            lib.gdn_dual_host_staging_size.restype = ctypes.c_size_t
+            lib.gdn_dual_host_staging_size.argtypes = [ctypes.POINTER(Desc), ip, ip, ctypes.c_int32]
+            lib.gdn_dual_forward_host.restype = ctypes.c_int
+            lib.gdn_dual_forward_host.argtypes = ([ctypes.POINTER(Desc)] + [vp] * 10 + [ip, ip, vp, vp, vp, vp, vp,
+                                                  ctypes.c_size_t, ctypes.c_int32, vp])
+            lib.gdn_dual_host_read_device_status.restype = ctypes.c_int
+            lib.gdn_dual_host_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
             _lib = lib
     return _lib
 
@@ -277,6 +285,41 @@ def read_device_status(workspace: Workspace, stream=None) -> int:
     if stream is None:
         stream = torch.cuda.current_stream().cuda_stream
     return int(load_library().gdn_dual_read_device_status(_ptr(workspace.tensor), ctypes.c_void_p(stream)))
+
+
+def host_staging_size(desc: Desc, doc_offsets, prompt_len, groups: int) -> int:
+    """Device staging bytes gdn_dual_forward_host needs (0: invalid descriptor or layout)."""
+    offs, pl = _host_i32(doc_offsets), _host_i32(prompt_len)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    return int(load_library().gdn_dual_host_staging_size(ctypes.byref(desc), offs.ctypes.data_as(ip),
+                                                         pl.ctypes.data_as(ip), int(groups)))
+
+
+def forward_host_raw(desc: Desc, q, k, v, g, beta, qn, kn, vn, gn, betan, doc_offsets, prompt_len, conv_w,
+                     out, out_noisy, final_state, staging: torch.Tensor, groups: int, stream=None) -> int:
+    """C-ABI call of gdn_dual_forward_host: every tensor argument is a (pinned) CPU tensor, `staging`
+    a CUDA byte tensor of host_staging_size() bytes.  Returns the status code; the outputs are in
+    host memory once `stream` is synchronised."""
+    lib = load_library()
+    offs, pl = _host_i32(doc_offsets), _host_i32(prompt_len)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return int(lib.gdn_dual_forward_host(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                         _ptr(qn), _ptr(kn), _ptr(vn), _ptr(gn), _ptr(betan),
+                                         offs.ctypes.data_as(ip), pl.ctypes.data_as(ip), _ptr(conv_w),
+                                         _ptr(out), _ptr(out_noisy), _ptr(final_state), _ptr(staging),
+                                         ctypes.c_size_t(staging.numel()), int(groups), ctypes.c_void_p(stream)))
+
+
+def read_host_device_status(staging: torch.Tensor, stream=None):
+    """(status, where) recorded by the groups of the last gdn_dual_forward_host on `staging`."""
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    where = ctypes.c_int32(0)
+    st = int(load_library().gdn_dual_host_read_device_status(_ptr(staging), ctypes.byref(where),
+                                                             ctypes.c_void_p(stream)))
+    return st, int(where.value)
 
 
 def forward_problem(prob, **kw):

@@ -251,6 +251,42 @@ gdn_status gdn_dual_forward_noalloc(const gdn_dual_desc *desc,
  * the library's fixed scratch array.  No allocation.  (The FLARE notes have no counterpart.) */
 gdn_status gdn_dual_noalloc_read_device_status(gdn_stream_t stream);
 
+/*
+ * gdn_dual_forward from and to HOST buffers (same descriptor, layouts and results as
+ * gdn_dual_forward; every tensor argument is a host pointer, pinned for the copies to run
+ * asynchronously).  The documents are cut into `groups` contiguous groups of about equal token
+ * counts (at most min(groups, N, 64)); each group's inputs are copied into one of two device
+ * buffers inside `staging`, the group's forward runs on `stream`, and its outputs are copied
+ * back, on two streams of the call's own, so that one group's outputs travel to the host while the
+ * next group's inputs travel to the device.  Stream-ordered: it starts after the work already on
+ * `stream`, and `stream` reaches the outputs in host memory only after every copy has landed
+ * (synchronise `stream` before reading them).  Not capturable in a CUDA graph (it creates its two
+ * copy streams and destroys them when the work is done).
+ *   staging        DEVICE memory of at least gdn_dual_host_staging_size() bytes, 256-byte aligned.
+ *   Errors: the whole problem is validated on the host as gdn_dual_forward validates it before
+ *   anything is enqueued; GDN_ERR_INVALID_ARG also for groups < 1 or a staging area that is too
+ *   small; GDN_ERR_CUDA if a copy or launch fails (work already enqueued then still runs).
+ * Device-side status: gdn_dual_host_read_device_status.  (The FLARE notes have no counterpart:
+ * this is the library's host interface.) */
+size_t gdn_dual_host_staging_size(const gdn_dual_desc *desc, const int32_t *doc_offsets_host,
+                                  const int32_t *prompt_len_host, int32_t groups);
+
+gdn_status gdn_dual_forward_host(const gdn_dual_desc *desc,
+                                 const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 const void *qn, const void *kn, const void *vn,
+                                 const float *gn, const float *betan,
+                                 const int32_t *doc_offsets, const int32_t *prompt_len,
+                                 const float *conv_w,
+                                 void *out, void *out_noisy, float *final_state,
+                                 void *staging, size_t staging_bytes, int32_t groups,
+                                 gdn_stream_t stream);
+
+/* Synchronises `stream` and returns the first non-OK device-side status that the groups of the
+ * last gdn_dual_forward_host on `staging` recorded (GDN_OK or GDN_ERR_TIMEOUT), storing the
+ * diagnostic code of the wait that gave up in `where` when it is not NULL. */
+gdn_status gdn_dual_host_read_device_status(const void *staging, int32_t *where, gdn_stream_t stream);
+
 /* Synchronises `stream` and returns the device-side status recorded in `workspace` by the
  * last gdn_dual_forward on it (GDN_OK or GDN_ERR_TIMEOUT), or GDN_ERR_CUDA if the sync fails.
  * For debugging and tests; the forward path itself never synchronises. */

@@ -279,6 +279,45 @@ def test_route1_host_validation():
     assert _call(dt, offs, pl, conv_w=_Fake(0x7f0000000000), _ws_bytes=need_t) == b.GDN_ERR_CUDA
 
 
+@no_gpu
+def test_host_forward_validation():
+    """gdn_dual_forward_host rejects bad arguments on the host before anything is enqueued; a
+    valid call reaches the CUDA runtime (which fails here: no device)."""
+    d = b.make_desc(3, 2, 64, 64, 2, 4, b.GDN_BF16)
+    offs, pl = [0, 40, 40, 104], [8, 0, 32]
+    need = b.host_staging_size(d, offs, pl, 2)
+    assert need > 0 and need % 256 == 0
+    assert b.host_staging_size(d, offs, pl, 0) == 0                     # groups < 1
+    assert b.host_staging_size(d, [0, 40, 40, 103], pl, 2) == 0         # response not a multiple of B
+    assert b.host_staging_size(d, offs, pl, 64) >= b.host_staging_size(d, offs, pl, 1) // 4
+    lib = b.load_library()
+    ip = ctypes.POINTER(ctypes.c_int32)
+
+    def call(desc, offs, pl, groups, staging, nbytes, **over):
+        base = 0x7f0000000000
+        names = ["q", "k", "v", "g", "beta", "qn", "kn", "vn", "gn", "betan", "conv_w", "out", "out_noisy",
+                 "final_state"]
+        ptr = {n: ctypes.c_void_p(base + 0x10000000 * i) for i, n in enumerate(names)}
+        ptr["conv_w"] = None
+        ptr.update(over)
+        o = np.ascontiguousarray(offs, dtype=np.int32)
+        p = np.ascontiguousarray(pl, dtype=np.int32)
+        return lib.gdn_dual_forward_host(ctypes.byref(desc), *[ptr[n] for n in names[:10]], o.ctypes.data_as(ip),
+                                         p.ctypes.data_as(ip), ptr["conv_w"], ptr["out"], ptr["out_noisy"],
+                                         ptr["final_state"], ctypes.c_void_p(staging), ctypes.c_size_t(nbytes),
+                                         groups, None)
+
+    stg = 0x7e0000000000
+    assert call(d, offs, pl, 0, stg, need) == b.GDN_ERR_INVALID_ARG               # groups < 1
+    assert call(d, offs, pl, 2, stg, need - 256) == b.GDN_ERR_INVALID_ARG         # staging too small
+    assert call(d, offs, pl, 2, stg + 16, need) == b.GDN_ERR_INVALID_ARG          # staging not 256-aligned
+    assert call(d, offs, pl, 2, 0, need) == b.GDN_ERR_INVALID_ARG                 # no staging
+    assert call(d, offs, pl, 2, stg, need, q=None) == b.GDN_ERR_INVALID_ARG       # missing input
+    bad = b.make_desc(3, 2, 48, 48, 2, 4, b.GDN_BF16)                              # d = 48: unsupported
+    assert call(bad, offs, pl, 2, stg, b.host_staging_size(bad, offs, pl, 2)) == b.GDN_ERR_UNSUPPORTED
+    assert call(d, offs, pl, 2, stg, need) == b.GDN_ERR_CUDA                      # valid; no device here
+
+
 def _attn_call(desc, offs, pl, ws_bytes=None, **over):
     base = 0x7f0000000000
     names = ["q", "k", "v", "qn", "kn", "vn", "out", "out_noisy", "ws"]
