@@ -791,13 +791,20 @@ def run_backward(args, name, rank, world, local):
     replicas.shutdown(world)
     if rank != 0:
         return
+    # kernels of one backward call: the backward kernel and four slice reductions per stream (dq,
+    # dk, dg, dbeta); with ShortConv also the conv forward, the bf16 upstream-gradient casts (one
+    # per stream), the conv backward and the weight gradient
+    noisy_bwd = prob.num_views > 0 and prob.T_R > 0
+    bwd_launches = 1 + 4 + (4 if noisy_bwd else 0)
+    if prob.conv_width:
+        bwd_launches += 1 + ((1 + (1 if noisy_bwd else 0)) if prob.q.dtype == torch.bfloat16 else 0) + 2
     line = {"metric": BWD_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 I/O, fp32 arithmetic and gradients", "data": "synthetic",
             "config": {"workload": name, "layout": BWD_WORKLOADS[name], "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2"},
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
-            "gpu_launches": steps, "clocks": clocks.summary()}
+            "gpu_launches": bwd_launches * steps, "launches_per_step": bwd_launches, "clocks": clocks.summary()}
     print(json.dumps(line), flush=True)
 
 
@@ -895,9 +902,18 @@ def main():
                  and gb.workspace_size(desc, prob.doc_offsets) > 256)
     # Route I on tensor cores (bf16, d = 128, B in {16, 32}; ShortConv as a pass of its own first)
     r1_tc = (used_algo == gb.ALGO_ROUTE1 and prob.q.dtype == torch.bfloat16 and d == 128
-             and prob.block_size in (16, 32) and (V > 0 or prob.conv_width == 4))
+             and prob.block_size in (16, 32))
     if r1_tc:
         traffic = profiled_traffic("route1_tc", wl.name, work["bytes"])
+    # kernels one forward call launches: the chunked kernel once per pair of views (each launch
+    # recomputes the clean stream), plus the ShortConv pass; Route I two stages (plus the conv pass)
+    v_eff = V if TR > 0 else 0
+    if used_algo in (gb.ALGO_CHUNKED, gb.ALGO_PIPELINED):
+        launches = max(1, (v_eff + 1) // 2) + (1 if conv_pass else 0)
+    elif used_algo == gb.ALGO_ROUTE1:
+        launches = 1 + (1 if v_eff > 0 else 0) + (1 if r1_tc and prob.conv_width == 4 else 0)
+    else:
+        launches = 1
     kname = ("conv_pass_kernel + " + KERNEL_NAMES[used_algo] + " (one forward call)") if conv_pass \
         else ("conv_pass_kernel + " if prob.conv_width == 4 else "") + KERNEL_NAMES["route1_tc"] if r1_tc \
         else KERNEL_NAMES.get(used_algo)
@@ -966,7 +982,7 @@ def main():
                        "algo": {1: "sequential", 2: "chunked", 3: "route1", 4: "pipelined"}.get(used_algo, str(used_algo)),
                        "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush)"},
             "roofline": roofline, "cpu_baseline": cpu_baseline, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clocks.summary(),
+            "gpu_launches": launches * args.steps, "launches_per_step": launches, "clocks": clocks.summary(),
             "device_status": gb.status_string(dstatus), "kernel_ms_mean": kernel_ms}
     print(json.dumps(line), flush=True)
 
