@@ -764,12 +764,6 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             auto blob = [&](int b) {
                 return static_cast<uint8_t *>(P.states) + ((int64_t)(U.roff / B + b) * H + U.h) * 32768;
             };
-            if constexpr (EXPORT) {
-                if (tid == 0 && exporting && eb0 < enb && !dead) {   // the first block starts from S0
-                    bulk_store(blob(eb0), sm + OFF_S0, 32768);
-                    bulk_commit();
-                }
-            }
 
             // ================= PK1: [Q;K]K^T now, the noisy products once group B is in ========
             if (tid == 0) {
@@ -783,6 +777,14 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                 // barrier completes: those tiles are next written after it
                 bulk_wait_read_all();
                 commit_mma();
+                if constexpr (EXPORT) {
+                    // the first block starts from S0 (stored after the wait above, so that the
+                    // products need not wait for it; S0 is rewritten only after S3)
+                    if (exporting && eb0 < enb && !dead) {
+                        bulk_store(blob(eb0), sm + OFF_S0, 32768);
+                        bulk_commit();
+                    }
+                }
             }
             __syncwarp();
             // Khat = diag(e^{gamma_C - gamma_t}) K  (MN-major A tile, same swizzled layout), built by
@@ -1083,10 +1085,12 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
             // ================= S3 =================
             if (tid == 0) {
                 tc_fence_after();
+                bool o_stored = false;
                 if (o_tma && !dead && GDN_IN_RANGE(P.ws, cstart >= 0 && cstart + CH <= P.T, 206)) {
                     tma_store_3d(&M.o, sm + OFF_Y, 0, U.h, cstart);
                     tma_store_3d(&M.o, sm + OFF_Y + 8192, 64, U.h, cstart);
                     bulk_commit();
+                    o_stored = true;
                 }
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16(tb + TM_R0, dM_kh + ((kk * 2048) >> 4), dM_v + ((kk * 2048) >> 4),
@@ -1106,7 +1110,10 @@ gdn_chunked_kernel(const __grid_constant__ Params P, const __grid_constant__ Map
                                          make_idesc_bf16(128, 128, 1, 1), kk > 0);
                         }
                     }
-                    bulk_wait_read_all();    // the S0 blob has been read before the update rewrites S0
+                    // the S0 blob has been read before the update rewrites S0; the output tile's store,
+                    // the newest bulk group when issued just above, may still be reading
+                    if (o_stored) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                    else bulk_wait_read_all();
                 }
                 commit_mma();
                 if (!last && !dead) {
