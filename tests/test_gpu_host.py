@@ -85,6 +85,14 @@ def test_host_forward_route1(conv):
     _same(prob, b.ALGO_ROUTE1, 2)
 
 
+def test_host_forward_eight_views():
+    """Eight views: the chunked path runs one launch per pair of views inside every group."""
+    offs = np.concatenate([[0], np.cumsum(LENS)]).astype(np.int32)
+    prob = synth.make_problem_from_layout(offs, PROMPTS, num_heads=2, d_k=128, d_v=128, block_size=4, num_views=8,
+                                          dtype="bf16", seed=140, device="cuda")
+    _same(prob, b.ALGO_AUTO, 3)
+
+
 def test_host_forward_full_training_shape():
     """The training shape through the host path in eight groups, bit-identical to the device call."""
     prob = synth.make_problem("train_8x4096_h16_d128", device="cuda")

@@ -53,11 +53,11 @@ def test_route1_long_document_tiles():
 
 
 @pytest.mark.parametrize("B", [16, 32])
-@pytest.mark.parametrize("V", [1, 3])
+@pytest.mark.parametrize("V", [1, 3, 8])
 def test_route1_tensor_cores_odd_views_and_prompts(B, V):
     """bf16, d = 128, B = 16 / 32: Route I on tensor cores (the chunked kernel exporting the state
     before every response block, then the refine kernel by pairs of views; V odd leaves a pair with
-    one view).  Prompts that are not whole chunks, an empty response, and few units (split over two
+    one view, V = 8 gives four pairs per block).  Prompts that are not whole chunks, an empty response, and few units (split over two
     CTAs)."""
     lens, prompts = [40 + 4 * B, 96 + 6 * B, 72, 3 * B], [40, 96, 72, 0]
     offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
