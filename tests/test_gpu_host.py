@@ -93,6 +93,20 @@ def test_host_forward_eight_views():
     _same(prob, b.ALGO_AUTO, 3)
 
 
+def test_host_forward_empty_documents_and_more_groups_than_documents():
+    """Degenerate layouts: every document empty (only the zero final states come back), and more
+    groups asked for than there are documents (one document per group)."""
+    offs = np.zeros(4, np.int32)
+    prob = synth.make_problem_from_layout(offs, [0, 0, 0], num_heads=2, d_k=128, d_v=128, block_size=4,
+                                          num_views=2, dtype="bf16", seed=150, device="cuda")
+    out, outn, fs = _same(prob, b.ALGO_AUTO, 5)
+    assert torch.count_nonzero(fs) == 0
+    offs = np.concatenate([[0], np.cumsum([64, 0, 96])]).astype(np.int32)
+    prob = synth.make_problem_from_layout(offs, [32, 0, 0], num_heads=2, d_k=128, d_v=128, block_size=8,
+                                          num_views=1, dtype="bf16", seed=151, device="cuda")
+    _same(prob, b.ALGO_AUTO, 64)
+
+
 def test_host_forward_full_training_shape():
     """The training shape through the host path in eight groups, bit-identical to the device call."""
     prob = synth.make_problem("train_8x4096_h16_d128", device="cuda")
